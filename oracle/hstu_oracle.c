@@ -1,0 +1,257 @@
+/*
+ * hstu_oracle.c -- plain fp64 CPU oracle for the HSTU layer forward.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing here is part of the product path: only
+ * the tests, the package smoke check and the benchmark's CPU-baseline leg may
+ * load this library. It shares no code, header, table or constant with the
+ * CUDA implementation.
+ *
+ * What it computes (HSTU, "Actions Speak Louder than Words: Trillion-Parameter
+ * Sequential Transducers for Generative Recommendations", arXiv 2402.17152;
+ * the abstract names HSTU, the generative-recommenders README section
+ * "HSTU Ultra attention benchmark" names the layer order: UVQK projection,
+ * attention, output normalization and projection, residual connection):
+ *
+ *   for every sequence b (tokens o_b .. o_{b+1}-1), head h, position i:
+ *     A[o_b+i,h,:] = (1/N) * sum_{j<=i} silu(s_ij) * v[o_b+j,h,:]
+ *     s_ij = <q[o_b+i,h,:], k[o_b+j,h,:]>
+ *          + pos[h][min(i-j, P-1)]
+ *          + time[h][clamp(floor_log2(max(1, ts[o_b+i]-ts[o_b+j])), 0, NB-1)]
+ *
+ * N is the caller's max_seqlen. Layer: UVQK = silu(x W1^T + b1) split as
+ * U|V|Q|K, attention as above, Y = LayerNorm(A) * U over the H*d features of a
+ * token, out = x + Y W2^T + b2.
+ *
+ * Everything is evaluated in double precision, one output row at a time, in
+ * the order of the definition. No blocking, no fusion, no reordering.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* floor(log2(x)) for x >= 1 by counting halvings: integer arithmetic only,
+ * so int64 differences above 2^53 are still exact. */
+int32_t hstu_oracle_floor_log2(int64_t x) {
+    int32_t r = 0;
+    while (x > 1) {
+        x >>= 1;
+        r += 1;
+    }
+    return r;
+}
+
+/* Log-time bucket of a timestamp difference: clamp(floor(log2(max(1, dt))), 0, NB-1). */
+int32_t hstu_oracle_time_bucket(int64_t dt, int32_t num_buckets) {
+    int64_t x = dt < 1 ? 1 : dt;
+    int32_t bkt = hstu_oracle_floor_log2(x);
+    if (bkt < 0) bkt = 0;
+    if (bkt > num_buckets - 1) bkt = num_buckets - 1;
+    return bkt;
+}
+
+/* Relative-position index: min(i - j, P - 1) for j <= i. */
+int32_t hstu_oracle_pos_index(int64_t i, int64_t j, int32_t num_pos) {
+    int64_t r = i - j;
+    if (r > num_pos - 1) r = num_pos - 1;
+    return (int32_t)r;
+}
+
+double hstu_oracle_silu(double x) { return x / (1.0 + exp(-x)); }
+
+/* For every sequence, every i, every j <= i (row-major in i, then j), write the
+ * relative-position index and the time bucket. Arrays hold sum_b n_b(n_b+1)/2
+ * entries. pos_idx or bucket may be NULL. */
+void hstu_oracle_bias_indices(const int64_t* seq_offsets, int32_t B, const int64_t* ts,
+                              int32_t num_pos, int32_t num_buckets,
+                              int32_t* pos_idx, int32_t* bucket) {
+    int64_t e = 0;
+    for (int32_t b = 0; b < B; ++b) {
+        int64_t o = seq_offsets[b], n = seq_offsets[b + 1] - seq_offsets[b];
+        for (int64_t i = 0; i < n; ++i) {
+            for (int64_t j = 0; j <= i; ++j) {
+                if (pos_idx) pos_idx[e] = hstu_oracle_pos_index(i, j, num_pos);
+                if (bucket) bucket[e] = hstu_oracle_time_bucket(ts[o + i] - ts[o + j], num_buckets);
+                ++e;
+            }
+        }
+    }
+}
+
+/* Sequence that holds token t (seq_offsets is non-decreasing). */
+static int32_t seq_of_token(const int64_t* seq_offsets, int32_t B, int64_t t) {
+    for (int32_t b = 0; b < B; ++b)
+        if (t >= seq_offsets[b] && t < seq_offsets[b + 1]) return b;
+    return -1;
+}
+
+/* One output row (token t, all heads) of the attention. q,k,v are addressed with
+ * explicit token strides so the layer can pass its U|V|Q|K buffer. */
+static void attn_row(int64_t t, int32_t b, const int64_t* seq_offsets, int32_t H,
+                     int32_t dqk, int32_t dv,
+                     const double* q, int64_t q_tok, const double* k, int64_t k_tok,
+                     const double* v, int64_t v_tok, const int64_t* ts,
+                     const double* pos, int32_t num_pos, const double* tbias,
+                     int32_t num_buckets, int32_t max_seqlen, double* out_row) {
+    int64_t o = seq_offsets[b];
+    int64_t i = t - o;
+    for (int32_t h = 0; h < H; ++h) {
+        double* a = out_row + (int64_t)h * dv;
+        for (int32_t c = 0; c < dv; ++c) a[c] = 0.0;
+        const double* qi = q + t * q_tok + (int64_t)h * dqk;
+        for (int64_t j = 0; j <= i; ++j) {
+            const double* kj = k + (o + j) * k_tok + (int64_t)h * dqk;
+            const double* vj = v + (o + j) * v_tok + (int64_t)h * dv;
+            double s = 0.0;
+            for (int32_t c = 0; c < dqk; ++c) s += qi[c] * kj[c];
+            if (pos) s += pos[(int64_t)h * num_pos + hstu_oracle_pos_index(i, j, num_pos)];
+            if (ts && tbias)
+                s += tbias[(int64_t)h * num_buckets +
+                           hstu_oracle_time_bucket(ts[o + i] - ts[o + j], num_buckets)];
+            double p = hstu_oracle_silu(s);
+            for (int32_t c = 0; c < dv; ++c) a[c] += p * vj[c];
+        }
+        for (int32_t c = 0; c < dv; ++c) a[c] /= (double)max_seqlen;
+    }
+}
+
+/* Attention forward. q,k: [T,H,dqk]; v: [T,H,dv] (token strides given in
+ * elements). rows == NULL: out is [T,H,dv]. Otherwise out is [n_rows,H,dv] and
+ * holds the requested tokens only. pos / ts / tbias may be NULL (term absent).
+ * Returns 0, or -1 if a requested row is outside every sequence. */
+int hstu_oracle_attn(const int64_t* seq_offsets, int32_t B, int32_t H, int32_t dqk, int32_t dv,
+                     const double* q, int64_t q_tok, const double* k, int64_t k_tok,
+                     const double* v, int64_t v_tok, const int64_t* ts,
+                     const double* pos, int32_t num_pos, const double* tbias,
+                     int32_t num_buckets, int32_t max_seqlen,
+                     const int64_t* rows, int64_t n_rows, double* out) {
+    int64_t T = seq_offsets[B];
+    int64_t n = rows ? n_rows : T;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 4) reduction(|:bad)
+    for (int64_t r = 0; r < n; ++r) {
+        int64_t t = rows ? rows[r] : r;
+        int32_t b = seq_of_token(seq_offsets, B, t);
+        if (b < 0) { bad = 1; continue; }
+        attn_row(t, b, seq_offsets, H, dqk, dv, q, q_tok, k, k_tok, v, v_tok, ts, pos,
+                 num_pos, tbias, num_buckets, max_seqlen, out + r * (int64_t)H * dv);
+    }
+    return bad ? -1 : 0;
+}
+
+/* y[m, :] = act(x[m, :] W^T + bias) + residual[m, :]; x [M,K], W [N,K].
+ * act = 1 applies SiLU. bias / residual may be NULL. */
+void hstu_oracle_linear(int64_t M, int32_t K, int32_t N, const double* x, const double* W,
+                        const double* bias, int32_t act_silu, const double* residual,
+                        double* y) {
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int32_t n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int32_t c = 0; c < K; ++c) acc += x[m * K + c] * W[(int64_t)n * K + c];
+            if (bias) acc += bias[n];
+            if (act_silu) acc = hstu_oracle_silu(acc);
+            if (residual) acc += residual[m * N + n];
+            y[m * N + n] = acc;
+        }
+    }
+}
+
+/* y[m, :] = LayerNorm(a[m, :]) * u[m, :] over F features: biased variance,
+ * eps inside the square root, then gamma / beta (NULL = 1 / 0).
+ * a, u, y have row strides a_ld, u_ld, F. */
+void hstu_oracle_layernorm_gate(int64_t M, int32_t F, const double* a, int64_t a_ld,
+                                const double* u, int64_t u_ld, const double* gamma,
+                                const double* beta, double eps, double* y) {
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        const double* ar = a + m * a_ld;
+        double mean = 0.0;
+        for (int32_t c = 0; c < F; ++c) mean += ar[c];
+        mean /= (double)F;
+        double var = 0.0;
+        for (int32_t c = 0; c < F; ++c) var += (ar[c] - mean) * (ar[c] - mean);
+        var /= (double)F;
+        double rstd = 1.0 / sqrt(var + eps);
+        for (int32_t c = 0; c < F; ++c) {
+            double g = gamma ? gamma[c] : 1.0;
+            double bt = beta ? beta[c] : 0.0;
+            y[m * F + c] = ((ar[c] - mean) * rstd * g + bt) * u[m * u_ld + c];
+        }
+    }
+}
+
+/* Full layer forward for the requested rows (rows == NULL: every token).
+ * x [T,D], W1 [4Hd,D] (output columns U|V|Q|K), W2 [D,Hd]; out [n,D].
+ * Only the prefix of each touched sequence up to its last requested row is
+ * projected, since later tokens cannot reach a requested row.
+ * Returns 0, -1 for a bad row, -2 on allocation failure. */
+int hstu_oracle_layer(int64_t T, int32_t D, const double* x, const double* W1,
+                      const double* b1, const double* W2, const double* b2,
+                      const double* gamma, const double* beta, double eps,
+                      const int64_t* seq_offsets, int32_t B, int32_t H, int32_t d,
+                      const int64_t* ts, const double* pos, int32_t num_pos,
+                      const double* tbias, int32_t num_buckets, int32_t max_seqlen,
+                      const int64_t* rows, int64_t n_rows, double* out) {
+    int64_t n = rows ? n_rows : T;
+    int64_t F = (int64_t)H * d, W = 4 * F;
+    int64_t* upto = (int64_t*)malloc(sizeof(int64_t) * (B > 0 ? B : 1));
+    double* uvqk = (double*)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1) * (size_t)W);
+    double* attn = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1) * (size_t)F);
+    double* ygate = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1) * (size_t)F);
+    double* urow = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1) * (size_t)F);
+    double* xrow = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1) * (size_t)D);
+    int rc = 0;
+    if (!upto || !uvqk || !attn || !ygate || !urow || !xrow) { rc = -2; goto done; }
+    for (int32_t b = 0; b < B; ++b) upto[b] = seq_offsets[b];  /* exclusive end */
+    for (int64_t r = 0; r < n; ++r) {
+        int64_t t = rows ? rows[r] : r;
+        int32_t b = seq_of_token(seq_offsets, B, t);
+        if (b < 0) { rc = -1; goto done; }
+        if (t + 1 > upto[b]) upto[b] = t + 1;
+    }
+    /* 1. UVQK = silu(x W1^T + b1) for each needed prefix */
+    for (int32_t b = 0; b < B; ++b) {
+        int64_t o = seq_offsets[b], m = upto[b] - o;
+        if (m > 0)
+            hstu_oracle_linear(m, D, (int32_t)W, x + o * D, W1, b1, 1, NULL, uvqk + o * W);
+    }
+    /* 2. attention with U|V|Q|K views of the projection (token stride 4Hd) */
+    rc = hstu_oracle_attn(seq_offsets, B, H, d, d, uvqk + 2 * F, W, uvqk + 3 * F, W,
+                          uvqk + F, W, ts, pos, num_pos, tbias, num_buckets, max_seqlen,
+                          rows ? rows : NULL, n, attn);
+    if (rc) goto done;
+    /* 3. Y = LayerNorm(A) * U */
+    for (int64_t r = 0; r < n; ++r) {
+        int64_t t = rows ? rows[r] : r;
+        memcpy(urow + r * F, uvqk + t * W, sizeof(double) * (size_t)F);
+    }
+    hstu_oracle_layernorm_gate(n, (int32_t)F, attn, F, urow, F, gamma, beta, eps, ygate);
+    /* 4. out = x + Y W2^T + b2 */
+    for (int64_t r = 0; r < n; ++r) {
+        int64_t t = rows ? rows[r] : r;
+        memcpy(xrow + r * D, x + t * D, sizeof(double) * (size_t)D);
+    }
+    hstu_oracle_linear(n, (int32_t)F, D, ygate, W2, b2, 0, xrow, out);
+done:
+    free(upto); free(uvqk); free(attn); free(ygate); free(urow); free(xrow);
+    return rc;
+}
+
+/* Threads an OpenMP parallel region actually uses (1 without OpenMP). */
+int hstu_oracle_num_threads(void) {
+    int nt = 1;
+#pragma omp parallel
+    {
+#pragma omp single
+        {
+#ifdef _OPENMP
+            nt = omp_get_num_threads();
+#endif
+        }
+    }
+    return nt;
+}
