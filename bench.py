@@ -1,0 +1,554 @@
+#!/usr/bin/env python
+"""Benchmark of the HSTU jagged causal attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 4] [--impl ours|reference]
+
+One step is one full pass of the hot path over one seeded synthetic batch:
+the work-list plan kernel plus the attention kernel (for --config 5, the
+whole HSTU layer: UVQK projection, plan, attention, LayerNorm gate, output
+projection). Inputs are resident in HBM before the timed region; the timed
+region is bracketed by a barrier and a device synchronisation on both sides
+and measured with CUDA events on the launching stream (max over ranks).
+
+Default workload: the 8192-length regime (16 sequences, lengths 8192*Beta(2,1),
+4 heads, d = 128), whose inputs (~0.3 GB) exceed the 126 MB L2, so no flush is
+needed between steps. Short workloads (--config 2/3) rotate over enough input
+copies to exceed 2x L2.
+
+For N > 1 (torchrun), every rank runs its own independently seeded batch of the
+same shape (weak scaling); there is no collective in the data path, only the
+timing reductions. Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle (the only reference this project
+has) on the host cores, on a bounded sample of the same workload per step.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "HSTU jagged attn fwd TFLOP/s (causal) & % of B200 BF16 peak; tokens/s"
+L2_BYTES = 126 * 2 ** 20
+NOMINAL_BF16_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PROFILE_DIR = os.path.join(ROOT, "profiles")
+ATTN_SRC = os.path.join(ROOT, "jagged_pointwise_attention_b200", "csrc", "attn_tc.cuh")
+
+
+# ----------------------------------------------------------------------------- accounting
+
+def causal_flops(lengths, H, dqk, dv) -> int:
+    """sum_b H (dqk + dv) n_b (n_b + 1): QK^T and PV over the causal lower
+    triangle including the diagonal, 2 flops per multiply-add."""
+    n = np.asarray(lengths, dtype=np.int64)
+    return int((H * (dqk + dv) * n * (n + 1)).sum())
+
+
+def row_causal_flops(pos_in_seq, H, dqk, dv) -> int:
+    """Causal flops of individual query rows (0-based position i: i+1 keys)."""
+    i = np.asarray(pos_in_seq, dtype=np.int64)
+    return int((2 * H * (dqk + dv) * (i + 1)).sum())
+
+
+def attn_bytes(T, B, H, dqk, dv, P, NB, elem=2) -> int:
+    """Algorithmic bytes of one attention pass: q, k, v read once, out written
+    once, timestamps, offsets and both bias tables read once."""
+    return T * H * (2 * dqk + dv) * elem + T * H * dv * elem + 8 * T + 8 * (B + 1) + 4 * H * (P + NB)
+
+
+def layer_flops(T, D, H, d) -> int:
+    return 2 * T * D * 4 * H * d + 2 * T * H * d * D
+
+
+# ----------------------------------------------------------------------------- env
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def reduce_timing(local_ms: float, local_units: float, world: int, device=None):
+    """(max elapsed ms over ranks, sum of work units over ranks)."""
+    if world == 1:
+        return local_ms, local_units
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([local_ms], dtype=torch.float64, device=device)
+    u = torch.tensor([local_units], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(u.item())
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML while running."""
+
+    REASONS = [(0x1, "gpu_idle"), (0x2, "applications_clocks_setting"), (0x4, "sw_power_cap"),
+               (0x8, "hw_slowdown"), (0x10, "sync_boost"), (0x20, "sw_thermal_slowdown"),
+               (0x40, "hw_thermal_slowdown"), (0x80, "hw_power_brake_slowdown"),
+               (0x100, "display_clock_setting")]
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thr = None
+        self.handle = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.handle = self._handle(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        except Exception as e:   # clocks are reported as unavailable, never faked
+            self.error = str(e)
+
+    def _handle(self, device_index):
+        import torch
+        pynvml = self.nv
+        try:
+            p = torch.cuda.get_device_properties(device_index)
+            bus = "%08x:%02x:%02x.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+            return pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(device_index)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM))
+                try:
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                except AttributeError:
+                    r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.handle)
+                self.reasons |= int(r)
+            except Exception:
+                pass
+            self._stop.wait(self.period)
+
+    def start(self):
+        if self.handle is not None:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+
+    def stop(self):
+        if self._thr is not None:
+            self._stop.set()
+            self._thr.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"],
+                    "samples": 0}
+        names = [n for bit, n in self.REASONS if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+def source_digest(path: str) -> str:
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profiled_traffic(kernel_tag: str):
+    """DRAM bytes per launch from the committed ncu summary of this kernel and
+    workload, if it was taken on the current kernel source; else None."""
+    path = os.path.join(PROFILE_DIR, kernel_tag + ".md")
+    try:
+        txt = open(path).read()
+    except OSError:
+        return None
+    m_b = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    m_h = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", txt)
+    if not m_b or not m_h or m_h.group(1) != source_digest(ATTN_SRC):
+        return None
+    return float(m_b.group(1))
+
+
+# ----------------------------------------------------------------------------- oracle leg
+
+def oracle_sample_rate(inp, budget_s: float, seed: int = 0):
+    """Time the fp64 oracle on a random sample of query rows of ``inp`` sized to
+    about ``budget_s`` seconds. Returns (TFLOP/s, rows, seconds, threads)."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    off = inp.seq_offsets
+    T = inp.T
+    seq_of = np.repeat(np.arange(inp.B), np.diff(off))
+    pos = np.arange(T) - off[seq_of]
+    H, dqk, dv = inp.H, inp.q.shape[2], inp.v.shape[2]
+
+    def run(rows):
+        t0 = time.perf_counter()
+        oracle.attn(off, inp.q, inp.k, inp.v, inp.timestamps, inp.pos_bias, inp.time_bias,
+                    inp.max_seqlen, rows=rows)
+        return time.perf_counter() - t0
+
+    order = rng.permutation(T)
+    probe = np.sort(order[:16])
+    dt = max(run(probe), 1e-4)
+    rate = row_causal_flops(pos[probe], H, dqk, dv) / dt          # flops / s
+    target = rate * budget_s
+    cum = np.cumsum(2 * H * (dqk + dv) * (pos[order] + 1))
+    nrows = int(np.clip(np.searchsorted(cum, target) + 1, 16, T))
+    rows = np.sort(order[:nrows])
+    dt = run(rows)
+    fl = row_causal_flops(pos[rows], H, dqk, dv)
+    return fl / dt / 1e12, nrows, dt, oracle.num_threads()
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def bench_attention(args, rank, world, local, peaks, peak_kind):
+    import torch
+    import jagged_pointwise_attention_b200 as hstu
+    from gen import CONFIGS, make_attn_inputs
+
+    cfg = CONFIGS[args.config]
+    seed = 1000 + args.config + 7919 * rank
+    inp = make_attn_inputs(args.config, seed=seed)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    bf = torch.bfloat16 if inp.dtype == "bf16" else torch.float32
+    H, d = inp.H, inp.d
+    lengths = inp.lengths
+    flops = causal_flops(lengths, H, d, d)
+    nbytes = attn_bytes(inp.T, inp.B, H, d, d, inp.pos_bias.shape[1], inp.time_bias.shape[1],
+                        2 if inp.dtype == "bf16" else 4)
+    in_bytes = inp.T * H * 3 * d * (2 if bf == torch.bfloat16 else 4)
+    ncopies = max(1, int(np.ceil(2 * L2_BYTES / max(in_bytes, 1))))
+
+    def to_dev(a, dt=None):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        return (t.to(dt) if dt is not None else t).to(dev)
+
+    copies = []
+    for _ in range(ncopies):
+        copies.append(dict(q=to_dev(inp.q, bf), k=to_dev(inp.k, bf), v=to_dev(inp.v, bf),
+                           out=torch.empty((inp.T, H, d), dtype=bf, device=dev)))
+    off = to_dev(inp.seq_offsets)
+    ts = to_dev(inp.timestamps)
+    pos = to_dev(inp.pos_bias)
+    tb = to_dev(inp.time_bias)
+    ws = torch.empty(max(16, hstu.hstu_attn_workspace_bytes(inp.B, inp.T, inp.max_seqlen)),
+                     dtype=torch.uint8, device=dev)
+
+    def step(i, ev=None):
+        c = copies[i % ncopies]
+        if bf == torch.bfloat16:
+            hstu.hstu_attn_plan(off, inp.max_seqlen, inp.T, ws)
+        if ev is not None:
+            ev[0].record(stream)
+        hstu.hstu_attn_run(c["q"], c["k"], c["v"], off, ts, pos, tb, inp.max_seqlen, c["out"], ws)
+        if ev is not None:
+            ev[1].record(stream)
+
+    launches_per_step = 2 if bf == torch.bfloat16 else 1
+    for i in range(args.warmup):
+        step(i)
+    st = hstu.hstu_device_status()
+    if st != 0:
+        raise RuntimeError("device status %d after warm-up" % st)
+
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    _barrier(world)
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    e0.record(stream)
+    for i in range(args.steps):
+        step(i, kev[i])
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    sampler.stop()
+    _barrier(world)
+    local_ms = e0.elapsed_time(e1)
+    kernel_ms = [a.elapsed_time(b) for a, b in kev]
+    st = hstu.hstu_device_status()
+    if st != 0:
+        raise RuntimeError("device status %d after timed steps" % st)
+    max_ms, total_flops = reduce_timing(local_ms, float(flops) * args.steps, world, dev)
+    _, total_tokens = reduce_timing(0.0, float(inp.T) * args.steps, world, dev)
+    ms_per_step = max_ms / args.steps
+    value = total_flops / (max_ms * 1e-3) / 1e12
+
+    # roofline of the attention kernel (tensor-bound at d = 128, long sequences)
+    k_avg_ms = float(np.mean(kernel_ms))
+    achieved = flops / (k_avg_ms * 1e-3) / 1e12
+    tag = "attn_fwd_bf16_" + cfg["name"]
+    traffic = profiled_traffic(tag)
+    roofline = {"bound": "tensor", "achieved": round(achieved, 2),
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(achieved / peaks["bf16_tflops"], 4),
+                "peak_kind": "burst bf16 dense, %s" % peak_kind,
+                "frac_of_nominal_2250": round(achieved / NOMINAL_BF16_TFLOPS, 4),
+                "traffic": traffic, "algorithmic_bytes": nbytes,
+                "kernel": "attn_fwd_bf16_kernel<%d>" % d, "kernel_ms": round(k_avg_ms, 4),
+                "hbm_gbs_achieved": round(nbytes / (k_avg_ms * 1e-3) / 1e9, 1)}
+
+    # end to end: pinned host inputs -> device, public API call, result -> pinned host
+    e2e = e2e_attention(args, inp, dev, stream, flops, world)
+
+    cpu = None
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        v, nrows, secs, thr = oracle_sample_rate(inp, args.cpu_budget_s)
+        cpu = {"value": round(v, 6), "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+               "sample": "%d random query rows (all heads) of the same batch, fp64, %.1f s"
+                         % (nrows, secs)}
+
+    clocks = sampler.summary()
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": inp.dtype,
+        "data": "synthetic (seeded generator; no dataset)",
+        "config": {"workload": cfg["name"], "B": inp.B, "H": H, "d": d,
+                   "total_tokens": inp.T, "max_seqlen": inp.max_seqlen,
+                   "num_pos": int(inp.pos_bias.shape[1]), "num_time_buckets":
+                   int(inp.time_bias.shape[1]), "seed": seed, "parallelism": "dp%d" % world,
+                   "l2": ("inputs %.0f MB > L2" % (in_bytes / 2 ** 20)) if ncopies == 1 else
+                         ("rotating %d input copies (%.0f MB) > 2x L2" %
+                          (ncopies, ncopies * in_bytes / 2 ** 20))},
+        "pct_of_bf16_peak": {"measured_burst": round(100 * value / peaks["bf16_tflops"], 2),
+                             "nominal_2250": round(100 * value / NOMINAL_BF16_TFLOPS, 2)},
+        "tokens_per_s": round(total_tokens / (max_ms * 1e-3), 1),
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps, "clocks": clocks,
+    }
+    return line
+
+
+def e2e_attention(args, inp, dev, stream, flops, world):
+    import torch
+    import jagged_pointwise_attention_b200 as hstu
+    bf = torch.bfloat16 if inp.dtype == "bf16" else torch.float32
+
+    def pinned(a, dt=None):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        return (t.to(dt) if dt is not None else t).pin_memory()
+
+    host = dict(q=pinned(inp.q, bf), k=pinned(inp.k, bf), v=pinned(inp.v, bf),
+                off=pinned(inp.seq_offsets), ts=pinned(inp.timestamps), pos=pinned(inp.pos_bias),
+                tb=pinned(inp.time_bias))
+    devb = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
+    out_host = torch.empty((inp.T, inp.H, inp.d), dtype=bf).pin_memory()
+    out_dev = torch.empty((inp.T, inp.H, inp.d), dtype=bf, device=dev)
+    ws = torch.empty(max(16, hstu.hstu_attn_workspace_bytes(inp.B, inp.T, inp.max_seqlen)),
+                     dtype=torch.uint8, device=dev)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def step():
+        for k in host:
+            devb[k].copy_(host[k], non_blocking=True)
+        hstu.hstu_attn_fwd(devb["q"], devb["k"], devb["v"], devb["off"], devb["ts"], devb["pos"],
+                           devb["tb"], inp.max_seqlen, out=out_dev, workspace=ws)
+        out_host.copy_(out_dev, non_blocking=True)
+
+    for _ in range(max(1, min(args.warmup, 3))):
+        step()
+    n = max(1, min(args.steps, args.e2e_steps))
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _barrier(world)
+    torch.cuda.synchronize(dev)
+    a.record(stream)
+    for _ in range(n):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    _barrier(world)
+    ms, tot = reduce_timing(a.elapsed_time(b), float(flops) * n, world, dev)
+    return {"value": round(tot / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": n,
+            "ms_per_step": round(ms / n, 4)}
+
+
+def bench_layer(args, rank, world, local, peaks, peak_kind):
+    import torch
+    import jagged_pointwise_attention_b200 as hstu
+    from gen import CONFIGS, make_layer_inputs
+
+    cfg = CONFIGS[args.config]
+    seed = 1000 + args.config + 7919 * rank
+    li = make_layer_inputs(args.config, seed=seed)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    bf = torch.bfloat16
+    to = lambda a, dt=None: (torch.from_numpy(np.ascontiguousarray(a)).to(dt)  # noqa: E731
+                             if dt else torch.from_numpy(np.ascontiguousarray(a))).to(dev)
+    x, W1, W2 = to(li.x, bf), to(li.W1, bf), to(li.W2, bf)
+    off, ts, pos, tb = to(li.seq_offsets), to(li.timestamps), to(li.pos_bias), to(li.time_bias)
+    out = torch.empty_like(x)
+    ws = torch.empty(hstu.hstu_layer_workspace_bytes(li.T, li.B, li.H, li.d, li.max_seqlen),
+                     dtype=torch.uint8, device=dev)
+    lengths = np.diff(li.seq_offsets)
+    fl = causal_flops(lengths, li.H, li.d, li.d) + layer_flops(li.T, li.D, li.H, li.d)
+
+    def step():
+        hstu.hstu_layer_fwd(x, W1, W2, off, ts, pos, tb, li.H, li.d, li.max_seqlen,
+                            ln_eps=li.ln_eps, out=out, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    assert hstu.hstu_device_status() == 0
+    sampler = ClockSampler(local)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _barrier(world)
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    sampler.stop()
+    _barrier(world)
+    assert hstu.hstu_device_status() == 0
+    max_ms, tot = reduce_timing(e0.elapsed_time(e1), float(fl) * args.steps, world, dev)
+    _, toks = reduce_timing(0.0, float(li.T) * args.steps, world, dev)
+    value = tot / (max_ms * 1e-3) / 1e12
+    return {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(max_ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded generator; no dataset)",
+        "config": {"workload": cfg["name"], "B": li.B, "D": li.D, "H": li.H, "d": li.d,
+                   "total_tokens": li.T, "parallelism": "dp%d" % world,
+                   "l2": "layer working set > L2"},
+        "tokens_per_s": round(toks / (max_ms * 1e-3), 1),
+        "pct_of_bf16_peak": {"measured_burst": round(100 * value / peaks["bf16_tflops"], 2)},
+        "roofline": None, "cpu_baseline": None, "e2e": None,
+        "gpu_launches": 5 * args.steps, "clocks": sampler.summary(),
+    }
+
+
+def _barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def bench_reference(args, rank, world):
+    """The fp64 CPU oracle on the host cores: each step a bounded row sample of
+    the same workload, sized so the whole run ends within a few minutes."""
+    if rank != 0:
+        return None
+    from gen import CONFIGS, make_attn_inputs
+    import oracle
+    cfg = CONFIGS[args.config]
+    if cfg["kind"] != "attn":
+        return {"impl": "reference", "unavailable": "reference arm covers the attention "
+                "workloads only"}
+    inp = make_attn_inputs(args.config, seed=1000 + args.config)
+    n_steps = args.steps + args.warmup
+    per_step = max(0.5, min(20.0, args.reference_budget_s / max(n_steps, 1)))
+    rates, secs, rows = [], 0.0, 0
+    for s in range(n_steps):
+        v, nr, dt, thr = oracle_sample_rate(inp, per_step, seed=s)
+        if s >= args.warmup:
+            rates.append(v)
+            secs += dt
+            rows += nr
+    value = float(np.mean(rates))
+    fl_step = causal_flops(inp.lengths, inp.H, inp.d, inp.d)
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(fl_step / (value * 1e12) * 1e3, 3) if value > 0 else None,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded generator; no dataset)",
+        "config": {"workload": cfg["name"], "B": inp.B, "H": inp.H, "d": inp.d,
+                   "total_tokens": inp.T, "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": "%d random query rows over %d steps (%.1f s of fp64 CPU work)"
+                                   % (rows, args.steps, secs)},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+# ----------------------------------------------------------------------------- main
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=4, choices=[2, 3, 4, 5])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-budget-s", type=float, default=15.0)
+    ap.add_argument("--reference-budget-s", type=float, default=120.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    a = ap.parse_args(argv)
+    if a.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    return a
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        line = bench_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return 0
+    import torch
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    peaks, kind = load_peaks()
+    from gen import CONFIGS
+    if CONFIGS[args.config]["kind"] == "layer":
+        line = bench_layer(args, rank, world, local, peaks, kind)
+    else:
+        line = bench_attention(args, rank, world, local, peaks, kind)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,201 @@
+/*
+ * hstu.h -- C ABI of libhstu: HSTU jagged causal pointwise attention and the
+ * HSTU layer forward on NVIDIA B200 (sm_100a).
+ *
+ * The operation (HSTU, "Actions Speak Louder than Words: Trillion-Parameter
+ * Sequential Transducers for Generative Recommendations", arXiv 2402.17152,
+ * abstract; the generative-recommenders README, sections "Efficiency
+ * experiments" and "HSTU Ultra attention benchmark", for the layer order):
+ * a batch of B user-action sequences is packed back to back ("jagged") into
+ * T = seq_offsets[B] tokens. For sequence b with tokens o = seq_offsets[b] ..
+ * seq_offsets[b+1]-1, head h and positions j <= i inside the sequence:
+ *
+ *   s_ij = <q[o+i,h,:], k[o+j,h,:]>
+ *        + pos_bias[h][min(i-j, num_pos-1)]
+ *        + time_bias[h][clamp(floor(log2(max(1, ts[o+i]-ts[o+j]))), 0, NB-1)]
+ *   out[o+i,h,:] = (1/max_seqlen) * sum_{j<=i} silu(s_ij) * v[o+j,h,:]
+ *
+ * with silu(x) = x * sigmoid(x). No softmax, no 1/sqrt(d) score scale.
+ *
+ * Conventions for every entry point:
+ *  - Pointers marked "device" must be device memory of the current CUDA device
+ *    (or managed memory); they are owned by the caller, and the library keeps
+ *    no reference after the call returns. The library never allocates: scratch
+ *    lives in a caller-provided workspace sized by the *_workspace_bytes query.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Every call is asynchronous on that stream and never synchronises, except
+ *    hstu_device_status(). Calls may be captured in a CUDA graph.
+ *  - Argument errors are detected on the host before anything is launched and
+ *    return HSTU_ERR_INVALID_ARG or HSTU_ERR_UNSUPPORTED. A failed launch
+ *    returns HSTU_ERR_CUDA. Conditions only visible on the device (a sequence
+ *    longer than max_seqlen, decreasing offsets, a pipeline wait that ran out)
+ *    set a per-device error word that hstu_device_status() reports; outputs
+ *    are then unspecified.
+ *  - Token strides are in elements. bf16 tensors need 16-byte aligned bases and
+ *    token strides that are multiples of 8 elements.
+ */
+#ifndef HSTU_H_
+#define HSTU_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define HSTU_ABI_VERSION 1
+
+typedef enum hstu_status {
+    HSTU_OK = 0,
+    HSTU_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad stride or alignment */
+    HSTU_ERR_UNSUPPORTED = 2,   /* valid but outside what the kernels implement */
+    HSTU_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
+    HSTU_ERR_TIMEOUT = 4,       /* device: a bounded pipeline wait ran out */
+    HSTU_ERR_BAD_INPUT = 5      /* device: offsets decrease or a sequence exceeds max_seqlen */
+} hstu_status_t;
+
+typedef enum hstu_dtype {
+    HSTU_DTYPE_F32 = 0,         /* fp32 in/out, fp32 arithmetic on CUDA cores */
+    HSTU_DTYPE_BF16 = 1         /* bf16 in/out, fp32 accumulation on tcgen05 tensor cores */
+} hstu_dtype_t;
+
+typedef enum hstu_epilogue {
+    HSTU_EPI_NONE = 0,          /* y = x W^T + b                */
+    HSTU_EPI_SILU = 1,          /* y = silu(x W^T + b)          */
+    HSTU_EPI_RESIDUAL = 2       /* y = r + x W^T + b            */
+} hstu_epilogue_t;
+
+int32_t hstu_abi_version(void);
+const char* hstu_status_string(hstu_status_t status);
+
+/* Synchronises `stream`, then returns and clears the device error word of the
+ * current device: HSTU_ERR_TIMEOUT, HSTU_ERR_BAD_INPUT, HSTU_ERR_CUDA if the
+ * synchronisation itself failed, else HSTU_OK. */
+hstu_status_t hstu_device_status(void* stream);
+
+/* ---------------------------------------------------------------- attention */
+
+/* Workspace bytes that hstu_attn_plan / hstu_attn_fwd need for a batch of B
+ * sequences, total_tokens tokens and the given max_seqlen (bf16 path; the
+ * fp32 path needs none). Returns 0 for invalid sizes. */
+size_t hstu_attn_workspace_bytes(int32_t B, int64_t total_tokens, int32_t max_seqlen);
+
+/* Builds the work list of the bf16 attention in `workspace` (device):
+ * one entry per (sequence, 128-query tile), ordered longest-first (a query
+ * tile t of a sequence needs t+1 key tiles under the causal mask, so tiles are
+ * listed by descending t). Reads seq_offsets (device, int64 [B+1], offsets[0]
+ * = 0, non-decreasing, offsets[B] = total_tokens). max_seqlen >= every
+ * sequence length, 1 <= max_seqlen <= 131072. One kernel launch. */
+hstu_status_t hstu_attn_plan(const int64_t* seq_offsets, int32_t B, int64_t total_tokens,
+                             int32_t max_seqlen, void* workspace, size_t workspace_bytes,
+                             void* stream);
+
+/* Runs the attention for a batch planned by hstu_attn_plan with the same
+ * seq_offsets, B, total_tokens and max_seqlen (bf16 path), or directly (fp32
+ * path, workspace ignored).
+ *   q, k : device [T, H, d_qk] of `dtype`, token strides q_tok_stride,
+ *          k_tok_stride (head stride is d_qk: heads are contiguous in a token)
+ *   v    : device [T, H, d_v], token stride v_tok_stride
+ *   timestamps : device int64 [T], or NULL to drop the time-bucket term
+ *   pos_bias   : device fp32 [H, num_pos], or NULL to drop the position term
+ *   time_bias  : device fp32 [H, num_time_buckets] (1..1024 buckets), or NULL
+ *   max_seqlen : N of the 1/N scale
+ *   out  : device [T, H, d_v] of `dtype`, token stride out_tok_stride; every row
+ *          of every sequence is written, nothing else is touched
+ * Supported: bf16 with d_qk == d_v in {64, 128}; fp32 with d_qk, d_v <= 128. */
+hstu_status_t hstu_attn_run(hstu_dtype_t dtype,
+                            const void* q, int64_t q_tok_stride,
+                            const void* k, int64_t k_tok_stride,
+                            const void* v, int64_t v_tok_stride,
+                            const int64_t* seq_offsets, int32_t B, int64_t total_tokens,
+                            int32_t H, int32_t d_qk, int32_t d_v,
+                            const int64_t* timestamps,
+                            const float* pos_bias, int32_t num_pos,
+                            const float* time_bias, int32_t num_time_buckets,
+                            int32_t max_seqlen,
+                            void* out, int64_t out_tok_stride,
+                            const void* workspace, size_t workspace_bytes, void* stream);
+
+/* hstu_attn_plan followed by hstu_attn_run (two launches for bf16, one for fp32). */
+hstu_status_t hstu_attn_fwd(hstu_dtype_t dtype,
+                            const void* q, int64_t q_tok_stride,
+                            const void* k, int64_t k_tok_stride,
+                            const void* v, int64_t v_tok_stride,
+                            const int64_t* seq_offsets, int32_t B, int64_t total_tokens,
+                            int32_t H, int32_t d_qk, int32_t d_v,
+                            const int64_t* timestamps,
+                            const float* pos_bias, int32_t num_pos,
+                            const float* time_bias, int32_t num_time_buckets,
+                            int32_t max_seqlen,
+                            void* out, int64_t out_tok_stride,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/* Test hook: for every sequence b, every i and every j <= i (sequence by
+ * sequence, row-major in i then j) writes the relative-position index
+ * min(i-j, num_pos-1) and the time bucket, computed by the same device
+ * functions the bf16 attention kernel uses. Outputs are device int32 arrays of
+ * sum_b n_b(n_b+1)/2 entries (either may be NULL). */
+hstu_status_t hstu_debug_bias_indices(const int64_t* seq_offsets, int32_t B,
+                                      int64_t total_tokens, const int64_t* timestamps,
+                                      int32_t num_pos, int32_t num_time_buckets,
+                                      int32_t* pos_idx_out, int32_t* bucket_out,
+                                      void* stream);
+
+/* Test hook for the bounded-wait machinery: launches one block that waits on a
+ * pipeline barrier nothing ever signals, with a limit of about `wait_us`
+ * microseconds (1..100000), after which it records HSTU_ERR_TIMEOUT in the
+ * device error word and returns. Never hangs, never faults. */
+hstu_status_t hstu_debug_wait_timeout(int32_t wait_us, void* stream);
+
+/* ---------------------------------------------------------------- layer */
+
+/* y[M, N] = epilogue(x[M, K] W[N, K]^T + bias[N]) on tcgen05 tensor cores.
+ * x, W, y, residual: device bf16, row strides ldx, ldw (=K typically), ldy, ldr.
+ * bias: device fp32 [N] or NULL. residual: [M, N] bf16, required for
+ * HSTU_EPI_RESIDUAL, else ignored. K % 64 == 0, N % 128 == 0.
+ * This is the UVQK projection (f1, SiLU epilogue) and the output projection
+ * (f2, residual epilogue) of the HSTU layer. */
+hstu_status_t hstu_linear_fwd(const void* x, int64_t ldx, int64_t M, int32_t K,
+                              const void* W, int64_t ldw, int32_t N, const float* bias,
+                              hstu_epilogue_t epilogue, const void* residual, int64_t ldr,
+                              void* y, int64_t ldy, void* stream);
+
+/* y[m, :] = LayerNorm(a[m, :]) * u[m, :] over F features (biased variance, eps
+ * inside the square root, then gamma, beta; NULL = 1, 0). a, u, y: device bf16
+ * with row strides lda, ldu, ldy; gamma, beta: device fp32 [F] or NULL.
+ * F % 256 == 0 and F <= 2048. The output normalization and gating step of
+ * the HSTU layer. */
+hstu_status_t hstu_layernorm_gate_fwd(const void* a, int64_t lda, const void* u, int64_t ldu,
+                                      int64_t M, int32_t F, const float* gamma,
+                                      const float* beta, float eps, void* y, int64_t ldy,
+                                      void* stream);
+
+/* Workspace bytes of hstu_layer_fwd. */
+size_t hstu_layer_workspace_bytes(int64_t total_tokens, int32_t B, int32_t H, int32_t d,
+                                  int32_t max_seqlen);
+
+/* One HSTU layer forward (bf16, fp32 accumulation), four steps on `stream`:
+ *   1. UVQK = silu(x W1^T + b1)     x [T, D], W1 [4*H*d, D]; columns U|V|Q|K
+ *   2. A = attention(Q, K, V)        as hstu_attn_fwd, d_qk = d_v = d
+ *   3. Y = LayerNorm(A) * U          over the H*d features of each token
+ *   4. out = x + Y W2^T + b2         W2 [D, H*d]
+ * x, W1, W2, out: device bf16 row-major; b1 [4Hd], b2 [D], ln_gamma, ln_beta
+ * [Hd]: device fp32 or NULL. Other arguments as hstu_attn_run. D % 128 == 0,
+ * D % 64 == 0, d in {64, 128}, H*d % 256 == 0. */
+hstu_status_t hstu_layer_fwd(const void* x, int64_t total_tokens, int32_t D,
+                             const void* W1, const float* b1,
+                             const void* W2, const float* b2,
+                             const float* ln_gamma, const float* ln_beta, float ln_eps,
+                             const int64_t* seq_offsets, int32_t B, int32_t H, int32_t d,
+                             const int64_t* timestamps,
+                             const float* pos_bias, int32_t num_pos,
+                             const float* time_bias, int32_t num_time_buckets,
+                             int32_t max_seqlen, void* out,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HSTU_H_ */

@@ -1,0 +1,461 @@
+// hstu_api.cu -- host side of libhstu's C ABI (declared in include/hstu.h):
+// argument validation, TMA tensor-map encoding, workspace carving and kernel
+// launches. Every device kernel of the library is compiled in this one
+// translation unit so they share the per-device error word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "hstu.h"
+#include "attn_simt.cuh"
+#include "attn_tc.cuh"
+#include "common.cuh"
+#include "debug.cuh"
+#include "gemm_tc.cuh"
+#include "ln_gate.cuh"
+#include "plan.cuh"
+
+using namespace hstu;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point, so the
+// library does not link libcuda directly.
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000,
+                                             cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2-D bf16 tensor map over a row-major [rows, inner] view with the given row
+// stride (bytes); 64 x 128 boxes with the 128-byte swizzle the UMMA
+// descriptors expect.
+bool make_tmap_bf16(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t rows,
+                    uint64_t row_stride_bytes, uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {row_stride_bytes};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// Raise a kernel's dynamic shared-memory limit once per device.
+template <typename K>
+bool ensure_smem(K kernel, int bytes, int* done_flags) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+    if (!done_flags[dev]) {
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+            cudaSuccess)
+            return false;
+        done_flags[dev] = 1;
+    }
+    return true;
+}
+
+hstu_status_t launch_status() {
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+int max_tiles_of(int32_t max_seqlen) { return (max_seqlen + kTile - 1) / kTile; }
+
+int64_t max_units_of(int32_t B, int64_t T, int32_t max_seqlen) {
+    const int64_t by_tokens = T / kTile + B + 1;   // >= sum_b ceil(n_b / 128)
+    const int64_t by_lengths = static_cast<int64_t>(B) * max_tiles_of(max_seqlen);
+    return by_tokens < by_lengths ? by_tokens : by_lengths;
+}
+
+constexpr size_t kAttnWsHeader = 256;   // unit count, padded
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool plan_sizes_ok(int32_t B, int64_t T, int32_t max_seqlen) {
+    return B >= 0 && T >= 0 && T <= (int64_t{1} << 31) - 1 - 2 * kTile && max_seqlen >= 1 &&
+           max_seqlen <= kMaxSeqlen;
+}
+
+struct AttnCall {
+    hstu_dtype_t dtype;
+    const void *q, *k, *v;
+    int64_t qs, ks, vs;
+    const int64_t* off;
+    int32_t B;
+    int64_t T;
+    int32_t H, dqk, dv;
+    const int64_t* ts;
+    const float* pos;
+    int32_t P;
+    const float* tb;
+    int32_t NB;
+    int32_t max_seqlen;
+    void* out;
+    int64_t os;
+    const void* ws;
+    size_t ws_bytes;
+    cudaStream_t stream;
+};
+
+hstu_status_t validate_attn(const AttnCall& c) {
+    if (c.dtype != HSTU_DTYPE_F32 && c.dtype != HSTU_DTYPE_BF16) return HSTU_ERR_INVALID_ARG;
+    if (!plan_sizes_ok(c.B, c.T, c.max_seqlen)) return HSTU_ERR_INVALID_ARG;
+    if (c.H < 1 || c.dqk < 1 || c.dv < 1) return HSTU_ERR_INVALID_ARG;
+    if (c.B == 0 || c.T == 0) return HSTU_OK;
+    if (!c.q || !c.k || !c.v || !c.out || !c.off) return HSTU_ERR_INVALID_ARG;
+    if (c.qs < int64_t{c.H} * c.dqk || c.ks < int64_t{c.H} * c.dqk || c.vs < int64_t{c.H} * c.dv ||
+        c.os < int64_t{c.H} * c.dv)
+        return HSTU_ERR_INVALID_ARG;
+    if (c.pos && c.P < 1) return HSTU_ERR_INVALID_ARG;
+    if (c.tb && (c.NB < 1 || c.NB > kMaxTimeBuckets)) return HSTU_ERR_INVALID_ARG;
+    if (c.dtype == HSTU_DTYPE_BF16) {
+        if (c.dqk != c.dv || (c.dqk != 64 && c.dqk != 128)) return HSTU_ERR_UNSUPPORTED;
+        if (!aligned16(c.q) || !aligned16(c.k) || !aligned16(c.v) || !aligned16(c.out))
+            return HSTU_ERR_INVALID_ARG;
+        if (c.qs % 8 || c.ks % 8 || c.vs % 8 || c.os % 8) return HSTU_ERR_INVALID_ARG;
+        if (!c.ws || c.ws_bytes < hstu_attn_workspace_bytes(c.B, c.T, c.max_seqlen))
+            return HSTU_ERR_INVALID_ARG;
+        if (!aligned16(c.ws)) return HSTU_ERR_INVALID_ARG;
+    } else {
+        if (c.dqk > 128 || c.dv > 128) return HSTU_ERR_UNSUPPORTED;
+        if (c.H > 65535) return HSTU_ERR_UNSUPPORTED;
+    }
+    return HSTU_OK;
+}
+
+hstu_status_t run_attn(const AttnCall& c) {
+    const hstu_status_t st = validate_attn(c);
+    if (st != HSTU_OK || c.B == 0 || c.T == 0) return st;
+    const bool use_time = c.ts != nullptr && c.tb != nullptr;
+    const float inv_n = 1.0f / static_cast<float>(c.max_seqlen);
+    if (c.dtype == HSTU_DTYPE_F32) {
+        AttnF32Args a{static_cast<const float*>(c.q), c.qs, static_cast<const float*>(c.k), c.ks,
+                      static_cast<const float*>(c.v), c.vs, c.off, c.B, c.T, c.H, c.dqk, c.dv,
+                      use_time ? c.ts : nullptr, c.pos, c.P, use_time ? c.tb : nullptr,
+                      use_time ? c.NB : 1, inv_n, static_cast<float*>(c.out), c.os};
+        const dim3 grid(static_cast<unsigned>((c.T + 127) / 128), static_cast<unsigned>(c.H));
+        const int dmax = c.dqk > c.dv ? c.dqk : c.dv;
+        if (dmax <= 32) attn_fwd_f32_kernel<32><<<grid, 128, 0, c.stream>>>(a);
+        else if (dmax <= 64) attn_fwd_f32_kernel<64><<<grid, 128, 0, c.stream>>>(a);
+        else attn_fwd_f32_kernel<128><<<grid, 128, 0, c.stream>>>(a);
+        return launch_status();
+    }
+    CUtensorMap tq, tk, tv;
+    const uint64_t inner = static_cast<uint64_t>(c.H) * c.dqk;
+    if (!make_tmap_bf16(&tq, c.q, inner, c.T, c.qs * 2, 128) ||
+        !make_tmap_bf16(&tk, c.k, inner, c.T, c.ks * 2, 128) ||
+        !make_tmap_bf16(&tv, c.v, inner, c.T, c.vs * 2, 128))
+        return HSTU_ERR_CUDA;
+    const int64_t max_units = max_units_of(c.B, c.T, c.max_seqlen);
+    const uint8_t* ws = static_cast<const uint8_t*>(c.ws);
+    AttnArgs a{reinterpret_cast<const int4*>(ws + kAttnWsHeader),
+               reinterpret_cast<const int*>(ws),
+               c.H,
+               c.T,
+               use_time ? c.ts : nullptr,
+               c.pos,
+               c.pos ? c.P : 1,
+               use_time ? c.tb : nullptr,
+               use_time ? c.NB : 0,
+               inv_n,
+               static_cast<__nv_bfloat16*>(c.out),
+               c.os};
+    const int64_t grid = max_units * c.H;
+    if (grid > 0x7fffffff) return HSTU_ERR_UNSUPPORTED;
+    static int smem_done64[kMaxDevices] = {0}, smem_done128[kMaxDevices] = {0};
+    if (c.dqk == 64) {
+        if (!ensure_smem(attn_fwd_bf16_kernel<64>, AttnSmem<64>::kAlloc, smem_done64))
+            return HSTU_ERR_CUDA;
+        attn_fwd_bf16_kernel<64><<<static_cast<unsigned>(grid), kAttnThreads, AttnSmem<64>::kAlloc,
+                                   c.stream>>>(tq, tk, tv, a);
+    } else {
+        if (!ensure_smem(attn_fwd_bf16_kernel<128>, AttnSmem<128>::kAlloc, smem_done128))
+            return HSTU_ERR_CUDA;
+        attn_fwd_bf16_kernel<128><<<static_cast<unsigned>(grid), kAttnThreads,
+                                    AttnSmem<128>::kAlloc, c.stream>>>(tq, tk, tv, a);
+    }
+    return launch_status();
+}
+
+hstu_status_t plan_attn(const int64_t* off, int32_t B, int64_t T, int32_t max_seqlen, void* ws,
+                        size_t ws_bytes, cudaStream_t stream) {
+    if (!plan_sizes_ok(B, T, max_seqlen)) return HSTU_ERR_INVALID_ARG;
+    if (B == 0 || T == 0) return HSTU_OK;
+    if (!off || !ws || !aligned16(ws) || ws_bytes < hstu_attn_workspace_bytes(B, T, max_seqlen))
+        return HSTU_ERR_INVALID_ARG;
+    const int max_tiles = max_tiles_of(max_seqlen);
+    const int64_t max_units = max_units_of(B, T, max_seqlen);
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    plan_kernel<<<1, 1024, 3 * max_tiles * sizeof(int), stream>>>(
+        off, B, max_seqlen, max_tiles, static_cast<int>(max_units),
+        reinterpret_cast<int4*>(w + kAttnWsHeader), reinterpret_cast<int*>(w));
+    return launch_status();
+}
+
+hstu_status_t run_linear(const void* x, int64_t ldx, int64_t M, int32_t K, const void* W,
+                         int64_t ldw, int32_t N, const float* bias, hstu_epilogue_t epi,
+                         const void* residual, int64_t ldr, void* y, int64_t ldy,
+                         cudaStream_t stream) {
+    if (M < 0 || K < 1 || N < 1) return HSTU_ERR_INVALID_ARG;
+    if (epi != HSTU_EPI_NONE && epi != HSTU_EPI_SILU && epi != HSTU_EPI_RESIDUAL)
+        return HSTU_ERR_INVALID_ARG;
+    if (K % 64 || N % 128) return HSTU_ERR_UNSUPPORTED;
+    if (M == 0) return HSTU_OK;
+    if (M > (int64_t{1} << 31) - 256) return HSTU_ERR_UNSUPPORTED;
+    if (!x || !W || !y) return HSTU_ERR_INVALID_ARG;
+    if (ldx < K || ldw < K || ldy < N || ldx % 8 || ldw % 8 || ldy % 8) return HSTU_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(W) || !aligned16(y)) return HSTU_ERR_INVALID_ARG;
+    if (epi == HSTU_EPI_RESIDUAL && (!residual || ldr < N || ldr % 8 || !aligned16(residual)))
+        return HSTU_ERR_INVALID_ARG;
+    CUtensorMap ta, tb;
+    if (!make_tmap_bf16(&ta, x, K, M, ldx * 2, 128) || !make_tmap_bf16(&tb, W, K, N, ldw * 2, 128))
+        return HSTU_ERR_CUDA;
+    GemmArgs g{M, N, K, bias, static_cast<const __nv_bfloat16*>(residual), ldr,
+               static_cast<__nv_bfloat16*>(y), ldy};
+    const dim3 grid(static_cast<unsigned>((M + 127) / 128), static_cast<unsigned>(N / 128));
+    static int done0[kMaxDevices] = {0}, done1[kMaxDevices] = {0}, done2[kMaxDevices] = {0};
+    switch (epi) {
+        case HSTU_EPI_NONE:
+            if (!ensure_smem(gemm_bf16_kernel<0>, GemmSmem::kAlloc, done0)) return HSTU_ERR_CUDA;
+            gemm_bf16_kernel<0><<<grid, kGemmThreads, GemmSmem::kAlloc, stream>>>(ta, tb, g);
+            break;
+        case HSTU_EPI_SILU:
+            if (!ensure_smem(gemm_bf16_kernel<1>, GemmSmem::kAlloc, done1)) return HSTU_ERR_CUDA;
+            gemm_bf16_kernel<1><<<grid, kGemmThreads, GemmSmem::kAlloc, stream>>>(ta, tb, g);
+            break;
+        default:
+            if (!ensure_smem(gemm_bf16_kernel<2>, GemmSmem::kAlloc, done2)) return HSTU_ERR_CUDA;
+            gemm_bf16_kernel<2><<<grid, kGemmThreads, GemmSmem::kAlloc, stream>>>(ta, tb, g);
+            break;
+    }
+    return launch_status();
+}
+
+hstu_status_t run_ln_gate(const void* a, int64_t lda, const void* u, int64_t ldu, int64_t M,
+                          int32_t F, const float* gamma, const float* beta, float eps, void* y,
+                          int64_t ldy, cudaStream_t stream) {
+    if (M < 0 || F < 1 || !(eps >= 0.0f)) return HSTU_ERR_INVALID_ARG;
+    if (F % 256 || F > 2048) return HSTU_ERR_UNSUPPORTED;
+    if (M == 0) return HSTU_OK;
+    if (!a || !u || !y) return HSTU_ERR_INVALID_ARG;
+    if (lda < F || ldu < F || ldy < F || lda % 8 || ldu % 8 || ldy % 8) return HSTU_ERR_INVALID_ARG;
+    if (!aligned16(a) || !aligned16(u) || !aligned16(y)) return HSTU_ERR_INVALID_ARG;
+    LnGateArgs args{static_cast<const __nv_bfloat16*>(a), lda, static_cast<const __nv_bfloat16*>(u),
+                    ldu, M, gamma, beta, eps, static_cast<__nv_bfloat16*>(y), ldy};
+    const unsigned grid = static_cast<unsigned>((M + 7) / 8);
+    switch (F / 256) {
+        case 1: ln_gate_kernel<1><<<grid, 256, 0, stream>>>(args); break;
+        case 2: ln_gate_kernel<2><<<grid, 256, 0, stream>>>(args); break;
+        case 3: ln_gate_kernel<3><<<grid, 256, 0, stream>>>(args); break;
+        case 4: ln_gate_kernel<4><<<grid, 256, 0, stream>>>(args); break;
+        case 5: ln_gate_kernel<5><<<grid, 256, 0, stream>>>(args); break;
+        case 6: ln_gate_kernel<6><<<grid, 256, 0, stream>>>(args); break;
+        case 7: ln_gate_kernel<7><<<grid, 256, 0, stream>>>(args); break;
+        default: ln_gate_kernel<8><<<grid, 256, 0, stream>>>(args); break;
+    }
+    return launch_status();
+}
+
+struct LayerWs {
+    size_t uvqk, attn, y, plan, total;
+};
+
+LayerWs layer_ws(int64_t T, int32_t B, int32_t H, int32_t d, int32_t max_seqlen) {
+    LayerWs w{};
+    const size_t F = static_cast<size_t>(H) * d;
+    w.uvqk = 0;
+    w.attn = round_up(w.uvqk + static_cast<size_t>(T) * 4 * F * 2, 256);
+    w.y = round_up(w.attn + static_cast<size_t>(T) * F * 2, 256);
+    w.plan = round_up(w.y + static_cast<size_t>(T) * F * 2, 256);
+    w.total = w.plan + hstu_attn_workspace_bytes(B, T, max_seqlen);
+    return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t hstu_abi_version(void) { return HSTU_ABI_VERSION; }
+
+const char* hstu_status_string(hstu_status_t s) {
+    switch (s) {
+        case HSTU_OK: return "ok";
+        case HSTU_ERR_INVALID_ARG: return "invalid argument";
+        case HSTU_ERR_UNSUPPORTED: return "unsupported configuration";
+        case HSTU_ERR_CUDA: return "CUDA error";
+        case HSTU_ERR_TIMEOUT: return "device pipeline wait timed out";
+        case HSTU_ERR_BAD_INPUT: return "bad device input (offsets or lengths)";
+    }
+    return "unknown status";
+}
+
+hstu_status_t hstu_device_status(void* stream) {
+    if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return HSTU_ERR_CUDA;
+    unsigned int word = 0;
+    if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return HSTU_ERR_CUDA;
+    if (word != 0) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess)
+            return HSTU_ERR_CUDA;
+    }
+    if (word & kErrTimeout) return HSTU_ERR_TIMEOUT;
+    if (word & kErrBadInput) return HSTU_ERR_BAD_INPUT;
+    return HSTU_OK;
+}
+
+size_t hstu_attn_workspace_bytes(int32_t B, int64_t total_tokens, int32_t max_seqlen) {
+    if (!plan_sizes_ok(B, total_tokens, max_seqlen)) return 0;
+    return kAttnWsHeader + static_cast<size_t>(max_units_of(B, total_tokens, max_seqlen)) * 16;
+}
+
+hstu_status_t hstu_attn_plan(const int64_t* seq_offsets, int32_t B, int64_t total_tokens,
+                             int32_t max_seqlen, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+    return plan_attn(seq_offsets, B, total_tokens, max_seqlen, workspace, workspace_bytes,
+                     as_stream(stream));
+}
+
+hstu_status_t hstu_attn_run(hstu_dtype_t dtype, const void* q, int64_t q_tok_stride,
+                            const void* k, int64_t k_tok_stride, const void* v,
+                            int64_t v_tok_stride, const int64_t* seq_offsets, int32_t B,
+                            int64_t total_tokens, int32_t H, int32_t d_qk, int32_t d_v,
+                            const int64_t* timestamps, const float* pos_bias, int32_t num_pos,
+                            const float* time_bias, int32_t num_time_buckets, int32_t max_seqlen,
+                            void* out, int64_t out_tok_stride, const void* workspace,
+                            size_t workspace_bytes, void* stream) {
+    AttnCall c{dtype, q, k, v, q_tok_stride, k_tok_stride, v_tok_stride, seq_offsets, B,
+               total_tokens, H, d_qk, d_v, timestamps, pos_bias, num_pos, time_bias,
+               num_time_buckets, max_seqlen, out, out_tok_stride, workspace, workspace_bytes,
+               as_stream(stream)};
+    return run_attn(c);
+}
+
+hstu_status_t hstu_attn_fwd(hstu_dtype_t dtype, const void* q, int64_t q_tok_stride,
+                            const void* k, int64_t k_tok_stride, const void* v,
+                            int64_t v_tok_stride, const int64_t* seq_offsets, int32_t B,
+                            int64_t total_tokens, int32_t H, int32_t d_qk, int32_t d_v,
+                            const int64_t* timestamps, const float* pos_bias, int32_t num_pos,
+                            const float* time_bias, int32_t num_time_buckets, int32_t max_seqlen,
+                            void* out, int64_t out_tok_stride, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+    AttnCall c{dtype, q, k, v, q_tok_stride, k_tok_stride, v_tok_stride, seq_offsets, B,
+               total_tokens, H, d_qk, d_v, timestamps, pos_bias, num_pos, time_bias,
+               num_time_buckets, max_seqlen, out, out_tok_stride, workspace, workspace_bytes,
+               as_stream(stream)};
+    hstu_status_t st = validate_attn(c);
+    if (st != HSTU_OK || B == 0 || total_tokens == 0) return st;
+    if (dtype == HSTU_DTYPE_BF16) {
+        st = plan_attn(seq_offsets, B, total_tokens, max_seqlen, workspace, workspace_bytes,
+                       as_stream(stream));
+        if (st != HSTU_OK) return st;
+    }
+    return run_attn(c);
+}
+
+hstu_status_t hstu_debug_bias_indices(const int64_t* seq_offsets, int32_t B, int64_t total_tokens,
+                                      const int64_t* timestamps, int32_t num_pos,
+                                      int32_t num_time_buckets, int32_t* pos_idx_out,
+                                      int32_t* bucket_out, void* stream) {
+    if (B < 0 || total_tokens < 0 || num_pos < 1 || num_time_buckets < 1) return HSTU_ERR_INVALID_ARG;
+    if (B == 0 || total_tokens == 0) return HSTU_OK;
+    if (!seq_offsets || (bucket_out && !timestamps)) return HSTU_ERR_INVALID_ARG;
+    bias_indices_kernel<<<B, 256, 0, as_stream(stream)>>>(seq_offsets, B, timestamps, num_pos,
+                                                          num_time_buckets, pos_idx_out, bucket_out);
+    return launch_status();
+}
+
+hstu_status_t hstu_debug_wait_timeout(int32_t wait_us, void* stream) {
+    if (wait_us < 1 || wait_us > 100000) return HSTU_ERR_INVALID_ARG;
+    int dev = 0, khz = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&khz, cudaDevAttrClockRate, dev) != cudaSuccess)
+        return HSTU_ERR_CUDA;
+    const long long limit = static_cast<long long>(wait_us) * (khz > 0 ? khz : 2000000) / 1000;
+    wait_timeout_kernel<<<1, 32, 0, as_stream(stream)>>>(limit);
+    return launch_status();
+}
+
+hstu_status_t hstu_linear_fwd(const void* x, int64_t ldx, int64_t M, int32_t K, const void* W,
+                              int64_t ldw, int32_t N, const float* bias, hstu_epilogue_t epilogue,
+                              const void* residual, int64_t ldr, void* y, int64_t ldy,
+                              void* stream) {
+    return run_linear(x, ldx, M, K, W, ldw, N, bias, epilogue, residual, ldr, y, ldy,
+                      as_stream(stream));
+}
+
+hstu_status_t hstu_layernorm_gate_fwd(const void* a, int64_t lda, const void* u, int64_t ldu,
+                                      int64_t M, int32_t F, const float* gamma, const float* beta,
+                                      float eps, void* y, int64_t ldy, void* stream) {
+    return run_ln_gate(a, lda, u, ldu, M, F, gamma, beta, eps, y, ldy, as_stream(stream));
+}
+
+size_t hstu_layer_workspace_bytes(int64_t total_tokens, int32_t B, int32_t H, int32_t d,
+                                  int32_t max_seqlen) {
+    if (total_tokens < 0 || H < 1 || d < 1 || !plan_sizes_ok(B, total_tokens, max_seqlen)) return 0;
+    return layer_ws(total_tokens, B, H, d, max_seqlen).total;
+}
+
+hstu_status_t hstu_layer_fwd(const void* x, int64_t total_tokens, int32_t D, const void* W1,
+                             const float* b1, const void* W2, const float* b2,
+                             const float* ln_gamma, const float* ln_beta, float ln_eps,
+                             const int64_t* seq_offsets, int32_t B, int32_t H, int32_t d,
+                             const int64_t* timestamps, const float* pos_bias, int32_t num_pos,
+                             const float* time_bias, int32_t num_time_buckets,
+                             int32_t max_seqlen, void* out, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+    const int64_t T = total_tokens;
+    if (T < 0 || D < 1 || H < 1 || d < 1 || !plan_sizes_ok(B, T, max_seqlen))
+        return HSTU_ERR_INVALID_ARG;
+    const int32_t F = H * d;
+    if (D % 128 || (d != 64 && d != 128) || F % 256 || F > 2048 || (4 * F) % 128)
+        return HSTU_ERR_UNSUPPORTED;
+    if (T == 0 || B == 0) return HSTU_OK;
+    if (!x || !W1 || !W2 || !out || !seq_offsets || !workspace) return HSTU_ERR_INVALID_ARG;
+    const LayerWs w = layer_ws(T, B, H, d, max_seqlen);
+    if (workspace_bytes < w.total || !aligned16(workspace)) return HSTU_ERR_INVALID_ARG;
+    cudaStream_t s = as_stream(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    __nv_bfloat16* uvqk = reinterpret_cast<__nv_bfloat16*>(ws + w.uvqk);
+    __nv_bfloat16* attn = reinterpret_cast<__nv_bfloat16*>(ws + w.attn);
+    __nv_bfloat16* ygate = reinterpret_cast<__nv_bfloat16*>(ws + w.y);
+    void* plan_ws = ws + w.plan;
+    const size_t plan_bytes = workspace_bytes - w.plan;
+    hstu_status_t st = run_linear(x, D, T, D, W1, D, 4 * F, b1, HSTU_EPI_SILU, nullptr, 0, uvqk,
+                                  4 * F, s);
+    if (st != HSTU_OK) return st;
+    st = plan_attn(seq_offsets, B, T, max_seqlen, plan_ws, plan_bytes, s);
+    if (st != HSTU_OK) return st;
+    AttnCall c{HSTU_DTYPE_BF16, uvqk + 2 * F, uvqk + 3 * F, uvqk + F, 4 * F, 4 * F, 4 * F,
+               seq_offsets, B, T, H, d, d, timestamps, pos_bias, num_pos, time_bias,
+               num_time_buckets, max_seqlen, attn, F, plan_ws, plan_bytes, s};
+    st = run_attn(c);
+    if (st != HSTU_OK) return st;
+    st = run_ln_gate(attn, F, uvqk, 4 * F, T, F, ln_gamma, ln_beta, ln_eps, ygate, F, s);
+    if (st != HSTU_OK) return st;
+    return run_linear(ygate, F, T, F, W2, F, D, b2, HSTU_EPI_RESIDUAL, x, D, out, D, s);
+}
+
+}  // extern "C"

@@ -1,0 +1,89 @@
+// ln_gate.cuh -- Y = LayerNorm(A) * U, one warp per token row.
+//
+// Each lane holds 8 contiguous features per 256-feature block (16-byte
+// loads). Mean first, then the biased variance of the centred values (two
+// passes over registers, so no cancellation), rsqrt(var + eps), affine, gate.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+
+namespace hstu {
+
+struct LnGateArgs {
+    const __nv_bfloat16* a;
+    int64_t lda;
+    const __nv_bfloat16* u;
+    int64_t ldu;
+    int64_t M;
+    const float* gamma;
+    const float* beta;
+    float eps;
+    __nv_bfloat16* y;
+    int64_t ldy;
+};
+
+__device__ __forceinline__ void unpack8(const uint4 w, float (&f)[8]) {
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        f[2 * q] = __uint_as_float(ww[q] << 16);
+        f[2 * q + 1] = __uint_as_float(ww[q] & 0xffff0000u);
+    }
+}
+
+template <int NV>   // F = 256 * NV features
+__global__ void __launch_bounds__(256) ln_gate_kernel(const LnGateArgs a) {
+    constexpr int F = 256 * NV;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t m = static_cast<int64_t>(blockIdx.x) * 8 + warp;
+    if (m >= a.M) return;
+    float x[NV][8];
+    float sum = 0.f;
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+        const uint4 w = *reinterpret_cast<const uint4*>(a.a + m * a.lda + k * 256 + lane * 8);
+        unpack8(w, x[k]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) sum += x[k][e];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    const float mean = sum * (1.0f / F);
+    float sq = 0.f;
+#pragma unroll
+    for (int k = 0; k < NV; ++k)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float dlt = x[k][e] - mean;
+            sq = fmaf(dlt, dlt, sq);
+        }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+    const float rstd = rsqrtf(sq * (1.0f / F) + a.eps);
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+        const int col = k * 256 + lane * 8;
+        float uf[8];
+        unpack8(*reinterpret_cast<const uint4*>(a.u + m * a.ldu + col), uf);
+        float g[8], bt[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            g[e] = a.gamma ? a.gamma[col + e] : 1.f;
+            bt[e] = a.beta ? a.beta[col + e] : 0.f;
+        }
+        uint32_t out[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float y0 = fmaf((x[k][2 * q] - mean) * rstd, g[2 * q], bt[2 * q]) * uf[2 * q];
+            const float y1 =
+                fmaf((x[k][2 * q + 1] - mean) * rstd, g[2 * q + 1], bt[2 * q + 1]) * uf[2 * q + 1];
+            __nv_bfloat162 v2 = __floats2bfloat162_rn(y0, y1);
+            out[q] = *reinterpret_cast<uint32_t*>(&v2);
+        }
+        *reinterpret_cast<uint4*>(a.y + m * a.ldy + col) = make_uint4(out[0], out[1], out[2], out[3]);
+    }
+}
+
+}  // namespace hstu

@@ -1,0 +1,220 @@
+"""HSTU attention on the GPU (through the C ABI) against the fp64 oracle."""
+
+import numpy as np
+import pytest
+import torch
+
+import jagged_pointwise_attention_b200 as hstu
+import oracle
+from gen import custom_attn_inputs, make_attn_inputs
+from gpu_util import (assert_bf16_close, assert_f32_close, attn_tensors, dev, sampled_rows)
+
+pytestmark = pytest.mark.gpu
+
+
+def run_gpu(inp, **over):
+    t = attn_tensors(inp)
+    t.update(over)
+    out = hstu.hstu_attn_fwd(t["q"], t["k"], t["v"], t["seq_offsets"], t["timestamps"],
+                             t["pos_bias"], t["time_bias"], t["max_seqlen"])
+    assert hstu.hstu_device_status() == 0
+    return out.float().cpu().numpy()
+
+
+def run_oracle(inp, rows=None, **over):
+    a = dict(timestamps=inp.timestamps, pos_bias=inp.pos_bias, time_bias=inp.time_bias)
+    a.update(over)
+    return oracle.attn(inp.seq_offsets, inp.q, inp.k, inp.v, a["timestamps"], a["pos_bias"],
+                       a["time_bias"], inp.max_seqlen, rows=rows)
+
+
+# ----------------------------------------------------------------- workloads
+
+
+def test_tiny_fp32_workload():
+    inp = make_attn_inputs(1)
+    assert_f32_close(run_gpu(inp), run_oracle(inp), "tiny fp32")
+
+
+@pytest.mark.parametrize("cfg", [2, 3])
+def test_short_workloads_full(cfg):
+    inp = make_attn_inputs(cfg)
+    assert_bf16_close(run_gpu(inp), run_oracle(inp), "config %d" % cfg)
+
+
+def test_long_workload_sampled_rows():
+    inp = make_attn_inputs(4)
+    got = run_gpu(inp)
+    rows = sampled_rows(inp.seq_offsets)
+    assert_bf16_close(got[rows], run_oracle(inp, rows=rows), "long 8192 (sampled)")
+    assert np.all(np.isfinite(got))
+
+
+# ----------------------------------------------------------------- multi-tile ragged
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_ragged_multi_tile_full(d):
+    lens = [1, 127, 128, 129, 300, 0, 513, 64, 255, 256, 2]
+    inp = custom_attn_inputs(lens, H=3, d=d, num_pos=400, num_buckets=128, dtype="bf16", seed=d)
+    assert_bf16_close(run_gpu(inp), run_oracle(inp), "ragged d=%d" % d)
+
+
+def test_fp32_ragged_dims():
+    inp = custom_attn_inputs([3, 0, 70, 129], H=2, d=48, num_pos=50, num_buckets=16, dtype="f32",
+                             seed=3)
+    assert_f32_close(run_gpu(inp), run_oracle(inp), "fp32 d=48")
+
+
+# ----------------------------------------------------------------- edge cases
+
+
+def test_empty_batches():
+    inp = custom_attn_inputs([0, 0, 0], H=2, d=64, num_pos=8, num_buckets=8, seed=1)
+    assert run_gpu(inp).shape == (0, 2, 64)
+    inp = custom_attn_inputs([5], H=2, d=64, num_pos=8, num_buckets=8, seed=1)
+    t = attn_tensors(inp)
+    out = torch.full_like(t["q"], 7.0)
+    hstu.hstu_attn_fwd(t["q"][:0], t["k"][:0], t["v"][:0], dev(np.array([0], np.int64)), None,
+                       None, None, 5, out=out[:0])
+    assert hstu.hstu_device_status() == 0
+
+
+def test_length_one_sequences_and_zeros_between():
+    inp = custom_attn_inputs([1, 0, 1, 1, 0, 3], H=2, d=128, num_pos=8, num_buckets=8, seed=4)
+    assert_bf16_close(run_gpu(inp), run_oracle(inp), "length-1")
+
+
+def test_position_clip_and_bucket_clamp_bind():
+    # P < sequence length (clip binds); 6 buckets with hour gaps (clamp binds)
+    inp = custom_attn_inputs([300, 50], H=2, d=64, num_pos=17, num_buckets=6, seed=5,
+                             bias_std=0.5)
+    assert_bf16_close(run_gpu(inp), run_oracle(inp), "clip/clamp")
+
+
+def test_terms_dropped():
+    inp = custom_attn_inputs([200, 31], H=2, d=64, num_pos=256, num_buckets=32, seed=6,
+                             bias_std=0.5)
+    got = run_gpu(inp, timestamps=None)
+    assert_bf16_close(got, run_oracle(inp, timestamps=None, time_bias=None), "no time")
+    got = run_gpu(inp, pos_bias=None, time_bias=None)
+    assert_bf16_close(got, run_oracle(inp, pos_bias=None, time_bias=None), "no bias")
+
+
+def test_non_monotone_and_huge_timestamps():
+    inp = custom_attn_inputs([260, 140], H=2, d=64, num_pos=512, num_buckets=64, seed=7,
+                             bias_std=0.5)
+    rng = np.random.default_rng(7)
+    # random order inside the sequence, spans far beyond 2^31 (64-bit bucket path)
+    inp.timestamps = rng.integers(-(2 ** 40), 2 ** 40, size=inp.T).astype(np.int64)
+    assert_bf16_close(run_gpu(inp), run_oracle(inp), "huge/non-monotone timestamps")
+
+
+def test_scaled_by_max_seqlen_argument():
+    inp = custom_attn_inputs([90, 40], H=2, d=64, num_pos=128, num_buckets=16, seed=8)
+    inp.max_seqlen = 1000
+    assert_bf16_close(run_gpu(inp), run_oracle(inp), "N=1000")
+
+
+def test_strided_views():
+    """q, k, v, out as column slices of wider token rows (the layer's U|V|Q|K layout)."""
+    inp = custom_attn_inputs([150, 7, 260], H=2, d=128, num_pos=300, num_buckets=32, seed=9)
+    T, H, d = inp.q.shape
+    big = torch.zeros(T, 4, H * d, dtype=torch.bfloat16, device="cuda")
+    big[:, 1] = dev(inp.v.reshape(T, H * d), torch.bfloat16)
+    big[:, 2] = dev(inp.q.reshape(T, H * d), torch.bfloat16)
+    big[:, 3] = dev(inp.k.reshape(T, H * d), torch.bfloat16)
+    outbig = torch.zeros(T, 2, H * d, dtype=torch.bfloat16, device="cuda")
+    q, k, v = big[:, 2].unflatten(1, (H, d)), big[:, 3].unflatten(1, (H, d)), big[:, 1].unflatten(1, (H, d))
+    out = outbig[:, 1].unflatten(1, (H, d))
+    assert q.stride(0) == 4 * H * d
+    t = attn_tensors(inp)
+    hstu.hstu_attn_fwd(q, k, v, t["seq_offsets"], t["timestamps"], t["pos_bias"], t["time_bias"],
+                       inp.max_seqlen, out=out)
+    assert hstu.hstu_device_status() == 0
+    assert torch.count_nonzero(outbig[:, 0]) == 0, "writes outside out"
+    assert_bf16_close(out.float().cpu().numpy(), run_oracle(inp), "strided")
+
+
+def test_deterministic_and_batch_independent():
+    lens = [300, 129, 1, 600]
+    inp = custom_attn_inputs(lens, H=2, d=64, num_pos=700, num_buckets=64, seed=10)
+    a = run_gpu(inp)
+    b = run_gpu(inp)
+    assert np.array_equal(a, b)
+    off = inp.seq_offsets
+    for s in range(len(lens)):
+        sl = slice(int(off[s]), int(off[s + 1]))
+        t = attn_tensors(inp)
+        alone = hstu.hstu_attn_fwd(t["q"][sl], t["k"][sl], t["v"][sl],
+                                   dev(np.array([0, lens[s]], np.int64)), t["timestamps"][sl],
+                                   t["pos_bias"], t["time_bias"], inp.max_seqlen)
+        assert np.array_equal(alone.float().cpu().numpy(), a[sl]), s
+
+
+def test_causality_on_gpu():
+    lens = [400]
+    inp = custom_attn_inputs(lens, H=2, d=128, num_pos=512, num_buckets=64, seed=11)
+    base = run_gpu(inp)
+    cut = 200
+    inp.q[cut + 1:] = -inp.q[cut + 1:]
+    inp.k[cut + 1:] = 0.5 * inp.k[cut + 1:]
+    inp.v[cut + 1:] = -inp.v[cut + 1:]
+    inp.timestamps[cut + 1:] += 99999
+    pert = run_gpu(inp)
+    assert np.array_equal(base[:cut + 1], pert[:cut + 1])
+    assert not np.array_equal(base[cut + 1:], pert[cut + 1:])
+
+
+def test_plan_then_run_matches_fwd():
+    inp = make_attn_inputs(2)
+    t = attn_tensors(inp)
+    ws = torch.empty(hstu.hstu_attn_workspace_bytes(inp.B, inp.T, inp.max_seqlen),
+                     dtype=torch.uint8, device="cuda")
+    hstu.hstu_attn_plan(t["seq_offsets"], inp.max_seqlen, inp.T, ws)
+    out = torch.empty_like(t["q"])
+    for _ in range(2):   # a plan is reusable
+        hstu.hstu_attn_run(t["q"], t["k"], t["v"], t["seq_offsets"], t["timestamps"],
+                           t["pos_bias"], t["time_bias"], inp.max_seqlen, out, ws)
+    assert hstu.hstu_device_status() == 0
+    assert np.array_equal(out.float().cpu().numpy(), run_gpu(inp))
+
+
+def test_sequence_longer_than_max_seqlen_is_reported():
+    inp = custom_attn_inputs([300], H=2, d=64, num_pos=8, num_buckets=8, seed=12)
+    t = attn_tensors(inp)
+    hstu.hstu_attn_fwd(t["q"], t["k"], t["v"], t["seq_offsets"], t["timestamps"], t["pos_bias"],
+                       t["time_bias"], 200)
+    assert hstu.hstu_device_status() == 5          # HSTU_ERR_BAD_INPUT
+    assert hstu.hstu_device_status() == 0          # cleared
+
+
+# ----------------------------------------------------------------- integer pieces
+
+
+@pytest.mark.parametrize("case", ["workload", "edges"])
+def test_bias_indices_bit_exact(case):
+    if case == "workload":
+        inp = make_attn_inputs(2, max_batch=6)
+        ts = inp.timestamps
+        off = inp.seq_offsets
+        P, NB = 200, 128
+    else:
+        diffs = [0, 1, 2, 3, 4, 7, 8, 9, 2 ** 31 - 1, 2 ** 31, 2 ** 31 + 1, 2 ** 32, 2 ** 40 + 5,
+                 2 ** 61]
+        ts = np.array([0] + diffs + [-5, 10, 10, -(2 ** 61)], dtype=np.int64)
+        off = np.array([0, 6, len(ts)], dtype=np.int64)
+        P, NB = 4, 40
+    pos, bkt = hstu.hstu_debug_bias_indices(dev(off), dev(ts), P, NB)
+    assert hstu.hstu_device_status() == 0
+    wp, wb = oracle.bias_indices(off, ts, P, NB)
+    assert np.array_equal(pos.cpu().numpy(), wp)
+    assert np.array_equal(bkt.cpu().numpy(), wb)
+
+
+def test_bounded_wait_reports_timeout():
+    hstu.hstu_debug_wait_timeout(2000)            # about 2 ms, then gives up
+    assert hstu.hstu_device_status() == 4          # HSTU_ERR_TIMEOUT
+    assert hstu.hstu_device_status() == 0          # cleared; the context stays usable
+    inp = custom_attn_inputs([33], H=1, d=64, num_pos=8, num_buckets=8, seed=13)
+    assert_bf16_close(run_gpu(inp), run_oracle(inp), "after timeout")

@@ -1,0 +1,97 @@
+"""HSTU layer pieces and the full layer on the GPU (through the C ABI) against
+the fp64 oracle."""
+
+import numpy as np
+import pytest
+import torch
+
+import jagged_pointwise_attention_b200 as hstu
+import oracle
+from gen import make_layer_inputs, round_to_bf16
+from gpu_util import assert_bf16_close, dev
+
+pytestmark = pytest.mark.gpu
+
+
+def bf(a):
+    return dev(a, torch.bfloat16)
+
+
+def test_linear_silu_and_residual():
+    rng = np.random.default_rng(0)
+    M, K, N = 300, 512, 384          # ragged M tail, several N tiles
+    x = round_to_bf16(rng.standard_normal((M, K)).astype(np.float32))
+    W = round_to_bf16((rng.standard_normal((N, K)) / np.sqrt(K)).astype(np.float32))
+    b = (0.1 * rng.standard_normal(N)).astype(np.float32)
+    r = round_to_bf16(rng.standard_normal((M, N)).astype(np.float32))
+    got = hstu.hstu_linear_fwd(bf(x), bf(W), dev(b), "silu")
+    assert hstu.hstu_device_status() == 0
+    assert_bf16_close(got.float().cpu().numpy(), oracle.linear(x, W, b, act_silu=True), "silu")
+    got = hstu.hstu_linear_fwd(bf(x), bf(W), None, "residual", residual=bf(r))
+    assert_bf16_close(got.float().cpu().numpy(), oracle.linear(x, W, None, False, r), "residual")
+    got = hstu.hstu_linear_fwd(bf(x), bf(W), dev(b), "none")
+    assert_bf16_close(got.float().cpu().numpy(), oracle.linear(x, W, b), "plain")
+
+
+def test_linear_projection_shapes():
+    """The layer's shapes: [T, 512] x [2048, 512]^T and [T, 512] x [512, 512]^T."""
+    rng = np.random.default_rng(1)
+    M = 1000
+    x = round_to_bf16(rng.standard_normal((M, 512)).astype(np.float32))
+    W1 = round_to_bf16((rng.standard_normal((2048, 512)) / np.sqrt(512)).astype(np.float32))
+    got = hstu.hstu_linear_fwd(bf(x), bf(W1), None, "silu")
+    assert hstu.hstu_device_status() == 0
+    rows = np.arange(0, M, 7)
+    assert_bf16_close(got.float().cpu().numpy()[rows], oracle.linear(x[rows], W1, act_silu=True),
+                      "f1 shape")
+
+
+def test_layernorm_gate():
+    rng = np.random.default_rng(2)
+    M, F = 517, 512
+    a = round_to_bf16((rng.standard_normal((M, F)) * 0.01 + 0.003).astype(np.float32))
+    a[:5] *= 1e-3                                   # rows where eps dominates the variance
+    u = round_to_bf16(rng.standard_normal((M, 4 * F)).astype(np.float32))
+    g = (1 + 0.1 * rng.standard_normal(F)).astype(np.float32)
+    bt = (0.1 * rng.standard_normal(F)).astype(np.float32)
+    ud = bf(u)
+    got = hstu.hstu_layernorm_gate_fwd(bf(a), ud[:, :F], dev(g), dev(bt), 1e-5)
+    assert hstu.hstu_device_status() == 0
+    want = oracle.layernorm_gate(a, u[:, :F], g, bt, 1e-5)
+    assert_bf16_close(got.float().cpu().numpy(), want, "ln gate")
+    got = hstu.hstu_layernorm_gate_fwd(bf(a), ud[:, :F])
+    assert_bf16_close(got.float().cpu().numpy(), oracle.layernorm_gate(a, u[:, :F]), "ln identity")
+
+
+def _layer_gpu(li, **kw):
+    out = hstu.hstu_layer_fwd(bf(li.x), bf(li.W1), bf(li.W2), dev(li.seq_offsets),
+                              dev(li.timestamps), dev(li.pos_bias), dev(li.time_bias), li.H, li.d,
+                              li.max_seqlen, ln_eps=li.ln_eps, **kw)
+    assert hstu.hstu_device_status() == 0
+    return out.float().cpu().numpy()
+
+
+def _layer_oracle(li, rows=None):
+    return oracle.layer(li.seq_offsets, li.x, li.W1, li.W2, li.H, li.d, li.timestamps,
+                        li.pos_bias, li.time_bias, li.max_seqlen, ln_eps=li.ln_eps, rows=rows)
+
+
+def test_layer_small_full():
+    li = make_layer_inputs(5, lengths_override=[130, 0, 1, 257, 40])
+    assert_bf16_close(_layer_gpu(li), _layer_oracle(li), "layer small")
+
+
+def test_layer_workload_sampled_rows():
+    li = make_layer_inputs(5)
+    got = _layer_gpu(li)
+    assert np.all(np.isfinite(got))
+    # rows from a few sequences keep the oracle's projection prefixes short
+    off = li.seq_offsets
+    lens = np.diff(off)
+    seqs = [int(np.argmin(lens)), 3, 17]
+    rows = []
+    for s in seqs:
+        o, n = int(off[s]), int(lens[s])
+        rows += [o, o + 1, o + 127, o + 128, o + n // 2, o + n - 1]
+    rows = np.array(sorted(set(r for r in rows if r < li.T)), dtype=np.int64)
+    assert_bf16_close(got[rows], _layer_oracle(li, rows), "layer workload")
