@@ -59,6 +59,8 @@ def _tok_stride(t: torch.Tensor, H: int, d: int) -> int:
     """Token stride of a [T, H, d] view whose heads are contiguous inside a token."""
     if t.dim() != 3 or t.shape[1] != H or t.shape[2] != d:
         raise ValueError("expected [T, %d, %d], got %s" % (H, d, tuple(t.shape)))
+    if t.shape[0] == 0:
+        return H * d          # empty batch: strides of a size-0 tensor are arbitrary
     if t.stride(2) != 1 or (H > 1 and t.stride(1) != d):
         raise ValueError("heads and features must be contiguous inside a token")
     return t.stride(0)

@@ -40,12 +40,20 @@ def errors(got, want):
     return rel, float(np.abs(diff).max())
 
 
-def assert_bf16_close(got, want, what=""):
+def assert_bf16_close(got, want, what="", strict_abs=False):
+    """bf16 bar: relative Frobenius error <= 1e-2 and max abs error <= 3e-2.
+    The absolute bar presumes outputs of magnitude <= 1, which the workloads
+    have (the 1/N scale); bf16 rounds P and the output to 2^-9 relative, so for
+    edge cases at other scales (strict_abs=False) it is applied relative to the
+    largest |output|."""
     rel, mx = errors(got, want)
     assert np.all(np.isfinite(np.asarray(got, dtype=np.float64))), what + ": non-finite output"
-    assert rel <= BF16_REL_FROB and mx <= BF16_MAX_ABS, \
-        "%s: rel-Frobenius %.3e (<= %.0e), max-abs %.3e (<= %.0e)" % (
-            what, rel, BF16_REL_FROB, mx, BF16_MAX_ABS)
+    want_a = np.asarray(want, dtype=np.float64)
+    scale = 1.0 if strict_abs or want_a.size == 0 else max(1.0, float(np.abs(want_a).max()))
+    bound = BF16_MAX_ABS * scale
+    assert rel <= BF16_REL_FROB and mx <= bound, \
+        "%s: rel-Frobenius %.3e (<= %.0e), max-abs %.3e (<= %.3e)" % (
+            what, rel, BF16_REL_FROB, mx, bound)
     return rel, mx
 
 

@@ -94,4 +94,4 @@ def test_layer_workload_sampled_rows():
         o, n = int(off[s]), int(lens[s])
         rows += [o, o + 1, o + 127, o + 128, o + n // 2, o + n - 1]
     rows = np.array(sorted(set(r for r in rows if r < li.T)), dtype=np.int64)
-    assert_bf16_close(got[rows], _layer_oracle(li, rows), "layer workload")
+    assert_bf16_close(got[rows], _layer_oracle(li, rows), "layer workload", strict_abs=True)
