@@ -3,20 +3,43 @@
 // One CTA computes one (128-row query tile, head) work unit. For every key
 // tile j of the unit (causal tiles only):
 //     S_j  = Q K_j^T                         tcgen05.mma, SMEM x SMEM -> TMEM (fp32)
-//     P_j  = silu(S_j + pos + time) * mask   TMEM -> registers -> bf16 SMEM
-//     O   += P_j V_j                          tcgen05.mma, SMEM x SMEM -> TMEM (fp32)
+//     P_j  = silu(S_j + pos + time) * mask   TMEM -> registers -> bf16 TMEM
+//     O   += P_j V_j                          tcgen05.mma, TMEM x SMEM -> TMEM (fp32)
 // and finally out = O / max_seqlen (bf16). There is no softmax: no running
-// max, no rescale, no row sum, so O accumulates untouched across key tiles.
+// max, no rescale, no row sum, so O accumulates untouched across key tiles
+// and the whole per-element budget goes to the bias gathers and the SiLU.
 //
-// Warp roles (224 threads):
-//   warps 0-3  pointwise stage: one query row (TMEM lane) per thread
-//   warp 4     TMA producer: Q once, K/V tiles into a 2-stage ring
-//   warp 5     MMA issuer (one thread) and TMEM owner
-//   warp 6     bias staging: key timestamps and the relative-position window
-// TMEM (512 columns): S double buffer at 0 and 128, O at 256.
+// Warp roles (352 threads):
+//   warps 0-7  pointwise stage: warp w owns TMEM lanes 32*(w%4).. (one query
+//              row per thread) and S columns 64*(w/4)..+63
+//   warp 8     TMA producers: lane 0 loads Q and the K ring, lane 1 the V ring
+//              (2 stages each; K_j+2 is fetched as soon as S_j is done, V_j+2
+//              as soon as PV_j is done)
+//   warp 9     MMA issuer (one thread) and TMEM owner
+//   warp 10    bias staging: per key tile, key timestamps (int64 and their low
+//              32 bits), tile min/max and monotonicity, and the window of the
+//              relative-position table the tile needs, one stage per S buffer
+// TMEM (512 columns): S double buffer at 0 and 128, O at 256. P_j overwrites
+// the S_j buffer it came from: the warp that read S columns 64h..64h+63 writes
+// their 64 bf16 results into columns 64h..64h+31 (two per 32-bit column), so
+// no warp writes columns another warp still has to read.
+//
+// Per key tile the pointwise warps wait once (S_j and its bias stage ready)
+// and arrive once (P_j written); the MMA issues PV_j and then S_j+2 into the
+// same buffer, in order.
+//
+// Pointwise arithmetic per score, with h = x/2 folded into the bias adds:
+//   h = s/2 + pos/2 + time/2;  silu(x) = h + h*tanh(h)  (packed bf16x2, one
+//   MUFU op per two scores). The time bucket floor(log2(max(1, dt))) is the
+//   exponent field of dt converted exactly to double (no bit-find unit), and
+//   the bucket's bias comes from a 32-entry register table via a shuffle. When
+//   the key timestamps of a 32-key chunk are non-decreasing and every row of
+//   the warp sees one bucket at both ends of the chunk, the bucket is constant
+//   over the chunk and the per-score bucket work is skipped.
+//
 // Every wait is bounded; a wait that runs out raises kErrTimeout, the other
-// roles notice through a shared abort flag, and the CTA drains its own
-// copies and MMAs before it frees TMEM and exits.
+// roles notice through a shared abort flag, and the CTA drains its own copies
+// and MMAs before it frees TMEM and exits.
 #pragma once
 
 #include "common.cuh"
@@ -39,44 +62,51 @@ struct AttnArgs {
     int64_t out_stride;         // elements per token
 };
 
+constexpr int kPointwiseWarps = 8;
+constexpr int kPointwiseThreads = kPointwiseWarps * 32;
+constexpr int kWarpTMA = 8, kWarpMMA = 9, kWarpMeta = 10;
+constexpr int kAttnThreads = 11 * 32;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemO = 256;
+
+// One stage of staged bias data for one key tile.
+struct MetaStage {
+    float w[256];          // w[m] = pos[h][clamp(q0 - kt0 - 127 + m, 0, P-1)] / 2
+    int32_t kt32[128];     // low 32 bits of the key timestamps
+    int64_t kt64[128];     // key timestamps
+    int64_t tmin, tmax;    // over keys of the unit (< q_end)
+    int32_t mono;          // keys non-decreasing over the tile (keys < q_end)
+    int32_t pad[3];
+};
+
 template <int D>
 struct AttnSmem {
     static constexpr int kQBytes = kTile * D * 2;       // Q tile, D/64 swizzled 16 KB blocks
     static constexpr int kKVBytes = kTile * D * 2;      // one K (or V) stage
-    static constexpr int kPBytes = kTile * kTile * 2;   // P tile, 2 swizzled 16 KB blocks
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + kQBytes;
     static constexpr int kOffV = kOffK + 2 * kKVBytes;
-    static constexpr int kOffP = kOffV + 2 * kKVBytes;
-    static constexpr int kOffTB = kOffP + kPBytes;                  // float[kMaxTimeBuckets]
-    static constexpr int kOffW = kOffTB + kMaxTimeBuckets * 4;      // float[2][256]
-    static constexpr int kOffKT64 = kOffW + 2 * 256 * 4;            // int64[2][128]
-    static constexpr int kOffKT32 = kOffKT64 + 2 * 128 * 8;         // int32[2][128]
-    static constexpr int kOffTMinMax = kOffKT32 + 2 * 128 * 4;      // int64[2][2]
-    static constexpr int kOffBar = kOffTMinMax + 64;
-    static constexpr int kNumBars = 16;
+    static constexpr int kOffTB = kOffV + 2 * kKVBytes;                 // float[kMaxTimeBuckets]
+    static constexpr int kOffMeta = kOffTB + kMaxTimeBuckets * 4;       // MetaStage[2]
+    static constexpr int kOffBar = kOffMeta + 2 * static_cast<int>(sizeof(MetaStage));
+    static constexpr int kNumBars = 32;
     static constexpr int kOffTmem = kOffBar + kNumBars * 8;
     static constexpr int kOffAbort = kOffTmem + 8;
     static constexpr int kBytes = kOffAbort + 8;
-    static constexpr int kAlloc = kBytes + 1024;                    // 1 KB alignment slack
+    static constexpr int kAlloc = kBytes + 1024;                        // 1 KB alignment slack
 };
-
-constexpr int kAttnThreads = 224;
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemO = 256;
 
 // barrier slots
 enum {
     kBarQFull = 0,
-    kBarKVFull = 1,    // +stage
-    kBarKVFree = 3,    // +stage
-    kBarSFull = 5,     // +buffer
-    kBarSFree = 7,     // +buffer
-    kBarPFull = 9,
-    kBarPFree = 10,
-    kBarOFull = 11,
-    kBarDrain = 12,
-    kBarMeta = 13,     // +buffer
+    kBarKFull = 1,      // +stage (2)
+    kBarKFree = 3,      // +stage (2)
+    kBarVFull = 5,      // +stage (2)
+    kBarVFree = 7,      // +stage (2)
+    kBarSFull = 9,      // +buffer (2): MMA commit + 32 bias-staging lanes
+    kBarPFull = 11,     // +buffer (2): 256 pointwise threads
+    kBarOFull = 13,
+    kBarDrain = 14,
 };
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
@@ -84,44 +114,85 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
     return __all_sync(0xffffffffu, ok);
 }
 
-__device__ __forceinline__ uint32_t bfind_u32(uint32_t x) {
-    uint32_t r;
-    asm("bfind.u32 %0, %1;" : "=r"(r) : "r"(x));
-    return r;
+// silu of a packed pair of half-scores: h + h * tanh(h), bf16x2.
+__device__ __forceinline__ uint32_t silu_half_bf16x2(float h0, float h1) {
+    const uint32_t hp = pack_bf16x2(h0, h1);
+    uint32_t t, y;
+    asm("tanh.approx.bf16x2 %0, %1;" : "=r"(t) : "r"(hp));
+    asm("fma.rn.bf16x2 %0, %1, %2, %1;" : "=r"(y) : "r"(hp), "r"(t));
+    return y;
 }
 
-// Pointwise stage for one 32-column chunk of S. kFast: every valid pair of
-// this warp has |t_i - t_j| < 2^31, so 32-bit differences are exact.
-// kMask: some pair of this warp's rows lies outside [lo, hi] (causal/sequence).
-template <bool kFast, bool kMask>
-__device__ __forceinline__ void pointwise_chunk(const uint32_t (&sv)[32], int c_base,
-                                                const float* __restrict__ wrow,
-                                                const float* __restrict__ tb_s,
-                                                const int32_t* __restrict__ kt32,
-                                                const int64_t* __restrict__ kt64, int32_t ti32,
-                                                int64_t ti, int nbm1, int lo, int hi,
-                                                uint32_t* pk) {
+// Per-chunk pointwise paths. sv: 32 fp32 scores of columns c0..c0+31 of this
+// thread's row; wrow[-c] = pos/2 of column c; pk: 16 packed bf16x2 outputs.
+
+// Constant time bucket over the chunk: tconst = time/2 for every column.
+template <bool kMask>
+__device__ __forceinline__ void pw_const(const uint32_t* sv, int c0,
+                                         const float* __restrict__ wrow, float tconst, int lo,
+                                         int hi, uint32_t* pk) {
 #pragma unroll
     for (int e = 0; e < 32; e += 2) {
-        float p[2];
+        float h[2];
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-            const int c = c_base + e + u;
-            float x = __uint_as_float(sv[e + u]) + wrow[-c];
-            int bkt;
-            if (kFast) {
-                const int32_t dt = static_cast<int32_t>(static_cast<uint32_t>(ti32) -
-                                                        static_cast<uint32_t>(kt32[c]));
-                bkt = min(static_cast<int>(bfind_u32(static_cast<uint32_t>(max(dt, 1)))), nbm1);
-            } else {
-                bkt = time_bucket64(ti - kt64[c], nbm1);
-            }
-            x += tb_s[bkt];
-            float y = silu_tanh(x);
-            if (kMask) y = (c >= lo && c <= hi) ? y : 0.0f;
-            p[u] = y;
+            const int c = c0 + e + u;
+            float v = fmaf(__uint_as_float(sv[e + u]), 0.5f, wrow[-c]) + tconst;
+            if (kMask) v = (c >= lo && c <= hi) ? v : 0.0f;
+            h[u] = v;
         }
-        pk[e >> 1] = pack_bf16x2(p[0], p[1]);
+        pk[e >> 1] = silu_half_bf16x2(h[0], h[1]);
+    }
+}
+
+// Bucket per score, differences exact in 32 bits. tbr: this lane's entry of
+// the register table (lane L holds time/2 of bucket min((L+1) mod 32, NB-1)).
+template <bool kMask>
+__device__ __forceinline__ void pw_fast(const uint32_t* sv, int c0,
+                                        const float* __restrict__ wrow,
+                                        const int32_t* __restrict__ kt32, int32_t ti32, float tbr,
+                                        int lo, int hi, uint32_t* pk) {
+    const int4* k4 = reinterpret_cast<const int4*>(kt32 + c0);
+#pragma unroll
+    for (int e = 0; e < 32; e += 4) {
+        const int4 kk = k4[e >> 2];
+        const int32_t kv[4] = {kk.x, kk.y, kk.z, kk.w};
+        float h[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int c = c0 + e + u;
+            const int32_t dt = static_cast<int32_t>(static_cast<uint32_t>(ti32) -
+                                                    static_cast<uint32_t>(kv[u]));
+            const uint32_t ef = log2_exponent_field(static_cast<uint32_t>(max(dt, 1)));
+            const float tv = __shfl_sync(0xffffffffu, tbr, static_cast<int>(ef));
+            float v = fmaf(__uint_as_float(sv[e + u]), 0.5f, wrow[-c]) + tv;
+            if (kMask) v = (c >= lo && c <= hi) ? v : 0.0f;
+            h[u] = v;
+        }
+        pk[e >> 1] = silu_half_bf16x2(h[0], h[1]);
+        pk[(e >> 1) + 1] = silu_half_bf16x2(h[2], h[3]);
+    }
+}
+
+// Any int64 timestamps: 64-bit bucket, table read from shared memory.
+template <bool kMask>
+__device__ __forceinline__ void pw_slow(const uint32_t* sv, int c0,
+                                        const float* __restrict__ wrow,
+                                        const int64_t* __restrict__ kt64, int64_t ti,
+                                        const float* __restrict__ tb_s, int nbm1, int lo, int hi,
+                                        uint32_t* pk) {
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+        float h[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int c = c0 + e + u;
+            const float tv = tb_s[time_bucket64(ti - kt64[c], nbm1)];
+            float v = fmaf(__uint_as_float(sv[e + u]), 0.5f, wrow[-c]) + tv;
+            if (kMask) v = (c >= lo && c <= hi) ? v : 0.0f;
+            h[u] = v;
+        }
+        pk[e >> 1] = silu_half_bf16x2(h[0], h[1]);
     }
 }
 
@@ -152,34 +223,32 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffTmem);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffAbort);
     float* tb_s = reinterpret_cast<float*>(smem + L::kOffTB);
-    float* w_s = reinterpret_cast<float*>(smem + L::kOffW);
-    int64_t* kt64_s = reinterpret_cast<int64_t*>(smem + L::kOffKT64);
-    int32_t* kt32_s = reinterpret_cast<int32_t*>(smem + L::kOffKT32);
-    int64_t* tmm_s = reinterpret_cast<int64_t*>(smem + L::kOffTMinMax);
+    MetaStage* meta = reinterpret_cast<MetaStage*>(smem + L::kOffMeta);
+    const bool use_time = args.ts != nullptr && args.tb != nullptr && args.NB > 0;
+    const int nbm1 = use_time ? args.NB - 1 : 0;
 
     if (tid == 0) {
         *abort_flag = 0;
         mbar_init(&bars[kBarQFull], 1);
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&bars[kBarKVFull + s], 1);
-            mbar_init(&bars[kBarKVFree + s], 1);
-            mbar_init(&bars[kBarSFull + s], 1);
-            mbar_init(&bars[kBarSFree + s], 128);
-            mbar_init(&bars[kBarMeta + s], 32);
+            mbar_init(&bars[kBarKFull + s], 1);
+            mbar_init(&bars[kBarKFree + s], 1);
+            mbar_init(&bars[kBarVFull + s], 1);
+            mbar_init(&bars[kBarVFree + s], 1);
+            mbar_init(&bars[kBarSFull + s], 1 + 32);
+            mbar_init(&bars[kBarPFull + s], kPointwiseThreads);
         }
-        mbar_init(&bars[kBarPFull], 128);
-        mbar_init(&bars[kBarPFree], 1);
         mbar_init(&bars[kBarOFull], 1);
         mbar_init(&bars[kBarDrain], 1);
         mbar_fence_init();
     }
-    if (warp == 5) {
+    if (warp == kWarpMMA) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
-    if (tid < 128) {
-        for (int b = tid; b < args.NB; b += 128) tb_s[b] = args.tb ? args.tb[h * args.NB + b] : 0.f;
-        if (args.NB <= 0 && tid == 0) tb_s[0] = 0.f;
+    if (tid < kPointwiseThreads) {
+        for (int b = tid; b < kMaxTimeBuckets; b += kPointwiseThreads)
+            tb_s[b] = (use_time && b < args.NB) ? 0.5f * args.tb[static_cast<int64_t>(h) * args.NB + b] : 0.f;
     }
     tc_fence_before();
     __syncthreads();
@@ -189,63 +258,68 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
     const uint32_t sQ = smem_u32(smem + L::kOffQ);
     const uint32_t sK = smem_u32(smem + L::kOffK);
     const uint32_t sV = smem_u32(smem + L::kOffV);
-    const uint32_t sP = smem_u32(smem + L::kOffP);
 
-    if (warp == 4) {
-        // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            tma_prefetch_desc(&tmQ);
-            tma_prefetch_desc(&tmK);
-            tma_prefetch_desc(&tmV);
-            mbar_arrive_expect_tx(&bars[kBarQFull], L::kQBytes);
+    if (warp == kWarpTMA) {
+        // ------------------------------------------------------------ TMA producers
+        if (lane < 2) {
+            const bool is_k = lane == 0;
+            const CUtensorMap* tm = is_k ? &tmK : &tmV;
+            const int ring = is_k ? L::kOffK : L::kOffV;
+            uint64_t* full = &bars[is_k ? kBarKFull : kBarVFull];
+            uint64_t* freeb = &bars[is_k ? kBarKFree : kBarVFree];
+            tma_prefetch_desc(tm);
+            if (is_k) {
+                tma_prefetch_desc(&tmQ);
+                mbar_arrive_expect_tx(&bars[kBarQFull], L::kQBytes);
 #pragma unroll
-            for (int kb = 0; kb < kKB; ++kb)
-                tma_load_2d(smem + L::kOffQ + kb * 16384, &tmQ, &bars[kBarQFull], h * D + kb * 64, q0);
-            int issued[2] = {0, 0};
+                for (int kb = 0; kb < kKB; ++kb)
+                    tma_load_2d(smem + L::kOffQ + kb * 16384, &tmQ, &bars[kBarQFull], h * D + kb * 64, q0);
+            }
+            int issued0 = 0, issued1 = 0;
             for (int j = 0; j < nk; ++j) {
                 const int s = j & 1;
-                if (j >= 2 && !mbar_wait(&bars[kBarKVFree + s], ((j >> 1) - 1) & 1, abort_flag)) break;
-                mbar_arrive_expect_tx(&bars[kBarKVFull + s], 2 * L::kKVBytes);
+                if (j >= 2 && !mbar_wait(&freeb[s], ((j >> 1) - 1) & 1, abort_flag)) break;
+                mbar_arrive_expect_tx(&full[s], L::kKVBytes);
                 const int kt0 = k0 + j * kTile;
 #pragma unroll
-                for (int kb = 0; kb < kKB; ++kb) {
-                    tma_load_2d(smem + L::kOffK + s * L::kKVBytes + kb * 16384, &tmK,
-                                &bars[kBarKVFull + s], h * D + kb * 64, kt0);
-                    tma_load_2d(smem + L::kOffV + s * L::kKVBytes + kb * 16384, &tmV,
-                                &bars[kBarKVFull + s], h * D + kb * 64, kt0);
-                }
-                ++issued[s];
+                for (int kb = 0; kb < kKB; ++kb)
+                    tma_load_2d(smem + ring + s * L::kKVBytes + kb * 16384, tm, &full[s],
+                                h * D + kb * 64, kt0);
+                if (s == 0) ++issued0; else ++issued1;
             }
             // drain: every copy this thread started has landed before the CTA ends
-            if (!mbar_wait(&bars[kBarQFull], 0, nullptr)) raise_error(kErrTimeout);
-            for (int s = 0; s < 2; ++s)
-                if (issued[s] > 0 && !mbar_wait(&bars[kBarKVFull + s], (issued[s] - 1) & 1, nullptr))
-                    raise_error(kErrTimeout);
+            if (is_k && !mbar_wait(&bars[kBarQFull], 0, nullptr)) raise_error(kErrTimeout);
+            if (issued0 > 0 && !mbar_wait(&full[0], (issued0 - 1) & 1, nullptr)) raise_error(kErrTimeout);
+            if (issued1 > 0 && !mbar_wait(&full[1], (issued1 - 1) & 1, nullptr)) raise_error(kErrTimeout);
         }
-    } else if (warp == 5) {
+        __syncwarp();
+    } else if (warp == kWarpMMA) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
             auto issue_pv = [&](int jj) -> bool {
-                if (!mbar_wait(&bars[kBarPFull], jj & 1, abort_flag)) return false;
+                const int sb = jj & 1;
+                if (!mbar_wait(&bars[kBarPFull + sb], (jj >> 1) & 1, abort_flag)) return false;
+                if (!mbar_wait(&bars[kBarVFull + sb], (jj >> 1) & 1, abort_flag)) return false;
                 tc_fence_after();
-                const uint32_t vb = sV + (jj & 1) * L::kKVBytes;
+                const uint32_t vb = sV + sb * L::kKVBytes;
+                const uint32_t pb = tmem + sb * 128;
 #pragma unroll
                 for (int kk = 0; kk < kTile / 16; ++kk) {
-                    const uint64_t a = desc_kmajor_sw128(sP + (kk >> 2) * 16384 + (kk & 3) * 32);
+                    // keys 16kk..16kk+15: columns (kk/4)*64 + (kk%4)*8 of the P buffer
+                    const uint32_t a = pb + (kk >> 2) * 64 + (kk & 3) * 8;
                     const uint64_t b = desc_mnmajor_sw128(vb + kk * 2048, 16384);
-                    umma_bf16_ss(tmem + kTmemO, a, b, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
+                    umma_bf16_ts(tmem + kTmemO, a, b, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
                 }
-                umma_commit(&bars[kBarPFree]);
-                umma_commit(&bars[kBarKVFree + (jj & 1)]);
+                umma_commit(&bars[kBarVFree + sb]);
                 return true;
             };
             bool ok = mbar_wait(&bars[kBarQFull], 0, abort_flag);
             for (int j = 0; ok && j < nk; ++j) {
                 const int s = j & 1;
-                ok = mbar_wait(&bars[kBarKVFull + s], (j >> 1) & 1, abort_flag);
-                if (ok && j >= 2) ok = mbar_wait(&bars[kBarSFree + s], ((j >> 1) - 1) & 1, abort_flag);
+                // buffer s last held P_j-2, read by PV_j-2, issued earlier by this thread
+                ok = mbar_wait(&bars[kBarKFull + s], (j >> 1) & 1, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t kb_base = sK + s * L::kKVBytes;
@@ -256,6 +330,7 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                                  desc_kmajor_sw128(kb_base + off), idesc_qk, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(&bars[kBarSFull + s]);
+                umma_commit(&bars[kBarKFree + s]);
                 if (j >= 1) ok = issue_pv(j - 1);
             }
             if (ok) ok = issue_pv(nk - 1);
@@ -264,36 +339,53 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
             if (!mbar_wait(&bars[kBarDrain], 0, nullptr)) raise_error(kErrTimeout);
         }
         __syncwarp();
-    } else if (warp == 6) {
+    } else if (warp == kWarpMeta) {
         // ------------------------------------------------------------ bias staging
         for (int j = 0; j < nk; ++j) {
             const int s = j & 1;
-            if (j >= 2 && !warp_wait(&bars[kBarSFree + s], ((j >> 1) - 1) & 1, abort_flag)) break;
+            // stage s last served tile j-2; P_j-2 written means it has been read
+            if (j >= 2 && !warp_wait(&bars[kBarPFull + s], ((j >> 1) - 1) & 1, abort_flag)) break;
+            MetaStage& ms = meta[s];
             const int kt0 = k0 + j * kTile;
-            int64_t tmin = INT64_MAX, tmax = INT64_MIN;
-            for (int m = lane; m < kTile; m += 32) {
-                const int64_t key = static_cast<int64_t>(kt0) + m;
-                int64_t t = 0;
-                if (args.ts) {
-                    t = args.ts[key < args.T ? key : args.T - 1];
-                    if (key < q_end) {
-                        tmin = t < tmin ? t : tmin;
-                        tmax = t > tmax ? t : tmax;
-                    }
-                }
-                kt64_s[s * 128 + m] = t;
-                kt32_s[s * 128 + m] = static_cast<int32_t>(static_cast<uint64_t>(t));
-            }
-            // window w[m] = pos[h][clamp(q0 - kt0 - 127 + m, 0, P-1)], m = 127 + r - c
-            for (int m = lane; m < 256; m += 32) {
-                float wv = 0.f;
-                if (args.pos && m < 255) {
-                    int64_t dd = static_cast<int64_t>(q0) - kt0 - 127 + m;
+            // relative-position window, pre-halved (4 + 4 independent loads per lane)
+            float wv[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int mm = lane + 32 * u;
+                wv[u] = 0.f;
+                if (args.pos && mm < 255) {
+                    int64_t dd = static_cast<int64_t>(q0) - kt0 - 127 + mm;
                     dd = dd < 0 ? 0 : (dd > args.P - 1 ? args.P - 1 : dd);
-                    wv = args.pos[static_cast<int64_t>(h) * args.P + dd];
+                    wv[u] = args.pos[static_cast<int64_t>(h) * args.P + dd];
                 }
-                w_s[s * 256 + m] = wv;
             }
+            int64_t tv[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int64_t key = static_cast<int64_t>(kt0) + lane + 32 * u;
+                tv[u] = use_time ? args.ts[key < args.T ? key : args.T - 1] : 0;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) ms.w[lane + 32 * u] = 0.5f * wv[u];
+            int64_t tmin = INT64_MAX, tmax = INT64_MIN;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int mm = lane + 32 * u;
+                ms.kt64[mm] = tv[u];
+                ms.kt32[mm] = static_cast<int32_t>(static_cast<uint64_t>(tv[u]));
+                if (kt0 + mm < q_end) {
+                    tmin = tv[u] < tmin ? tv[u] : tmin;
+                    tmax = tv[u] > tmax ? tv[u] : tmax;
+                }
+            }
+            __syncwarp();
+            bool mono = true;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int mm = lane + 32 * u;
+                if (mm < 127 && kt0 + mm + 1 < q_end) mono = mono && (ms.kt64[mm] <= ms.kt64[mm + 1]);
+            }
+            mono = __all_sync(0xffffffffu, mono);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
                 const int64_t a = __shfl_xor_sync(0xffffffffu, tmin, o);
@@ -302,97 +394,99 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                 tmax = b > tmax ? b : tmax;
             }
             if (lane == 0) {
-                tmm_s[s * 2 + 0] = tmin;
-                tmm_s[s * 2 + 1] = tmax;
+                ms.tmin = tmin;
+                ms.tmax = tmax;
+                ms.mono = mono ? 1 : 0;
             }
             __syncwarp();
-            mbar_arrive(&bars[kBarMeta + s]);
+            mbar_arrive(&bars[kBarSFull + s]);
         }
     } else {
         // ------------------------------------------------------------ pointwise stage
-        const int r = tid;                                  // query row = TMEM lane
-        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        const int qd = warp & 3;                            // TMEM lane quarter
+        const int half = warp >> 2;                         // S columns 64*half..
+        const int r = qd * 32 + lane;                       // query row = TMEM lane
+        const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
         const int64_t i = static_cast<int64_t>(q0) + r;
         const bool row_valid = i < q_end;
-        const int64_t ti = (args.ts && row_valid) ? args.ts[i < args.T ? i : args.T - 1] : 0;
+        const int64_t ti = (use_time && row_valid) ? args.ts[i < args.T ? i : args.T - 1] : 0;
         const int32_t ti32 = static_cast<int32_t>(static_cast<uint64_t>(ti));
-        const int nbm1 = args.NB > 0 ? args.NB - 1 : 0;
-        uint32_t pk[64];
+        // register table: lane L holds time/2 of bucket min((L + 1) mod 32, NB - 1)
+        const float tbr = tb_s[min((lane + 1) & 31, nbm1)];
         bool ok = true;
         for (int j = 0; j < nk; ++j) {
             const int s = j & 1;
-            ok = warp_wait(&bars[kBarMeta + s], (j >> 1) & 1, abort_flag);
-            if (ok) ok = warp_wait(&bars[kBarSFull + s], (j >> 1) & 1, abort_flag);
+            ok = warp_wait(&bars[kBarSFull + s], (j >> 1) & 1, abort_flag);
             if (!ok) break;
             tc_fence_after();
+            const MetaStage& ms = meta[s];
             const int kt0 = k0 + j * kTile;
             const int lo = k0 - kt0;                        // first key of the sequence
             const int hi = row_valid ? static_cast<int>(i - kt0) : -1;
-            const int64_t tmin = tmm_s[s * 2 + 0], tmax = tmm_s[s * 2 + 1];
             bool fast = true;
-            if (row_valid && args.ts && tmin <= tmax) {
-                const int64_t lo_t = ti < tmin ? ti : tmin;
-                const int64_t hi_t = ti > tmax ? ti : tmax;
+            if (row_valid && use_time) {
+                const int64_t lo_t = ti < ms.tmin ? ti : ms.tmin;
+                const int64_t hi_t = ti > ms.tmax ? ti : ms.tmax;
                 fast = static_cast<uint64_t>(hi_t) - static_cast<uint64_t>(lo_t) < (1ull << 31);
             }
             const bool fast_w = __all_sync(0xffffffffu, fast);
-            const bool full_w = __all_sync(0xffffffffu, lo <= 0 && hi >= kTile - 1);
-            const float* wrow = w_s + s * 256 + 127 + r;
-            const int32_t* kt32 = kt32_s + s * 128;
-            const int64_t* kt64 = kt64_s + s * 128;
-            const uint32_t s_col = tmem + lane_base + static_cast<uint32_t>(s * 128);
-#pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-                uint32_t sv[32];
-                __syncwarp();
-                tmem_ld32(s_col + ch * 32, sv);
-                uint32_t* pkc = pk + ch * 16;
-                if (fast_w) {
-                    if (full_w)
-                        pointwise_chunk<true, false>(sv, ch * 32, wrow, tb_s, kt32, kt64, ti32, ti, nbm1, lo, hi, pkc);
-                    else
-                        pointwise_chunk<true, true>(sv, ch * 32, wrow, tb_s, kt32, kt64, ti32, ti, nbm1, lo, hi, pkc);
-                } else {
-                    if (full_w)
-                        pointwise_chunk<false, false>(sv, ch * 32, wrow, tb_s, kt32, kt64, ti32, ti, nbm1, lo, hi, pkc);
-                    else
-                        pointwise_chunk<false, true>(sv, ch * 32, wrow, tb_s, kt32, kt64, ti32, ti, nbm1, lo, hi, pkc);
+            const bool mono = ms.mono != 0;
+            const float* wrow = ms.w + 127 + r;
+            const uint32_t s_col = tmem + lane_base + static_cast<uint32_t>(s * 128 + half * 64);
+            uint32_t sv[64];
+            __syncwarp();
+            tmem_ld64(s_col, sv);
+            uint32_t pk[32];
+            // one 32-column chunk of this warp's 64 columns -> 16 packed P words
+            auto chunk = [&](int q, uint32_t* pkc) {
+                const uint32_t* svc = sv + 32 * q;
+                const int c0 = half * 64 + 32 * q;
+                const bool full = __all_sync(0xffffffffu, lo <= c0 && hi >= c0 + 31);
+                if (!fast_w) {
+                    if (full) pw_slow<false>(svc, c0, wrow, ms.kt64, ti, tb_s, nbm1, lo, hi, pkc);
+                    else pw_slow<true>(svc, c0, wrow, ms.kt64, ti, tb_s, nbm1, lo, hi, pkc);
+                    return;
                 }
-            }
+                if (full && mono) {
+                    const uint32_t ef0 = log2_exponent_field(static_cast<uint32_t>(max(
+                        static_cast<int32_t>(static_cast<uint32_t>(ti32) - static_cast<uint32_t>(ms.kt32[c0])), 1)));
+                    const uint32_t ef1 = log2_exponent_field(static_cast<uint32_t>(max(
+                        static_cast<int32_t>(static_cast<uint32_t>(ti32) - static_cast<uint32_t>(ms.kt32[c0 + 31])), 1)));
+                    const float tconst = __shfl_sync(0xffffffffu, tbr, static_cast<int>(ef0));
+                    if (__all_sync(0xffffffffu, ef0 == ef1)) {
+                        pw_const<false>(svc, c0, wrow, tconst, lo, hi, pkc);
+                        return;
+                    }
+                }
+                if (full) pw_fast<false>(svc, c0, wrow, ms.kt32, ti32, tbr, lo, hi, pkc);
+                else pw_fast<true>(svc, c0, wrow, ms.kt32, ti32, tbr, lo, hi, pkc);
+            };
+            chunk(0, pk);
+            chunk(1, pk + 16);
+            // P (64 bf16 of this row) -> columns 64h..64h+31 of the S buffer just read
+            tmem_st32(s_col, pk);
             tc_fence_before();
-            mbar_arrive(&bars[kBarSFree + s]);
-            if (j >= 1 && !warp_wait(&bars[kBarPFree], (j - 1) & 1, abort_flag)) {
-                ok = false;
-                break;
-            }
-            // P row r -> two 128 B-swizzled K-major blocks (keys 0-63, 64-127)
-            const uint32_t prow = sP + r * 128;
-#pragma unroll
-            for (int c16 = 0; c16 < 16; ++c16) {
-                const uint32_t addr = prow + (c16 >> 3) * 16384 + (((c16 & 7) ^ (r & 7)) << 4);
-                st_shared_v4(addr, pk[4 * c16], pk[4 * c16 + 1], pk[4 * c16 + 2], pk[4 * c16 + 3]);
-            }
-            fence_proxy_async_smem();
-            mbar_arrive(&bars[kBarPFull]);
+            mbar_arrive(&bars[kBarPFull + s]);
         }
         if (ok && warp_wait(&bars[kBarOFull], 0, abort_flag)) {
             tc_fence_after();
             __nv_bfloat16* orow = args.out + i * args.out_stride + static_cast<int64_t>(h) * D;
 #pragma unroll
-            for (int ch = 0; ch < D / 32; ++ch) {
+            for (int ch = 0; ch < D / 64; ++ch) {
+                const int col = half * (D / 2) + ch * 32;
                 uint32_t ov[32];
                 __syncwarp();
-                tmem_ld32(tmem + lane_base + kTmemO + ch * 32, ov);
+                tmem_ld32(tmem + lane_base + kTmemO + col, ov);
                 if (row_valid) {
-                    uint32_t w[16];
+                    uint32_t wv[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e)
-                        w[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * args.inv_n,
-                                           __uint_as_float(ov[2 * e + 1]) * args.inv_n);
-                    uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+                        wv[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * args.inv_n,
+                                            __uint_as_float(ov[2 * e + 1]) * args.inv_n);
+                    uint4* dst = reinterpret_cast<uint4*>(orow + col);
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
-                        dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+                        dst[q] = make_uint4(wv[4 * q], wv[4 * q + 1], wv[4 * q + 2], wv[4 * q + 3]);
                 }
             }
         }
@@ -401,7 +495,7 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
     tc_fence_before();
     __syncthreads();
     if (tid == 0 && *abort_flag) raise_error(kErrTimeout);
-    if (warp == 5) {
+    if (warp == kWarpMMA) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }

@@ -29,10 +29,26 @@ __device__ __forceinline__ int time_bucket64(int64_t dt, int nb_minus_1) {
     return min(msb, nb_minus_1);
 }
 
+// Biased exponent of x (1 <= x < 2^32) as a double: 1023 + floor(log2(x)).
+// The double 2^52 + x is formed exactly by writing x into the low word of
+// 2^52; subtracting 2^52 leaves x exactly, so the exponent field is the bit
+// length of x minus one plus the bias. Runs on the FP64 pipe instead of the
+// shared bit-find/transcendental unit.
+__device__ __forceinline__ uint32_t log2_exponent_field(uint32_t x) {
+    uint32_t hi;
+    asm("{\n\t.reg .f64 t;\n\t.reg .b32 lo;\n\t"
+        "mov.b64 t, {%1, %2};\n\t"
+        "sub.rn.f64 t, t, 0d4330000000000000;\n\t"
+        "mov.b64 {lo, %0}, t;\n\t}"
+        : "=r"(hi)
+        : "r"(x), "r"(0x43300000u));
+    return hi >> 20;
+}
+
 // Same bucket for a difference already known to fit in int32.
 __device__ __forceinline__ int time_bucket32(int32_t dt, int nb_minus_1) {
-    const int x = max(dt, 1);
-    return min(31 - __clz(x), nb_minus_1);
+    const int k = static_cast<int>(log2_exponent_field(static_cast<uint32_t>(max(dt, 1)))) - 1023;
+    return min(k, nb_minus_1);
 }
 
 // Relative-position index min(i - j, P - 1), clamped at 0 for pairs that the
