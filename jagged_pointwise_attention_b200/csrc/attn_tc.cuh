@@ -9,24 +9,27 @@
 // max, no rescale, no row sum, so O accumulates untouched across key tiles
 // and the whole per-element budget goes to the bias gathers and the SiLU.
 //
-// Warp roles (352 threads):
-//   warps 0-7  pointwise stage: warp w owns TMEM lanes 32*(w%4).. (one query
-//              row per thread) and S columns 64*(w/4)..+63
-//   warp 8     TMA producers: lane 0 loads Q and the K ring, lane 1 the V ring
+// Warp roles ((4G + 3) warps for G pointwise groups):
+//   warps 0..4G-1  pointwise stage in G groups of 4 warps. Group g handles the
+//              key tiles j = g (mod G) in its own S buffer, so the G warps that
+//              share an SM sub-partition work on different tiles and hide each
+//              other's TMEM, MUFU and barrier latencies. Warp w owns TMEM lanes
+//              32*(w%4).. (one query row per thread) and all 128 columns.
+//   warp 4G    TMA producers: lane 0 loads Q and the K ring, lane 1 the V ring
 //              (2 stages each; K_j+2 is fetched as soon as S_j is done, V_j+2
 //              as soon as PV_j is done)
-//   warp 9     MMA issuer (one thread) and TMEM owner
-//   warp 10    bias staging: per key tile, key timestamps (int64 and their low
+//   warp 4G+1  MMA issuer (one thread) and TMEM owner
+//   warp 4G+2  bias staging: per key tile, key timestamps (int64 and their low
 //              32 bits), tile min/max and monotonicity, and the window of the
 //              relative-position table the tile needs, one stage per S buffer
-// TMEM (512 columns): S double buffer at 0 and 128, O at 256. P_j overwrites
-// the S_j buffer it came from: the warp that read S columns 64h..64h+63 writes
-// their 64 bf16 results into columns 64h..64h+31 (two per 32-bit column), so
-// no warp writes columns another warp still has to read.
+// TMEM (512 columns): S buffers at 128g, O at 128G. P_j overwrites the S_j
+// buffer it came from, chunk by chunk: after a thread has read S columns
+// 32c..32c+31 of its row it writes their 32 bf16 results into columns
+// 32c..32c+15 (two per 32-bit column).
 //
-// Per key tile the pointwise warps wait once (S_j and its bias stage ready)
-// and arrive once (P_j written); the MMA issues PV_j and then S_j+2 into the
-// same buffer, in order.
+// Per key tile a group waits once (S_j and its bias stage ready) and arrives
+// once (P_j written); the MMA issues PV_j and later S_j+G into the same
+// buffer, in order.
 //
 // Pointwise arithmetic per score, with h = x/2 folded into the bias adds:
 //   h = s/2 + pos/2 + time/2;  silu(x) = h + h*tanh(h)  (packed bf16x2, one
@@ -62,12 +65,16 @@ struct AttnArgs {
     int64_t out_stride;         // elements per token
 };
 
-constexpr int kPointwiseWarps = 8;
-constexpr int kPointwiseThreads = kPointwiseWarps * 32;
-constexpr int kWarpTMA = 8, kWarpMMA = 9, kWarpMeta = 10;
-constexpr int kAttnThreads = 11 * 32;
+constexpr int kAttnGroups = 3;          // pointwise groups (S buffers)
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemO = 256;
+
+template <int G>
+struct AttnRoles {
+    static constexpr int kPointwiseWarps = 4 * G;
+    static constexpr int kWarpTMA = 4 * G, kWarpMMA = 4 * G + 1, kWarpMeta = 4 * G + 2;
+    static constexpr int kThreads = (4 * G + 3) * 32;
+    static constexpr uint32_t kTmemO = 128 * G;
+};
 
 // One stage of staged bias data for one key tile.
 struct MetaStage {
@@ -79,7 +86,7 @@ struct MetaStage {
     int32_t pad[3];
 };
 
-template <int D>
+template <int D, int G>
 struct AttnSmem {
     static constexpr int kQBytes = kTile * D * 2;       // Q tile, D/64 swizzled 16 KB blocks
     static constexpr int kKVBytes = kTile * D * 2;      // one K (or V) stage
@@ -87,8 +94,8 @@ struct AttnSmem {
     static constexpr int kOffK = kOffQ + kQBytes;
     static constexpr int kOffV = kOffK + 2 * kKVBytes;
     static constexpr int kOffTB = kOffV + 2 * kKVBytes;                 // float[kMaxTimeBuckets]
-    static constexpr int kOffMeta = kOffTB + kMaxTimeBuckets * 4;       // MetaStage[2]
-    static constexpr int kOffBar = kOffMeta + 2 * static_cast<int>(sizeof(MetaStage));
+    static constexpr int kOffMeta = kOffTB + kMaxTimeBuckets * 4;       // MetaStage[G]
+    static constexpr int kOffBar = kOffMeta + G * static_cast<int>(sizeof(MetaStage));
     static constexpr int kNumBars = 32;
     static constexpr int kOffTmem = kOffBar + kNumBars * 8;
     static constexpr int kOffAbort = kOffTmem + 8;
@@ -103,10 +110,10 @@ enum {
     kBarKFree = 3,      // +stage (2)
     kBarVFull = 5,      // +stage (2)
     kBarVFree = 7,      // +stage (2)
-    kBarSFull = 9,      // +buffer (2): MMA commit + 32 bias-staging lanes
-    kBarPFull = 11,     // +buffer (2): 256 pointwise threads
-    kBarOFull = 13,
-    kBarDrain = 14,
+    kBarSFull = 9,      // +buffer (G <= 3): MMA commit + 32 bias-staging lanes
+    kBarPFull = 12,     // +buffer (G <= 3): the 128 threads of the buffer's group
+    kBarOFull = 15,
+    kBarDrain = 16,
 };
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
@@ -196,14 +203,17 @@ __device__ __forceinline__ void pw_slow(const uint32_t* sv, int c0,
     }
 }
 
-template <int D>
-__global__ void __launch_bounds__(kAttnThreads, 1)
+template <int D, int G>
+__global__ void __launch_bounds__(AttnRoles<G>::kThreads, 1)
 attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                      const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const AttnArgs args) {
-    using L = AttnSmem<D>;
+    using L = AttnSmem<D, G>;
+    using R = AttnRoles<G>;
     static_assert(D == 64 || D == 128, "head dim");
+    static_assert(G >= 1 && G <= 3 && 128 * G + D <= static_cast<int>(kTmemCols), "TMEM budget");
     constexpr int kKB = D / 64;   // 64-element (128-byte) column blocks per row
+    constexpr uint32_t kTmemO = R::kTmemO;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -235,19 +245,21 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
             mbar_init(&bars[kBarKFree + s], 1);
             mbar_init(&bars[kBarVFull + s], 1);
             mbar_init(&bars[kBarVFree + s], 1);
-            mbar_init(&bars[kBarSFull + s], 1 + 32);
-            mbar_init(&bars[kBarPFull + s], kPointwiseThreads);
+        }
+        for (int b = 0; b < G; ++b) {
+            mbar_init(&bars[kBarSFull + b], 1 + 32);
+            mbar_init(&bars[kBarPFull + b], 128);
         }
         mbar_init(&bars[kBarOFull], 1);
         mbar_init(&bars[kBarDrain], 1);
         mbar_fence_init();
     }
-    if (warp == kWarpMMA) {
+    if (warp == R::kWarpMMA) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
-    if (tid < kPointwiseThreads) {
-        for (int b = tid; b < kMaxTimeBuckets; b += kPointwiseThreads)
+    if (warp < R::kPointwiseWarps) {
+        for (int b = tid; b < kMaxTimeBuckets; b += 32 * R::kPointwiseWarps)
             tb_s[b] = (use_time && b < args.NB) ? 0.5f * args.tb[static_cast<int64_t>(h) * args.NB + b] : 0.f;
     }
     tc_fence_before();
@@ -259,7 +271,7 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
     const uint32_t sK = smem_u32(smem + L::kOffK);
     const uint32_t sV = smem_u32(smem + L::kOffV);
 
-    if (warp == kWarpTMA) {
+    if (warp == R::kWarpTMA) {
         // ------------------------------------------------------------ TMA producers
         if (lane < 2) {
             const bool is_k = lane == 0;
@@ -293,61 +305,70 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
             if (issued1 > 0 && !mbar_wait(&full[1], (issued1 - 1) & 1, nullptr)) raise_error(kErrTimeout);
         }
         __syncwarp();
-    } else if (warp == kWarpMMA) {
+    } else if (warp == R::kWarpMMA) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
             auto issue_pv = [&](int jj) -> bool {
-                const int sb = jj & 1;
-                if (!mbar_wait(&bars[kBarPFull + sb], (jj >> 1) & 1, abort_flag)) return false;
-                if (!mbar_wait(&bars[kBarVFull + sb], (jj >> 1) & 1, abort_flag)) return false;
+                const int b = jj % G;
+                const int sv = jj & 1;
+                if (!mbar_wait(&bars[kBarPFull + b], (jj / G) & 1, abort_flag)) return false;
+                if (!mbar_wait(&bars[kBarVFull + sv], (jj >> 1) & 1, abort_flag)) return false;
                 tc_fence_after();
-                const uint32_t vb = sV + sb * L::kKVBytes;
-                const uint32_t pb = tmem + sb * 128;
+                const uint32_t vb = sV + sv * L::kKVBytes;
+                const uint32_t pb = tmem + b * 128;
 #pragma unroll
                 for (int kk = 0; kk < kTile / 16; ++kk) {
-                    // keys 16kk..16kk+15: columns (kk/4)*64 + (kk%4)*8 of the P buffer
-                    const uint32_t a = pb + (kk >> 2) * 64 + (kk & 3) * 8;
-                    const uint64_t b = desc_mnmajor_sw128(vb + kk * 2048, 16384);
-                    umma_bf16_ts(tmem + kTmemO, a, b, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
+                    // keys 16kk..16kk+15: columns 32*(kk/2) + 8*(kk%2) of the P buffer
+                    const uint32_t a = pb + (kk >> 1) * 32 + (kk & 1) * 8;
+                    const uint64_t bd = desc_mnmajor_sw128(vb + kk * 2048, 16384);
+                    umma_bf16_ts(tmem + kTmemO, a, bd, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
                 }
-                umma_commit(&bars[kBarVFree + sb]);
+                umma_commit(&bars[kBarVFree + sv]);
                 return true;
             };
             bool ok = mbar_wait(&bars[kBarQFull], 0, abort_flag);
+            int pv_next = 0;
             for (int j = 0; ok && j < nk; ++j) {
                 const int s = j & 1;
-                // buffer s last held P_j-2, read by PV_j-2, issued earlier by this thread
+                // buffer j%G last held P_j-G, read by PV_j-G, issued earlier by this thread
                 ok = mbar_wait(&bars[kBarKFull + s], (j >> 1) & 1, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t kb_base = sK + s * L::kKVBytes;
+                const uint32_t sb = tmem + (j % G) * 128;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    umma_bf16_ss(tmem + s * 128, desc_kmajor_sw128(sQ + off),
-                                 desc_kmajor_sw128(kb_base + off), idesc_qk, kk > 0 ? 1u : 0u);
+                    umma_bf16_ss(sb, desc_kmajor_sw128(sQ + off), desc_kmajor_sw128(kb_base + off),
+                                 idesc_qk, kk > 0 ? 1u : 0u);
                 }
-                umma_commit(&bars[kBarSFull + s]);
+                umma_commit(&bars[kBarSFull + j % G]);
                 umma_commit(&bars[kBarKFree + s]);
-                if (j >= 1) ok = issue_pv(j - 1);
+                if (j >= G - 1) {
+                    ok = issue_pv(pv_next);
+                    ++pv_next;
+                }
             }
-            if (ok) ok = issue_pv(nk - 1);
+            while (ok && pv_next < nk) {
+                ok = issue_pv(pv_next);
+                ++pv_next;
+            }
             if (ok) umma_commit(&bars[kBarOFull]);
             umma_commit(&bars[kBarDrain]);
             if (!mbar_wait(&bars[kBarDrain], 0, nullptr)) raise_error(kErrTimeout);
         }
         __syncwarp();
-    } else if (warp == kWarpMeta) {
+    } else if (warp == R::kWarpMeta) {
         // ------------------------------------------------------------ bias staging
         for (int j = 0; j < nk; ++j) {
-            const int s = j & 1;
-            // stage s last served tile j-2; P_j-2 written means it has been read
-            if (j >= 2 && !warp_wait(&bars[kBarPFull + s], ((j >> 1) - 1) & 1, abort_flag)) break;
-            MetaStage& ms = meta[s];
+            const int b = j % G;
+            // stage b last served tile j-G; P_j-G written means it has been read
+            if (j >= G && !warp_wait(&bars[kBarPFull + b], ((j / G) - 1) & 1, abort_flag)) break;
+            MetaStage& ms = meta[b];
             const int kt0 = k0 + j * kTile;
-            // relative-position window, pre-halved (4 + 4 independent loads per lane)
+            // relative-position window, pre-halved (8 + 4 independent loads per lane)
             float wv[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
@@ -389,9 +410,9 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
                 const int64_t a = __shfl_xor_sync(0xffffffffu, tmin, o);
-                const int64_t b = __shfl_xor_sync(0xffffffffu, tmax, o);
+                const int64_t c = __shfl_xor_sync(0xffffffffu, tmax, o);
                 tmin = a < tmin ? a : tmin;
-                tmax = b > tmax ? b : tmax;
+                tmax = c > tmax ? c : tmax;
             }
             if (lane == 0) {
                 ms.tmin = tmin;
@@ -399,12 +420,12 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                 ms.mono = mono ? 1 : 0;
             }
             __syncwarp();
-            mbar_arrive(&bars[kBarSFull + s]);
+            mbar_arrive(&bars[kBarSFull + b]);
         }
     } else {
         // ------------------------------------------------------------ pointwise stage
+        const int g = warp >> 2;                            // group: tiles j = g (mod G)
         const int qd = warp & 3;                            // TMEM lane quarter
-        const int half = warp >> 2;                         // S columns 64*half..
         const int r = qd * 32 + lane;                       // query row = TMEM lane
         const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
         const int64_t i = static_cast<int64_t>(q0) + r;
@@ -413,13 +434,13 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
         const int32_t ti32 = static_cast<int32_t>(static_cast<uint64_t>(ti));
         // register table: lane L holds time/2 of bucket min((L + 1) mod 32, NB - 1)
         const float tbr = tb_s[min((lane + 1) & 31, nbm1)];
+        const MetaStage& ms = meta[g];
+        const uint32_t s_col = tmem + lane_base + static_cast<uint32_t>(g * 128);
         bool ok = true;
-        for (int j = 0; j < nk; ++j) {
-            const int s = j & 1;
-            ok = warp_wait(&bars[kBarSFull + s], (j >> 1) & 1, abort_flag);
+        for (int j = g; j < nk; j += G) {
+            ok = warp_wait(&bars[kBarSFull + g], (j / G) & 1, abort_flag);
             if (!ok) break;
             tc_fence_after();
-            const MetaStage& ms = meta[s];
             const int kt0 = k0 + j * kTile;
             const int lo = k0 - kt0;                        // first key of the sequence
             const int hi = row_valid ? static_cast<int>(i - kt0) : -1;
@@ -432,48 +453,46 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
             const bool fast_w = __all_sync(0xffffffffu, fast);
             const bool mono = ms.mono != 0;
             const float* wrow = ms.w + 127 + r;
-            const uint32_t s_col = tmem + lane_base + static_cast<uint32_t>(s * 128 + half * 64);
-            uint32_t sv[64];
-            __syncwarp();
-            tmem_ld64(s_col, sv);
-            uint32_t pk[32];
-            // one 32-column chunk of this warp's 64 columns -> 16 packed P words
-            auto chunk = [&](int q, uint32_t* pkc) {
-                const uint32_t* svc = sv + 32 * q;
-                const int c0 = half * 64 + 32 * q;
+#pragma unroll 1
+            for (int q = 0; q < 4; ++q) {
+                const int c0 = 32 * q;
+                uint32_t sv[32];
+                uint32_t pk[16];
+                __syncwarp();
+                tmem_ld32(s_col + c0, sv);
                 const bool full = __all_sync(0xffffffffu, lo <= c0 && hi >= c0 + 31);
+                bool done = false;
                 if (!fast_w) {
-                    if (full) pw_slow<false>(svc, c0, wrow, ms.kt64, ti, tb_s, nbm1, lo, hi, pkc);
-                    else pw_slow<true>(svc, c0, wrow, ms.kt64, ti, tb_s, nbm1, lo, hi, pkc);
-                    return;
-                }
-                if (full && mono) {
+                    if (full) pw_slow<false>(sv, c0, wrow, ms.kt64, ti, tb_s, nbm1, lo, hi, pk);
+                    else pw_slow<true>(sv, c0, wrow, ms.kt64, ti, tb_s, nbm1, lo, hi, pk);
+                    done = true;
+                } else if (full && mono) {
                     const uint32_t ef0 = log2_exponent_field(static_cast<uint32_t>(max(
                         static_cast<int32_t>(static_cast<uint32_t>(ti32) - static_cast<uint32_t>(ms.kt32[c0])), 1)));
                     const uint32_t ef1 = log2_exponent_field(static_cast<uint32_t>(max(
                         static_cast<int32_t>(static_cast<uint32_t>(ti32) - static_cast<uint32_t>(ms.kt32[c0 + 31])), 1)));
                     const float tconst = __shfl_sync(0xffffffffu, tbr, static_cast<int>(ef0));
                     if (__all_sync(0xffffffffu, ef0 == ef1)) {
-                        pw_const<false>(svc, c0, wrow, tconst, lo, hi, pkc);
-                        return;
+                        pw_const<false>(sv, c0, wrow, tconst, lo, hi, pk);
+                        done = true;
                     }
                 }
-                if (full) pw_fast<false>(svc, c0, wrow, ms.kt32, ti32, tbr, lo, hi, pkc);
-                else pw_fast<true>(svc, c0, wrow, ms.kt32, ti32, tbr, lo, hi, pkc);
-            };
-            chunk(0, pk);
-            chunk(1, pk + 16);
-            // P (64 bf16 of this row) -> columns 64h..64h+31 of the S buffer just read
-            tmem_st32(s_col, pk);
+                if (!done) {
+                    if (full) pw_fast<false>(sv, c0, wrow, ms.kt32, ti32, tbr, lo, hi, pk);
+                    else pw_fast<true>(sv, c0, wrow, ms.kt32, ti32, tbr, lo, hi, pk);
+                }
+                // 32 bf16 results -> columns 32q..32q+15 of the S buffer just read
+                tmem_st16(s_col + c0, pk);
+            }
             tc_fence_before();
-            mbar_arrive(&bars[kBarPFull + s]);
+            mbar_arrive(&bars[kBarPFull + g]);
         }
-        if (ok && warp_wait(&bars[kBarOFull], 0, abort_flag)) {
+        if (g < 2 && ok && warp_wait(&bars[kBarOFull], 0, abort_flag)) {
             tc_fence_after();
             __nv_bfloat16* orow = args.out + i * args.out_stride + static_cast<int64_t>(h) * D;
 #pragma unroll
             for (int ch = 0; ch < D / 64; ++ch) {
-                const int col = half * (D / 2) + ch * 32;
+                const int col = g * (D / 2) + ch * 32;
                 uint32_t ov[32];
                 __syncwarp();
                 tmem_ld32(tmem + lane_base + kTmemO + col, ov);
@@ -495,7 +514,7 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
     tc_fence_before();
     __syncthreads();
     if (tid == 0 && *abort_flag) raise_error(kErrTimeout);
-    if (warp == kWarpMMA) {
+    if (warp == R::kWarpMMA) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }

@@ -185,17 +185,18 @@ hstu_status_t run_attn(const AttnCall& c) {
                c.os};
     const int64_t grid = max_units * c.H;
     if (grid > 0x7fffffff) return HSTU_ERR_UNSUPPORTED;
+    constexpr int G = kAttnGroups;
     static int smem_done64[kMaxDevices] = {0}, smem_done128[kMaxDevices] = {0};
     if (c.dqk == 64) {
-        if (!ensure_smem(attn_fwd_bf16_kernel<64>, AttnSmem<64>::kAlloc, smem_done64))
+        if (!ensure_smem(attn_fwd_bf16_kernel<64, G>, AttnSmem<64, G>::kAlloc, smem_done64))
             return HSTU_ERR_CUDA;
-        attn_fwd_bf16_kernel<64><<<static_cast<unsigned>(grid), kAttnThreads, AttnSmem<64>::kAlloc,
-                                   c.stream>>>(tq, tk, tv, a);
+        attn_fwd_bf16_kernel<64, G><<<static_cast<unsigned>(grid), AttnRoles<G>::kThreads,
+                                      AttnSmem<64, G>::kAlloc, c.stream>>>(tq, tk, tv, a);
     } else {
-        if (!ensure_smem(attn_fwd_bf16_kernel<128>, AttnSmem<128>::kAlloc, smem_done128))
+        if (!ensure_smem(attn_fwd_bf16_kernel<128, G>, AttnSmem<128, G>::kAlloc, smem_done128))
             return HSTU_ERR_CUDA;
-        attn_fwd_bf16_kernel<128><<<static_cast<unsigned>(grid), kAttnThreads,
-                                    AttnSmem<128>::kAlloc, c.stream>>>(tq, tk, tv, a);
+        attn_fwd_bf16_kernel<128, G><<<static_cast<unsigned>(grid), AttnRoles<G>::kThreads,
+                                       AttnSmem<128, G>::kAlloc, c.stream>>>(tq, tk, tv, a);
     }
     return launch_status();
 }
