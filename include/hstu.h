@@ -131,6 +131,42 @@ hstu_status_t hstu_attn_fwd(hstu_dtype_t dtype,
                             void* out, int64_t out_tok_stride,
                             void* workspace, size_t workspace_bytes, void* stream);
 
+/* hstu_attn_fwd for callers that cannot allocate device memory when they run
+ * the attention, such as an inference-engine plugin whose enqueue step must
+ * not call cudaMalloc (it can synchronise the device and fail under memory
+ * pressure), or code that has no allocator at hand. The paper has no
+ * counterpart: this is an interface convenience of this library.
+ *
+ * Same arguments, layouts and results as hstu_attn_fwd, minus the workspace:
+ * the bf16 path keeps its work list in a file-scope device array of
+ * HSTU_NOALLOC_SCRATCH_BYTES (1 MiB), which every GPU that loads the library
+ * holds until the process exits. A batch needing more than that, i.e.
+ * hstu_attn_workspace_bytes(B, total_tokens, max_seqlen) > 1 MiB (about 65,500
+ * sequence-tiles: roughly B + total_tokens/128 > 65,519), returns
+ * HSTU_ERR_UNSUPPORTED before anything is launched; use hstu_attn_fwd then.
+ * Nothing is allocated or freed by this call, including by torch or any
+ * other library.
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream
+ * capture. Every call shares the one array and it keeps the last call's
+ * contents; the plan kernel rewrites the unit count and every unit it lists
+ * before the attention kernel reads them, so nothing has to be cleared. Calls
+ * whose executions overlap on the GPU (other streams, or graphs replayed
+ * concurrently) race on the array. */
+#define HSTU_NOALLOC_SCRATCH_BYTES 1048576
+hstu_status_t hstu_attn_fwd_noalloc(hstu_dtype_t dtype,
+                                    const void* q, int64_t q_tok_stride,
+                                    const void* k, int64_t k_tok_stride,
+                                    const void* v, int64_t v_tok_stride,
+                                    const int64_t* seq_offsets, int32_t B, int64_t total_tokens,
+                                    int32_t H, int32_t d_qk, int32_t d_v,
+                                    const int64_t* timestamps,
+                                    const float* pos_bias, int32_t num_pos,
+                                    const float* time_bias, int32_t num_time_buckets,
+                                    int32_t max_seqlen,
+                                    void* out, int64_t out_tok_stride, void* stream);
+
 /* Test hook: for every sequence b, every i and every j <= i (sequence by
  * sequence, row-major in i then j) writes the relative-position index
  * min(i-j, num_pos-1) and the time bucket, computed by the same device

@@ -25,6 +25,9 @@ SIGNATURES = {
     "hstu_attn_fwd": (ctypes.c_int, [ctypes.c_int, c_p, c_i64, c_p, c_i64, c_p, c_i64, c_p, c_i32,
                                      c_i64, c_i32, c_i32, c_i32, c_p, c_p, c_i32, c_p, c_i32,
                                      c_i32, c_p, c_i64, c_p, c_sz, c_p]),
+    "hstu_attn_fwd_noalloc": (ctypes.c_int, [ctypes.c_int, c_p, c_i64, c_p, c_i64, c_p, c_i64,
+                                             c_p, c_i32, c_i64, c_i32, c_i32, c_i32, c_p, c_p,
+                                             c_i32, c_p, c_i32, c_i32, c_p, c_i64, c_p]),
     "hstu_debug_bias_indices": (ctypes.c_int, [c_p, c_i32, c_i64, c_p, c_i32, c_i32, c_p, c_p,
                                                c_p]),
     "hstu_debug_wait_timeout": (ctypes.c_int, [c_i32, c_p]),

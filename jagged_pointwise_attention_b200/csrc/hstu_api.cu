@@ -460,3 +460,61 @@ hstu_status_t hstu_layer_fwd(const void* x, int64_t total_tokens, int32_t D, con
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Attention without any allocation by the library or the caller.
+//
+// Some callers cannot allocate device memory at the moment they run the
+// attention: an inference-engine plugin whose enqueue step must not call
+// cudaMalloc (it can synchronise the device and can fail under memory
+// pressure), or glue code that holds no allocator at all. For them the
+// scratch that hstu_attn_fwd takes as `workspace` (the work list of the plan
+// kernel) lives in this file-scope device array instead. Every GPU that loads
+// the library holds it until the process exits.
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[HSTU_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kMaxDevices] = {nullptr};
+
+// Device address of this device's scratch array. In host code the array's
+// name only stands in for the symbol, so the address is looked up once per
+// device, with that device current, and cached.
+hstu_status_t noalloc_scratch(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HSTU_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+            return HSTU_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return HSTU_OK;
+}
+
+}  // namespace
+
+extern "C" hstu_status_t hstu_attn_fwd_noalloc(
+    hstu_dtype_t dtype, const void* q, int64_t q_tok_stride, const void* k, int64_t k_tok_stride,
+    const void* v, int64_t v_tok_stride, const int64_t* seq_offsets, int32_t B,
+    int64_t total_tokens, int32_t H, int32_t d_qk, int32_t d_v, const int64_t* timestamps,
+    const float* pos_bias, int32_t num_pos, const float* time_bias, int32_t num_time_buckets,
+    int32_t max_seqlen, void* out, int64_t out_tok_stride, void* stream) {
+    void* scratch = nullptr;
+    if (dtype == HSTU_DTYPE_BF16 && B > 0 && total_tokens > 0) {
+        const size_t need = hstu_attn_workspace_bytes(B, total_tokens, max_seqlen);
+        if (need == 0) return HSTU_ERR_INVALID_ARG;
+        if (need > HSTU_NOALLOC_SCRATCH_BYTES) return HSTU_ERR_UNSUPPORTED;
+        const hstu_status_t st = noalloc_scratch(&scratch);
+        if (st != HSTU_OK) return st;
+    }
+    return hstu_attn_fwd(dtype, q, q_tok_stride, k, k_tok_stride, v, v_tok_stride, seq_offsets, B,
+                         total_tokens, H, d_qk, d_v, timestamps, pos_bias, num_pos, time_bias,
+                         num_time_buckets, max_seqlen, out, out_tok_stride, scratch,
+                         scratch ? HSTU_NOALLOC_SCRATCH_BYTES : 0, stream);
+}
+
