@@ -90,7 +90,25 @@ int64_t max_units_of(int32_t B, int64_t T, int32_t max_seqlen) {
     return by_tokens < by_lengths ? by_tokens : by_lengths;
 }
 
-constexpr size_t kAttnWsHeader = 256;   // unit count, padded
+constexpr size_t kAttnWsHeader = 256;   // unit count (int at 0), item counters (2 ints at 16)
+
+// attention workspace: [header][units: int4 x max_units][row_start: int32 x T]
+size_t attn_units_bytes(int32_t B, int64_t T, int32_t max_seqlen) {
+    return (static_cast<size_t>(max_units_of(B, T, max_seqlen)) * 16 + 255) / 256 * 256;
+}
+
+int num_sms() {
+    static int cached[kMaxDevices] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -133,6 +151,7 @@ hstu_status_t validate_attn(const AttnCall& c) {
     if (c.tb && (c.NB < 1 || c.NB > kMaxTimeBuckets)) return HSTU_ERR_INVALID_ARG;
     if (c.dtype == HSTU_DTYPE_BF16) {
         if (c.dqk != c.dv || (c.dqk != 64 && c.dqk != 128)) return HSTU_ERR_UNSUPPORTED;
+        if (c.H > kMaxHeadsTable) return HSTU_ERR_UNSUPPORTED;
         if (!aligned16(c.q) || !aligned16(c.k) || !aligned16(c.v) || !aligned16(c.out))
             return HSTU_ERR_INVALID_ARG;
         if (c.qs % 8 || c.ks % 8 || c.vs % 8 || c.os % 8) return HSTU_ERR_INVALID_ARG;
@@ -173,6 +192,9 @@ hstu_status_t run_attn(const AttnCall& c) {
     const uint8_t* ws = static_cast<const uint8_t*>(c.ws);
     AttnArgs a{reinterpret_cast<const int4*>(ws + kAttnWsHeader),
                reinterpret_cast<const int*>(ws),
+               reinterpret_cast<int*>(const_cast<uint8_t*>(ws) + 16),
+               reinterpret_cast<const int*>(ws + kAttnWsHeader +
+                                            attn_units_bytes(c.B, c.T, c.max_seqlen)),
                c.H,
                c.T,
                use_time ? c.ts : nullptr,
@@ -183,20 +205,22 @@ hstu_status_t run_attn(const AttnCall& c) {
                inv_n,
                static_cast<__nv_bfloat16*>(c.out),
                c.os};
-    const int64_t grid = max_units * c.H;
-    if (grid > 0x7fffffff) return HSTU_ERR_UNSUPPORTED;
+    const int64_t items = max_units * c.H;
+    if (items > 0x7fffffff) return HSTU_ERR_UNSUPPORTED;
+    // persistent: one CTA per SM, work items dealt round-robin
+    const unsigned grid = static_cast<unsigned>(items < num_sms() ? items : num_sms());
     constexpr int G = kAttnGroups;
     static int smem_done64[kMaxDevices] = {0}, smem_done128[kMaxDevices] = {0};
     if (c.dqk == 64) {
         if (!ensure_smem(attn_fwd_bf16_kernel<64, G>, AttnSmem<64, G>::kAlloc, smem_done64))
             return HSTU_ERR_CUDA;
-        attn_fwd_bf16_kernel<64, G><<<static_cast<unsigned>(grid), AttnRoles<G>::kThreads,
-                                      AttnSmem<64, G>::kAlloc, c.stream>>>(tq, tk, tv, a);
+        attn_fwd_bf16_kernel<64, G><<<grid, AttnCfg<64, G>::kThreads, AttnSmem<64, G>::kAlloc,
+                                      c.stream>>>(tq, tk, tv, a);
     } else {
         if (!ensure_smem(attn_fwd_bf16_kernel<128, G>, AttnSmem<128, G>::kAlloc, smem_done128))
             return HSTU_ERR_CUDA;
-        attn_fwd_bf16_kernel<128, G><<<static_cast<unsigned>(grid), AttnRoles<G>::kThreads,
-                                       AttnSmem<128, G>::kAlloc, c.stream>>>(tq, tk, tv, a);
+        attn_fwd_bf16_kernel<128, G><<<grid, AttnCfg<128, G>::kThreads, AttnSmem<128, G>::kAlloc,
+                                       c.stream>>>(tq, tk, tv, a);
     }
     return launch_status();
 }
@@ -210,9 +234,13 @@ hstu_status_t plan_attn(const int64_t* off, int32_t B, int64_t T, int32_t max_se
     const int max_tiles = max_tiles_of(max_seqlen);
     const int64_t max_units = max_units_of(B, T, max_seqlen);
     uint8_t* w = static_cast<uint8_t*>(ws);
-    plan_kernel<<<1, 1024, 3 * max_tiles * sizeof(int), stream>>>(
-        off, B, max_seqlen, max_tiles, static_cast<int>(max_units),
-        reinterpret_cast<int4*>(w + kAttnWsHeader), reinterpret_cast<int*>(w));
+    size_t smem = static_cast<size_t>((3 * (max_tiles + 1) + 1) & ~1) * sizeof(int);
+    if (B < kPlanSmemOffsets) smem += static_cast<size_t>(B + 1) * sizeof(int64_t);
+    plan_kernel<<<1, 1024, smem, stream>>>(
+        off, B, T, max_seqlen, max_tiles, static_cast<int>(max_units),
+        reinterpret_cast<int4*>(w + kAttnWsHeader), reinterpret_cast<int*>(w),
+        reinterpret_cast<int*>(w + 16),
+        reinterpret_cast<int*>(w + kAttnWsHeader + attn_units_bytes(B, T, max_seqlen)));
     return launch_status();
 }
 
@@ -329,7 +357,8 @@ hstu_status_t hstu_device_status(void* stream) {
 
 size_t hstu_attn_workspace_bytes(int32_t B, int64_t total_tokens, int32_t max_seqlen) {
     if (!plan_sizes_ok(B, total_tokens, max_seqlen)) return 0;
-    return kAttnWsHeader + static_cast<size_t>(max_units_of(B, total_tokens, max_seqlen)) * 16;
+    return kAttnWsHeader + attn_units_bytes(B, total_tokens, max_seqlen) +
+           static_cast<size_t>(total_tokens) * sizeof(int);
 }
 
 hstu_status_t hstu_attn_plan(const int64_t* seq_offsets, int32_t B, int64_t total_tokens,

@@ -1,55 +1,96 @@
-// plan.cuh -- longest-first work list for the jagged attention.
+// plan.cuh -- work list of the jagged attention.
 //
-// A work unit is one 128-row query tile of one sequence: rows [q0, q_end),
-// keys from the sequence start k0, nk = t + 1 key tiles for query tile t
-// (tiles after the diagonal are skipped by causality). Units are listed by
-// descending nk, so the block scheduler hands out the longest units first
-// (greedy longest-processing-time order); heads are expanded by the kernel.
+// A work unit is a tile of at most 128 query rows with the key range it needs:
+// (q0, q_end, k0, nk | packed << 31). Two kinds:
+//  * aligned: query tile t of a sequence longer than 128 tokens: rows
+//    [o + 128t, min(o + 128t + 128, o + n)), keys from the sequence start
+//    k0 = o, nk = t + 1 key tiles (tiles past the diagonal are causally empty).
+//  * packed: several whole sequences of at most 128 tokens each, consecutive in
+//    the batch, sharing one tile: rows [q0, q_end) = keys, nk = 1. Each row's
+//    own sequence start is written to row_start[] so the kernel can mask pairs
+//    that cross a sequence boundary. Packing is greedy inside each 128-token
+//    bucket of sequence start positions, so buckets are packed in parallel.
+// Units are listed longest first (descending nk, aligned before packed), so
+// handing them out in list order is greedy longest-processing-time scheduling.
+//
+// Aligned units are placed without per-unit atomics: sequences are counting-
+// sorted by their tile count nt (descending); the sequences with nt > t are
+// then a prefix of that order, so unit (b, t) goes to slot
+// start[t] + rank(b) where start[t] counts the units of all tiles above t.
 #pragma once
 
 #include "common.cuh"
 
 namespace hstu {
 
-// One block. Shared memory: 3 * max_tiles ints.
+constexpr int kPlanSmemOffsets = 4096;    // offsets cached in shared memory below this B
+
+// One block of 1024 threads. Dynamic shared memory: 3 * (max_tiles + 1) ints,
+// then (B + 1) int64 offsets when B < kPlanSmemOffsets.
 __global__ void __launch_bounds__(1024)
-plan_kernel(const int64_t* __restrict__ seq_offsets, int B, int max_seqlen, int max_tiles,
-            int max_units, int4* __restrict__ units, int* __restrict__ unit_count) {
+plan_kernel(const int64_t* __restrict__ seq_offsets, int B, int64_t T, int max_seqlen,
+            int max_tiles, int max_units, int4* __restrict__ units, int* __restrict__ unit_count,
+            int* __restrict__ item_counter, int* __restrict__ row_start) {
     extern __shared__ int plan_smem[];
-    int* hist = plan_smem;               // units with query tile t
-    int* start = hist + max_tiles;       // first list slot of tile t
-    int* fill = start + max_tiles;       // slots of tile t used so far
-    for (int t = threadIdx.x; t < max_tiles; t += blockDim.x) {
-        hist[t] = 0;
-        fill[t] = 0;
+    const int NT = max_tiles + 1;        // tile counts 0..max_tiles
+    int* cnt = plan_smem;                // sequences with nt == v
+    int* base = cnt + NT;                // first rank of nt == v in the descending order
+    int* start = base + NT;              // first slot of query tile t
+    __shared__ int n_aligned, n_packed;
+    const bool cache = B < kPlanSmemOffsets;
+    int64_t* off_s = reinterpret_cast<int64_t*>(plan_smem + ((3 * NT + 1) & ~1));
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+    for (int v = tid; v < NT; v += blockDim.x) cnt[v] = 0;
+    if (cache)
+        for (int b = tid; b <= B; b += blockDim.x) off_s[b] = seq_offsets[b];
+    if (tid == 0) {
+        n_packed = 0;
+        item_counter[0] = 0;   // next work item to hand out
+        item_counter[1] = 0;   // CTAs finished
     }
     __syncthreads();
-    for (int b = threadIdx.x; b < B; b += blockDim.x) {
-        int64_t n = seq_offsets[b + 1] - seq_offsets[b];
+    const int64_t* off = cache ? off_s : seq_offsets;
+    auto length = [&](int b) -> int64_t {
+        int64_t n = off[b + 1] - off[b];
         if (n < 0 || n > max_seqlen) {
             raise_error(kErrBadInput);
             n = n < 0 ? 0 : max_seqlen;
         }
-        const int nt = static_cast<int>((n + kTile - 1) / kTile);
-        for (int t = 0; t < nt; ++t) atomicAdd(&hist[t], 1);
+        return n;
+    };
+    auto tiles_of = [&](int64_t n) -> int {
+        return n > kTile ? static_cast<int>((n + kTile - 1) / kTile) : 0;   // 0: packed
+    };
+    // histogram of tile counts of the long sequences
+    for (int b = tid; b < B; b += blockDim.x) {
+        const int nt = tiles_of(length(b));
+        if (nt > 0) atomicAdd(&cnt[nt], 1);
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-        int acc = 0;
-        for (int t = max_tiles - 1; t >= 0; --t) {
-            start[t] = acc;
-            acc += hist[t];
+    if (tid == 0) {
+        int rank = 0, slots = 0, ge = 0;   // ge: sequences with nt > t
+        for (int v = max_tiles; v >= 1; --v) {
+            base[v] = rank;
+            rank += cnt[v];
         }
-        *unit_count = acc < max_units ? acc : max_units;
+        for (int t = max_tiles - 1; t >= 0; --t) {
+            ge += cnt[t + 1];
+            start[t] = slots;
+            slots += ge;
+        }
+        n_aligned = slots;
+        for (int v = 0; v < NT; ++v) cnt[v] = 0;   // reused as fill counters
     }
     __syncthreads();
-    for (int b = threadIdx.x; b < B; b += blockDim.x) {
-        const int64_t o = seq_offsets[b];
-        int64_t n = seq_offsets[b + 1] - o;
-        n = n < 0 ? 0 : (n > max_seqlen ? max_seqlen : n);
-        const int nt = static_cast<int>((n + kTile - 1) / kTile);
+    // aligned units: one rank per sequence, then its nt slots
+    for (int b = tid; b < B; b += blockDim.x) {
+        const int64_t n = length(b);
+        const int nt = tiles_of(n);
+        if (nt == 0) continue;
+        const int rank = base[nt] + atomicAdd(&cnt[nt], 1);
+        const int64_t o = off[b];
         for (int t = 0; t < nt; ++t) {
-            const int slot = start[t] + atomicAdd(&fill[t], 1);
+            const int slot = start[t] + rank;
             if (slot < max_units) {
                 const int64_t q0 = o + static_cast<int64_t>(t) * kTile;
                 const int64_t qe = q0 + kTile < o + n ? q0 + kTile : o + n;
@@ -57,6 +98,76 @@ plan_kernel(const int64_t* __restrict__ seq_offsets, int B, int max_seqlen, int 
                                         static_cast<int>(o), t + 1);
             }
         }
+    }
+    // packed units. The first non-empty short sequence of each 128-token start
+    // bucket packs the short sequences of its bucket greedily: once to count
+    // (slots reserved with one atomic per warp), once to write.
+    for (int b0 = warp * 32; b0 < B; b0 += nwarps * 32) {
+        const int b = b0 + lane;
+        bool first = false;
+        int64_t bucket = 0;
+        if (b < B) {
+            const int64_t n = length(b);
+            if (n > 0 && n <= kTile) {
+                bucket = off[b] / kTile;
+                first = true;
+                for (int c = b - 1; c >= 0; --c) {   // nearest earlier non-empty sequence
+                    if (off[c + 1] - off[c] == 0) continue;
+                    first = (off[c] / kTile) != bucket || (off[c + 1] - off[c]) > kTile;
+                    break;
+                }
+            }
+        }
+        // greedy pass; emit(k, ts0, te) is called for the k-th unit of the bucket
+        auto pack = [&](auto emit) {
+            int k = 0;
+            int64_t ts0 = -1, te = -1;
+            for (int c = b; c < B && off[c] / kTile == bucket; ++c) {
+                const int64_t nc = length(c);
+                if (nc == 0) continue;
+                if (nc > kTile) break;               // a long sequence ends the run
+                if (ts0 >= 0 && off[c] + nc - ts0 > kTile) {
+                    emit(k++, ts0, te);
+                    ts0 = -1;
+                }
+                if (ts0 < 0) ts0 = off[c];
+                te = off[c] + nc;
+            }
+            if (ts0 >= 0) emit(k++, ts0, te);
+            return k;
+        };
+        const int mine = first ? pack([](int, int64_t, int64_t) {}) : 0;
+        int incl = mine;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        int wbase = 0;
+        if (lane == 31) wbase = atomicAdd(&n_packed, incl);
+        wbase = __shfl_sync(0xffffffffu, wbase, 31);
+        if (first) {
+            const int my0 = wbase + incl - mine;
+            pack([&](int k, int64_t ts0, int64_t te) {
+                const int slot = n_aligned + my0 + k;
+                if (slot < max_units)
+                    units[slot] = make_int4(static_cast<int>(ts0), static_cast<int>(te),
+                                            static_cast<int>(ts0), static_cast<int>(0x80000001u));
+            });
+        }
+    }
+    // row_start of every short sequence's tokens, one warp per sequence (coalesced)
+    for (int b = warp; b < B; b += nwarps) {
+        const int64_t o = off[b];
+        const int64_t n = length(b);
+        if (n == 0 || n > kTile) continue;
+        for (int64_t i = o + lane; i < o + n; i += 32)
+            if (i < T) row_start[i] = static_cast<int>(o);
+    }
+    __syncthreads();
+    if (tid == 0) {
+        const int total = n_aligned + n_packed;
+        *unit_count = total < max_units ? total : max_units;
     }
 }
 
