@@ -4,8 +4,8 @@
 // times one head) from a global counter over a longest-first list -- greedy
 // longest-processing-time scheduling -- and streams their key tiles through one
 // continuous pipeline, so loads, tensor-core work and pointwise work of
-// consecutive items overlap. A scheduler lane fetches items ahead of time and
-// publishes them to every role through a ring in shared memory. For every key tile j:
+// consecutive items overlap. The K producer fetches items ahead of time and
+// publishes them to every other role through a ring in shared memory. For every key tile j:
 //     S_j  = Q K_j^T                         tcgen05.mma, SMEM x SMEM -> TMEM (fp32)
 //     P_j  = silu(S_j + pos + time) * mask   TMEM -> registers -> bf16 TMEM
 //     O   += P_j V_j                          tcgen05.mma, TMEM x SMEM -> TMEM (fp32)
@@ -13,7 +13,9 @@
 // softmax: no running max, no rescale, no row sum, so O accumulates untouched
 // across key tiles and the per-element budget goes to the bias gathers and SiLU.
 //
-// Warp roles ((4G + 3) warps for G pointwise groups):
+// Warp roles ((4G + 4) warps for G pointwise groups). Every role that blocks
+// on a barrier has a warp of its own: a lane suspended in a barrier wait holds
+// up the other lanes of its warp.
 //   warps 0..4G-1  pointwise stage in G groups of 4 warps. Counting the tiles a
 //              CTA processes as n = 0, 1, 2, ..., group g handles n = g (mod G)
 //              in its own S buffer, so the G warps that share an SM
@@ -21,10 +23,10 @@
 //              TMEM, MUFU and barrier latencies. Warp w owns TMEM lanes
 //              32*(w%4).. (one query row per thread) and all 128 columns. The
 //              group that handles an item's last tile also writes its output.
-//   warp 4G    TMA producers: lane 0 loads Q tiles and the K ring, lane 1 the
-//              V ring; lane 2 is the item scheduler
-//   warp 4G+1  MMA issuer (one thread) and TMEM owner
-//   warp 4G+2  bias staging: per key tile, key timestamps (int64 and low 32
+//   warp 4G    item scheduler and TMA producer of Q tiles and the K ring
+//   warp 4G+1  TMA producer of the V ring
+//   warp 4G+2  MMA issuer (one thread) and TMEM owner
+//   warp 4G+3  bias staging: per key tile, key timestamps (int64 and low 32
 //              bits), their min/max and monotonicity, the window of the
 //              relative-position table, and the query rows' timestamps and
 //              sequence starts; one stage per S buffer. Software-pipelined: the
@@ -90,8 +92,9 @@ struct AttnCfg {
     // (a second warp staging alternate tiles could wait a phase two steps ahead
     // of the barrier, which the parity test cannot tell from the one before).
     static constexpr int kMetaWarps = 1;
-    static constexpr int kWarpTMA = 4 * G, kWarpMMA = 4 * G + 1, kWarpMeta = 4 * G + 2;
-    static constexpr int kThreads = (4 * G + 2 + kMetaWarps) * 32;
+    static constexpr int kWarpK = 4 * G, kWarpV = 4 * G + 1, kWarpMMA = 4 * G + 2,
+                         kWarpMeta = 4 * G + 3;
+    static constexpr int kThreads = (4 * G + 3 + kMetaWarps) * 32;
     static constexpr int kStages = D == 64 ? 3 : 2;                     // Q, K and V rings
     static constexpr int kOBufs = 128 * G + 2 * D <= static_cast<int>(kTmemCols) ? 2 : 1;
     static constexpr uint32_t kTmemO = 128 * G;
@@ -295,7 +298,7 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
     float* tbh_s = reinterpret_cast<float*>(smem + L::kOffTB);
     MetaStage* meta = reinterpret_cast<MetaStage*>(smem + L::kOffMeta);
     volatile int* items = reinterpret_cast<volatile int*>(smem + L::kOffItems);
-    constexpr int kConsumers = 3 + C::kMetaWarps + C::kPointwiseWarps;   // K, V, MMA, bias, pointwise
+    constexpr int kConsumers = 2 + C::kMetaWarps + C::kPointwiseWarps;   // V, MMA, bias, pointwise
     const bool use_time = args.ts != nullptr && args.tb != nullptr && args.NB > 0;
     const int nbm1 = use_time ? args.NB - 1 : 0;
 
@@ -356,36 +359,10 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
         return true;
     };
 
-    if (warp == C::kWarpTMA) {
+    if (warp == C::kWarpK || warp == C::kWarpV) {
         // ------------------------------------------------------------ TMA producers
-        if (lane == 2) {
-            // item scheduler: greedy dynamic assignment from the global counter
-            for (int k = 0;; ++k) {
-                const int slot = k % kItemRing;
-                if (k >= kItemRing &&
-                    !mbar_wait(&bars[kBarItemFree + slot], ((k / kItemRing) - 1) & 1, abort_flag))
-                    break;
-                const int w = atomicAdd(args.item_counter, 1);
-                Item I;
-                if (w < n_items) {
-                    I = load_item(args, w);
-                } else {
-                    I.q0 = I.q_end = I.k0 = I.h = 0;
-                    I.nk = 0;
-                    I.packed = false;
-                }
-                volatile int* e = items + slot * 8;
-                e[0] = I.q0;
-                e[1] = I.q_end;
-                e[2] = I.k0;
-                e[3] = I.nk;
-                e[4] = I.h;
-                e[5] = I.packed ? 1 : 0;
-                mbar_arrive(&bars[kBarItemFull + slot]);
-                if (I.nk == 0) break;
-            }
-        } else if (lane < 2) {
-            const bool is_k = lane == 0;
+        if (lane == 0) {
+            const bool is_k = warp == C::kWarpK;
             const CUtensorMap* tm = is_k ? &tmK : &tmV;
             const int ring = is_k ? L::kOffK : L::kOffV;
             uint64_t* full = &bars[is_k ? kBarKFull : kBarVFull];
@@ -396,7 +373,32 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
             bool ok = true;
             for (;; ++it) {
                 Item I;
-                if (!take_item(it, false, I)) {
+                if (is_k) {
+                    // item scheduler: greedy dynamic assignment from the global counter,
+                    // published to the other roles through the ring
+                    const int slot = it % kItemRing;
+                    if (it >= kItemRing &&
+                        !mbar_wait(&bars[kBarItemFree + slot], ((it / kItemRing) - 1) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const int w = atomicAdd(args.item_counter, 1);
+                    if (w < n_items) {
+                        I = load_item(args, w);
+                    } else {
+                        I.q0 = I.q_end = I.k0 = I.h = 0;
+                        I.nk = 0;
+                        I.packed = false;
+                    }
+                    volatile int* e = items + slot * 8;
+                    e[0] = I.q0;
+                    e[1] = I.q_end;
+                    e[2] = I.k0;
+                    e[3] = I.nk;
+                    e[4] = I.h;
+                    e[5] = I.packed ? 1 : 0;
+                    mbar_arrive(&bars[kBarItemFull + slot]);
+                } else if (!take_item(it, false, I)) {
                     ok = false;
                     break;
                 }
@@ -443,85 +445,108 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
         __syncwarp();
     } else if (warp == C::kWarpMMA) {
         // ------------------------------------------------------------ MMA issuer
+        // Two cursors over the item stream: S runs G-1 tiles ahead of PV (PV_n
+        // is issued before S_n+G reuses buffer n % G). The S cursor takes items
+        // from the ring without releasing them; the PV cursor re-reads the same
+        // slot and releases it once the item's last PV is issued, so the slot
+        // stays valid in between.
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
-            // PV work lags S by G-1 tiles: pending[] holds (tile n, item, first/last)
-            int pend_n[G], pend_it[G], pend_fl[G];
-            int head = 0, count = 0;
-            auto issue_pv = [&](int n, int it, int fl) -> bool {
-                const int b = n % G, vs = n % S, ob = it % OB;
-                const bool first = fl & 1, last = fl & 2;
-                if (!mbar_wait(&bars[kBarPFull + b], (n / G) & 1, abort_flag)) return false;
-                if (!mbar_wait(&bars[kBarVFull + vs], (n / S) & 1, abort_flag)) return false;
-                if (first && it >= OB &&
-                    !mbar_wait(&bars[kBarOFree + ob], ((it / OB) - 1) & 1, abort_flag))
-                    return false;
-                tc_fence_after();
-                const uint32_t vb = sV + vs * kTileBytes;
-                const uint32_t pb = tmem + b * 128;
-#pragma unroll
-                for (int kk = 0; kk < kTile / 16; ++kk) {
-                    // keys 16kk..16kk+15: columns 32*(kk/2) + 8*(kk%2) of the P buffer
-                    const uint32_t a = pb + (kk >> 1) * 32 + (kk & 1) * 8;
-                    const uint64_t bd = desc_mnmajor_sw128(vb + kk * 2048, 16384);
-                    umma_bf16_ts(tmem + C::kTmemO + ob * D, a, bd, idesc_pv,
-                                 (first && kk == 0) ? 0u : 1u);
-                }
-                umma_commit(&bars[kBarVFree + vs]);
-                if (last) umma_commit(&bars[kBarOFull + b]);   // group b writes this item
+            constexpr uint32_t kStageDesc = kTileBytes >> 4;      // stage stride, descriptor units
+            const uint64_t dq0 = desc_kmajor_sw128(sQ);
+            const uint64_t dk0 = desc_kmajor_sw128(sK);
+            const uint64_t dv0 = desc_mnmajor_sw128(sV, 16384);
+            auto wait_item = [&](int k, Item& I) -> bool {
+                const int slot = k % kItemRing;
+                if (!mbar_wait(&bars[kBarItemFull + slot], (k / kItemRing) & 1, abort_flag)) return false;
+                I = read_item(items + slot * 8);
                 return true;
             };
             bool ok = true;
-            int n = 0, it = 0;
-            for (; ok; ++it) {
-                Item I;
-                if (!take_item(it, false, I)) {
-                    ok = false;
-                    break;
-                }
-                if (I.nk == 0) break;
-                const int qs = it % S;
-                if (!mbar_wait(&bars[kBarQFull + qs], (it / S) & 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                for (int j = 0; j < I.nk; ++j, ++n) {
-                    const int ks = n % S, b = n % G;
-                    // S buffer b last held P_n-G, read by PV_n-G, issued earlier by this thread
-                    if (!mbar_wait(&bars[kBarKFull + ks], (n / S) & 1, abort_flag)) {
+            // S cursor
+            int s_it = 0, s_j = 0, ns = 0;
+            Item si;
+            si.nk = -1;
+            bool s_live = wait_item(0, si) && si.nk > 0;
+            if (si.nk < 0) ok = false;                                        // aborted
+            // PV cursor
+            int p_it = 0, p_j = 0, np = 0;
+            Item pi = si;
+            while (ok && (s_live || np < ns)) {
+                if (s_live && ns - np < G) {
+                    // ---- S_ns = Q K^T into buffer ns % G
+                    const int qs = s_it % S, ks = ns % S, b = ns % G;
+                    if (s_j == 0 && !mbar_wait(&bars[kBarQFull + qs], (s_it / S) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    if (!mbar_wait(&bars[kBarKFull + ks], (ns / S) & 1, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t qb = sQ + qs * kTileBytes, kb_base = sK + ks * kTileBytes;
+                    const uint64_t dq = dq0 + static_cast<uint64_t>(qs * kStageDesc);
+                    const uint64_t dk = dk0 + static_cast<uint64_t>(ks * kStageDesc);
+                    const uint32_t dst = tmem + b * 128;
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                        umma_bf16_ss(tmem + b * 128, desc_kmajor_sw128(qb + off),
-                                     desc_kmajor_sw128(kb_base + off), idesc_qk, kk > 0 ? 1u : 0u);
+                        const uint64_t off = static_cast<uint64_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+                        umma_bf16_ss(dst, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
                     }
                     umma_commit(&bars[kBarSFull + b]);
                     umma_commit(&bars[kBarKFree + ks]);
-                    if (j == I.nk - 1) umma_commit(&bars[kBarQFree + qs]);
-                    const int slot = (head + count) % G;
-                    pend_n[slot] = n;
-                    pend_it[slot] = it;
-                    pend_fl[slot] = (j == 0 ? 1 : 0) | (j == I.nk - 1 ? 2 : 0);
-                    ++count;
-                    if (count == G) {
-                        ok = issue_pv(pend_n[head], pend_it[head], pend_fl[head]);
-                        head = (head + 1) % G;
-                        --count;
-                        if (!ok) break;
+                    ++ns;
+                    if (++s_j == si.nk) {
+                        umma_commit(&bars[kBarQFree + qs]);
+                        s_j = 0;
+                        ++s_it;
+                        si.nk = -1;
+                        s_live = wait_item(s_it, si) && si.nk > 0;
+                        if (si.nk < 0) {               // aborted while waiting for an item
+                            ok = false;
+                            break;
+                        }
+                    }
+                } else {
+                    // ---- PV_np: O += P V, A operand from TMEM
+                    const int b = np % G, vs = np % S, ob = p_it % OB;
+                    if (p_j == 0 && np > 0) {
+                        // the PV cursor enters item p_it: same ring slot the S cursor read
+                        pi = read_item(items + (p_it % kItemRing) * 8);
+                    }
+                    const bool first = p_j == 0, last = p_j == pi.nk - 1;
+                    if (!mbar_wait(&bars[kBarPFull + b], (np / G) & 1, abort_flag) ||
+                        !mbar_wait(&bars[kBarVFull + vs], (np / S) & 1, abort_flag) ||
+                        (first && p_it >= OB &&
+                         !mbar_wait(&bars[kBarOFree + ob], ((p_it / OB) - 1) & 1, abort_flag))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t dv = dv0 + static_cast<uint64_t>(vs * kStageDesc);
+                    const uint32_t pb = tmem + b * 128;
+                    const uint32_t dst = tmem + C::kTmemO + ob * D;
+#pragma unroll
+                    for (int kk = 0; kk < kTile / 16; ++kk) {
+                        // keys 16kk..16kk+15: columns 32*(kk/2) + 8*(kk%2) of the P buffer
+                        umma_bf16_ts(dst, pb + (kk >> 1) * 32 + (kk & 1) * 8,
+                                     dv + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv,
+                                     (first && kk == 0) ? 0u : 1u);
+                    }
+                    umma_commit(&bars[kBarVFree + vs]);
+                    ++np;
+                    if (last) {
+                        umma_commit(&bars[kBarOFull + b]);   // group b writes this item
+                        mbar_arrive(&bars[kBarItemFree + p_it % kItemRing]);
+                        p_j = 0;
+                        ++p_it;
+                    } else {
+                        ++p_j;
                     }
                 }
             }
-            while (ok && count > 0) {
-                ok = issue_pv(pend_n[head], pend_it[head], pend_fl[head]);
-                head = (head + 1) % G;
-                --count;
-            }
+            // (the end-of-stream slot is never reused, so it is not released)
             umma_commit(&bars[kBarDrain]);
             if (!mbar_wait(&bars[kBarDrain], 0, nullptr)) raise_error(kErrTimeout);
         }
