@@ -13,7 +13,7 @@
 // softmax: no running max, no rescale, no row sum, so O accumulates untouched
 // across key tiles and the per-element budget goes to the bias gathers and SiLU.
 //
-// Warp roles ((4G + 4) warps for G pointwise groups). Every role that blocks
+// Warp roles ((4G + 3) warps for G pointwise groups). Every role that blocks
 // on a barrier has a warp of its own: a lane suspended in a barrier wait holds
 // up the other lanes of its warp.
 //   warps 0..4G-1  pointwise stage in G groups of 4 warps. Counting the tiles a
@@ -23,20 +23,26 @@
 //              TMEM, MUFU and barrier latencies. Warp w owns TMEM lanes
 //              32*(w%4).. (one query row per thread) and all 128 columns. The
 //              group that handles an item's last tile also writes its output.
+//              Each group stages the bias data of its own tiles (below).
 //   warp 4G    item scheduler and TMA producer of Q tiles and the K ring
 //   warp 4G+1  TMA producer of the V ring
 //   warp 4G+2  MMA issuer (one thread) and TMEM owner
-//   warp 4G+3  bias staging: per key tile, key timestamps (int64 and low 32
-//              bits), their min/max and monotonicity, the window of the
-//              relative-position table, and the query rows' timestamps and
-//              sequence starts; one stage per S buffer. Software-pipelined: the
-//              global loads of the next tile are in flight while the current
-//              tile waits for its stage and is stored.
 // TMEM (512 columns): S buffers at 128g, then one or two O accumulators.
 // P_j overwrites the S_j buffer it came from, chunk by chunk: after a thread
 // has read S columns 32c..32c+31 of its row it writes their 32 bf16 results
 // into columns 32c..32c+15 (two per 32-bit column). The MMA issues PV_n and
 // only then S_n+G into the same buffer.
+//
+// Bias staging. Per key tile a group needs the tile's window of the
+// relative-position table and its key timestamps. The group's 128 threads
+// stage them into one of two stages of its own while the tile's S is still
+// being computed: right after finishing its previous tile, so the global loads
+// overlap the wait for S, and spread over 128 threads, so no single warp has
+// to keep up with every tile of the SM. Two stages per group suffice: a thread
+// refills a stage only after S of the group's previous tile was ready, which
+// the MMA issues only after every thread of the group finished the tile
+// before it (the stage's last reader). Per-row values (the row's timestamp,
+// its sequence start, the head's time-bias table) are loaded once per item.
 //
 // Masking: pair (i, j) is kept iff start(i) <= j <= i, with start(i) the first
 // token of row i's sequence (the unit's k0 for aligned units, a per-row value
@@ -48,10 +54,10 @@
 //   h = s/2 + pos/2 + time/2;  silu(x) = h + h*tanh(h)  (packed bf16x2, one
 //   MUFU op per two scores). The time bucket floor(log2(max(1, dt))) is the
 //   exponent field of dt converted exactly to double (no bit-find unit), and
-//   the bucket's bias comes from a 32-entry register table via a shuffle. When
-//   the key timestamps of a 32-key chunk are non-decreasing and every row of
-//   the warp sees one bucket at both ends of the chunk, the bucket is constant
-//   over the chunk and the per-score bucket work is skipped.
+//   the bucket's bias comes from a 32-entry register table via a shuffle. The
+//   bucket is monotone in dt, so when every row of a warp sees one bucket at
+//   the smallest and the largest key timestamp of a 32-key chunk, the bucket
+//   is constant over the chunk and the per-score bucket work is skipped.
 //
 // Every wait is bounded; a wait that runs out raises kErrTimeout, the other
 // roles notice through a shared abort flag, and the CTA drains its own copies
@@ -82,34 +88,36 @@ struct AttnArgs {
 
 constexpr int kAttnGroups = 3;          // pointwise groups (S buffers)
 constexpr int kItemRing = 8;            // work items published ahead of the pipeline
-constexpr int kMaxHeadsTable = 64;      // heads whose register time table is kept in SMEM
 constexpr uint32_t kTmemCols = 512;
 
 template <int D, int G>
 struct AttnCfg {
     static constexpr int kPointwiseWarps = 4 * G;
-    // One bias-staging warp: it must wait each stage's p_full phases in order
-    // (a second warp staging alternate tiles could wait a phase two steps ahead
-    // of the barrier, which the parity test cannot tell from the one before).
-    static constexpr int kMetaWarps = 1;
-    static constexpr int kWarpK = 4 * G, kWarpV = 4 * G + 1, kWarpMMA = 4 * G + 2,
-                         kWarpMeta = 4 * G + 3;
-    static constexpr int kThreads = (4 * G + 3 + kMetaWarps) * 32;
+    static constexpr int kWarpK = 4 * G, kWarpV = 4 * G + 1, kWarpMMA = 4 * G + 2;
+    static constexpr int kThreads = (4 * G + 3) * 32;
     static constexpr int kStages = D == 64 ? 3 : 2;                     // Q, K and V rings
     static constexpr int kOBufs = 128 * G + 2 * D <= static_cast<int>(kTmemCols) ? 2 : 1;
     static constexpr uint32_t kTmemO = 128 * G;
 };
 
-// One stage of staged bias data for one key tile.
-struct MetaStage {
-    float w[256];          // w[m] = pos[h][clamp(q0 - kt0 - 127 + m, 0, P-1)] / 2
+// Staged bias data of one key tile. The relative-position bias of the tile is
+// a 255-value window (pair (r, c) reads offset 127 + r - c). It is kept as
+// bf16 pos/2 in a sliding-window table: with R[k] = window offset 254 - k,
+// entry s of wb holds R[s..s+7], so row r reads the 32 values of columns
+// c0..c0+31 as entries k0, k0+8, k0+16, k0+24 (k0 = 127 - r + c0), four
+// 16-byte loads whose word p packs columns (c0+2p, c0+2p+1). Entry s lies in
+// 16-byte bank slot s mod 8, so the eight consecutive k0 of a quarter warp
+// never conflict.
+// Key timestamps are kept as their low 32 bits, which give exact differences
+// whenever every timestamp involved lies within 2^30 of `base` (the tile's
+// first key): ok[c] says so for the keys of chunk c, and cmin/cmax are the
+// chunk's smallest and largest key timestamp minus base.
+struct alignas(16) BiasStage {
+    uint4 wb[248];         // sliding-window table of bf16 pos/2
     int32_t kt32[128];     // low 32 bits of the key timestamps
-    int64_t kt64[128];     // key timestamps
-    int64_t rts[128];      // query-row timestamps
-    int32_t rstart[128];   // query-row sequence starts
-    int64_t tmin, tmax;    // over keys of the unit (< q_end)
-    int32_t mono;          // keys non-decreasing over the tile (keys < q_end)
-    int32_t pad[3];
+    int64_t base;          // timestamp of the tile's first key
+    int32_t cmin[4], cmax[4], ok[4];
+    int32_t pad[2];
 };
 
 template <int D, int G>
@@ -119,15 +127,15 @@ struct AttnSmem {
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + C::kStages * kTileBytes;
     static constexpr int kOffV = kOffK + C::kStages * kTileBytes;
-    static constexpr int kOffTB = kOffV + C::kStages * kTileBytes;      // float[kMaxHeadsTable][32]
-    static constexpr int kOffMeta = kOffTB + kMaxHeadsTable * 32 * 4;   // MetaStage[G]
-    static constexpr int kOffItems = kOffMeta + G * static_cast<int>(sizeof(MetaStage));
+    static constexpr int kOffStage = kOffV + C::kStages * kTileBytes;   // BiasStage[2G]
+    static constexpr int kOffItems = kOffStage + 2 * G * static_cast<int>(sizeof(BiasStage));
     static constexpr int kOffBar = kOffItems + kItemRing * 32;                // int[8] per slot
-    static constexpr int kNumBars = 48;
+    static constexpr int kNumBars = 56;
     static constexpr int kOffTmem = kOffBar + kNumBars * 8;
     static constexpr int kOffAbort = kOffTmem + 8;
     static constexpr int kBytes = kOffAbort + 8;
     static constexpr int kAlloc = kBytes + 1024;                        // 1 KB alignment slack
+    static_assert(kAlloc <= 227 * 1024, "shared memory per block");
 };
 
 // barrier slots (rings of up to 3 stages, up to 3 S buffers, up to 2 O buffers)
@@ -138,7 +146,7 @@ enum {
     kBarKFree = 9,      // +stage
     kBarVFull = 12,     // +stage
     kBarVFree = 15,     // +stage
-    kBarSFull = 18,     // +buffer: MMA commit + 32 bias-staging lanes
+    kBarSFull = 18,     // +buffer: MMA commit
     kBarPFull = 21,     // +buffer: the 128 threads of the buffer's group
     kBarOFull = 24,     // +group: MMA commit after the last PV of an item whose output
                         // that group writes (one barrier per group, so every barrier
@@ -148,6 +156,7 @@ enum {
     kBarDrain = 29,
     kBarItemFull = 30,  // +slot (8): scheduler published an item
     kBarItemFree = 38,  // +slot (8): every consumer has read it
+    kBarStage = 46,     // +2g+s (up to 6): the 128 threads of group g staged stage s
 };
 
 // A work item as the scheduler publishes it; nk == 0 ends the stream.
@@ -185,86 +194,112 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
     return __all_sync(0xffffffffu, ok);
 }
 
-// silu of a packed pair of half-scores: h + h * tanh(h), bf16x2.
-__device__ __forceinline__ uint32_t silu_half_bf16x2(float h0, float h1) {
-    const uint32_t hp = pack_bf16x2(h0, h1);
+// Per-chunk pointwise paths. sv: 32 fp32 scores of columns c0..c0+31 of this
+// thread's row; wbk: this row's entry k0 of the pos/2 window table (entries
+// wbk[0], wbk[8], wbk[16], wbk[24] cover the chunk); pk: 16 packed bf16x2
+// outputs, word p = columns (c0+2p, c0+2p+1).
+//
+// Every path computes a pair the same way, in packed bf16x2:
+//   h = bf16(s) * 0.5 + pos/2  (one rounding),  h = h + bf16(time/2),
+//   p = h + h * tanh(h)        (one MUFU op per pair)
+// and differs only in how it finds time/2, so which path a warp takes (a
+// choice made over all of its 32 rows) never changes a row's bits.
+
+// The half-score pair plus its bias pair.
+__device__ __forceinline__ uint32_t half_arg_bf16x2(uint32_t s0, uint32_t s1, uint32_t w2,
+                                                    uint32_t t2) {
+    const uint32_t s2 = pack_bf16x2(__uint_as_float(s0), __uint_as_float(s1));
+    uint32_t h, hb;
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(h) : "r"(s2), "r"(0x3f003f00u), "r"(w2));
+    asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(hb) : "r"(h), "r"(t2));
+    return hb;
+}
+
+// silu(2h) = h + h * tanh(h) on a packed pair.
+__device__ __forceinline__ uint32_t silu_of_half_bf16x2(uint32_t hb) {
     uint32_t t, y;
-    asm("tanh.approx.bf16x2 %0, %1;" : "=r"(t) : "r"(hp));
-    asm("fma.rn.bf16x2 %0, %1, %2, %1;" : "=r"(y) : "r"(hp), "r"(t));
+    asm("tanh.approx.bf16x2 %0, %1;" : "=r"(t) : "r"(hb));
+    asm("fma.rn.bf16x2 %0, %1, %2, %1;" : "=r"(y) : "r"(hb), "r"(t));
     return y;
 }
 
-// Per-chunk pointwise paths. sv: 32 fp32 scores of columns c0..c0+31 of this
-// thread's row; wrow[-c] = pos/2 of column c; pk: 16 packed bf16x2 outputs.
+// Keep-mask of the pair (c, c+1): pair (i, j) is kept iff lo <= j <= hi.
+__device__ __forceinline__ uint32_t pair_mask(int c, int lo, int hi) {
+    return ((c >= lo && c <= hi) ? 0x0000ffffu : 0u) | ((c + 1 >= lo && c + 1 <= hi) ? 0xffff0000u : 0u);
+}
 
-// Constant time bucket over the chunk: tconst = time/2 for every column.
-template <bool kMask>
-__device__ __forceinline__ void pw_const(const uint32_t* sv, int c0,
-                                         const float* __restrict__ wrow, float tconst, int lo,
-                                         int hi, uint32_t* pk) {
+// Constant time bucket over an unmasked chunk (t2 = time/2 in both halves).
+__device__ __forceinline__ void pw_const(const uint32_t* sv, const uint4* wbk, uint32_t t2,
+                                         uint32_t* pk) {
 #pragma unroll
-    for (int e = 0; e < 32; e += 2) {
-        float h[2];
+    for (int q = 0; q < 4; ++q) {
+        const uint4 W = wbk[8 * q];
+        const uint32_t wv[4] = {W.x, W.y, W.z, W.w};
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int c = c0 + e + u;
-            float v = fmaf(__uint_as_float(sv[e + u]), 0.5f, wrow[-c]) + tconst;
-            if (kMask) v = (c >= lo && c <= hi) ? v : 0.0f;
-            h[u] = v;
+        for (int u = 0; u < 4; ++u) {
+            const int p = 4 * q + u;
+            pk[p] = silu_of_half_bf16x2(half_arg_bf16x2(sv[2 * p], sv[2 * p + 1], wv[u], t2));
         }
-        pk[e >> 1] = silu_half_bf16x2(h[0], h[1]);
     }
 }
 
 // Bucket per score, differences exact in 32 bits. tbr: this lane's entry of
 // the register table (lane L holds time/2 of bucket min((L+1) mod 32, NB-1)).
 template <bool kMask>
-__device__ __forceinline__ void pw_fast(const uint32_t* sv, int c0,
-                                        const float* __restrict__ wrow,
+__device__ __forceinline__ void pw_fast(const uint32_t* sv, int c0, const uint4* wbk,
                                         const int32_t* __restrict__ kt32, int32_t ti32, float tbr,
                                         int lo, int hi, uint32_t* pk) {
     const int4* k4 = reinterpret_cast<const int4*>(kt32 + c0);
 #pragma unroll
-    for (int e = 0; e < 32; e += 4) {
-        const int4 kk = k4[e >> 2];
-        const int32_t kv[4] = {kk.x, kk.y, kk.z, kk.w};
-        float h[4];
+    for (int q = 0; q < 4; ++q) {
+        const uint4 W = wbk[8 * q];
+        const uint32_t wv[4] = {W.x, W.y, W.z, W.w};
+        const int4 ka = k4[2 * q], kb = k4[2 * q + 1];
+        const int32_t kv[8] = {ka.x, ka.y, ka.z, ka.w, kb.x, kb.y, kb.z, kb.w};
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-            const int c = c0 + e + u;
-            const int32_t dt = static_cast<int32_t>(static_cast<uint32_t>(ti32) -
-                                                    static_cast<uint32_t>(kv[u]));
-            const uint32_t ef = log2_exponent_field(static_cast<uint32_t>(max(dt, 1)));
-            const float tv = __shfl_sync(0xffffffffu, tbr, static_cast<int>(ef));
-            float v = fmaf(__uint_as_float(sv[e + u]), 0.5f, wrow[-c]) + tv;
-            if (kMask) v = (c >= lo && c <= hi) ? v : 0.0f;
-            h[u] = v;
+            float tv[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int32_t dt = static_cast<int32_t>(static_cast<uint32_t>(ti32) -
+                                                        static_cast<uint32_t>(kv[2 * u + e]));
+                const uint32_t ef = log2_exponent_field(static_cast<uint32_t>(max(dt, 1)));
+                tv[e] = __shfl_sync(0xffffffffu, tbr, static_cast<int>(ef));
+            }
+            const int p = 4 * q + u;
+            uint32_t hb = half_arg_bf16x2(sv[2 * p], sv[2 * p + 1], wv[u], pack_bf16x2(tv[0], tv[1]));
+            if (kMask) hb &= pair_mask(c0 + 2 * p, lo, hi);
+            pk[p] = silu_of_half_bf16x2(hb);
         }
-        pk[e >> 1] = silu_half_bf16x2(h[0], h[1]);
-        pk[(e >> 1) + 1] = silu_half_bf16x2(h[2], h[3]);
     }
 }
 
-// Any int64 timestamps: 64-bit bucket, table row of this head read through
-// the read-only cache (tbh = time_bias + h * NB, or null).
+// Any int64 timestamps: 64-bit bucket from the key timestamps in global
+// memory (kts = timestamps of the tile's keys, column c read at min(c, lastc)
+// so a tile past the end of the batch stays in bounds), table row of this
+// head read through the read-only cache (tbh = time_bias + h * NB, or null).
 template <bool kMask>
-__device__ __forceinline__ void pw_slow(const uint32_t* sv, int c0,
-                                        const float* __restrict__ wrow,
-                                        const int64_t* __restrict__ kt64, int64_t ti,
+__device__ __forceinline__ void pw_slow(const uint32_t* sv, int c0, const uint4* wbk,
+                                        const int64_t* __restrict__ kts, int lastc, int64_t ti,
                                         const float* __restrict__ tbh, int nbm1, int lo, int hi,
                                         uint32_t* pk) {
 #pragma unroll
-    for (int e = 0; e < 32; e += 2) {
-        float h[2];
+    for (int q = 0; q < 4; ++q) {
+        const uint4 W = wbk[8 * q];
+        const uint32_t wv[4] = {W.x, W.y, W.z, W.w};
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int c = c0 + e + u;
-            const float tv = tbh ? 0.5f * __ldg(tbh + time_bucket64(ti - kt64[c], nbm1)) : 0.f;
-            float v = fmaf(__uint_as_float(sv[e + u]), 0.5f, wrow[-c]) + tv;
-            if (kMask) v = (c >= lo && c <= hi) ? v : 0.0f;
-            h[u] = v;
+        for (int u = 0; u < 4; ++u) {
+            const int p = 4 * q + u;
+            const int c = c0 + 2 * p;
+            float tv[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+                tv[e] = tbh ? 0.5f * __ldg(tbh + time_bucket64(ti - __ldg(kts + min(c + e, lastc)), nbm1))
+                            : 0.f;
+            uint32_t hb = half_arg_bf16x2(sv[2 * p], sv[2 * p + 1], wv[u], pack_bf16x2(tv[0], tv[1]));
+            if (kMask) hb &= pair_mask(c, lo, hi);
+            pk[p] = silu_of_half_bf16x2(hb);
         }
-        pk[e >> 1] = silu_half_bf16x2(h[0], h[1]);
     }
 }
 
@@ -295,10 +330,9 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffTmem);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffAbort);
-    float* tbh_s = reinterpret_cast<float*>(smem + L::kOffTB);
-    MetaStage* meta = reinterpret_cast<MetaStage*>(smem + L::kOffMeta);
+    BiasStage* stages = reinterpret_cast<BiasStage*>(smem + L::kOffStage);
     volatile int* items = reinterpret_cast<volatile int*>(smem + L::kOffItems);
-    constexpr int kConsumers = 2 + C::kMetaWarps + C::kPointwiseWarps;   // V, MMA, bias, pointwise
+    constexpr int kConsumers = 2 + C::kPointwiseWarps;   // V, MMA, pointwise
     const bool use_time = args.ts != nullptr && args.tb != nullptr && args.NB > 0;
     const int nbm1 = use_time ? args.NB - 1 : 0;
 
@@ -313,8 +347,10 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
             mbar_init(&bars[kBarVFree + s], 1);
         }
         for (int b = 0; b < G; ++b) {
-            mbar_init(&bars[kBarSFull + b], 1 + 32);
+            mbar_init(&bars[kBarSFull + b], 1);
             mbar_init(&bars[kBarPFull + b], 128);
+            mbar_init(&bars[kBarStage + 2 * b], 128);
+            mbar_init(&bars[kBarStage + 2 * b + 1], 128);
         }
         for (int b = 0; b < G; ++b) mbar_init(&bars[kBarOFull + b], 1);
         for (int o = 0; o < OB; ++o) mbar_init(&bars[kBarOFree + o], 128);
@@ -328,15 +364,6 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
     if (warp == C::kWarpMMA) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
-    }
-    if (warp < C::kPointwiseWarps) {
-        // register-table source: [h][L] = time/2 of bucket min((L + 1) mod 32, NB - 1)
-        for (int idx = tid; idx < args.H * 32; idx += 32 * C::kPointwiseWarps) {
-            const int hh = idx >> 5, ll = idx & 31;
-            tbh_s[idx] = use_time ? 0.5f * args.tb[static_cast<int64_t>(hh) * args.NB +
-                                                   min((ll + 1) & 31, nbm1)]
-                                  : 0.f;
-        }
     }
     tc_fence_before();
     __syncthreads();
@@ -551,112 +578,61 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
             if (!mbar_wait(&bars[kBarDrain], 0, nullptr)) raise_error(kErrTimeout);
         }
         __syncwarp();
-    } else if (warp == C::kWarpMeta) {
-        // ------------------------------------------------------------ bias staging
-        // Per-tile values this lane stages: pos window (8), key timestamps (4),
-        // query-row timestamps (4) and sequence starts (4).
-        struct Staged {
-            float w[8];
-            int64_t kt[4], rt[4];
-            int32_t rs[4];
-        };
-        auto load_tile = [&](const Item& I, int j, Staged& d) {
-            const int kt0 = I.k0 + j * kTile;
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int mm = lane + 32 * u;
-                d.w[u] = 0.f;
-                if (args.pos && mm < 255) {
-                    int64_t dd = static_cast<int64_t>(I.q0) - kt0 - 127 + mm;
-                    dd = dd < 0 ? 0 : (dd > args.P - 1 ? args.P - 1 : dd);
-                    d.w[u] = args.pos[static_cast<int64_t>(I.h) * args.P + dd];
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int64_t key = static_cast<int64_t>(kt0) + lane + 32 * u;
-                d.kt[u] = use_time ? args.ts[key < args.T ? key : args.T - 1] : 0;
-                const int64_t i = static_cast<int64_t>(I.q0) + lane + 32 * u;
-                const bool v = i < I.q_end;
-                d.rt[u] = (use_time && v) ? args.ts[i < args.T ? i : args.T - 1] : 0;
-                d.rs[u] = (I.packed && v) ? args.row_start[i] : I.k0;
-            }
-        };
-        Item cur;
-        int it = 0, j = 0, n = 0;
-        bool have = take_item(it++, true, cur) && cur.nk > 0;
-        Staged st;
-        if (have) load_tile(cur, 0, st);
-        while (have) {
-            // the following tile: its loads fly while this tile is stored
-            Item nxt = cur;
-            int nj = j + 1;
-            bool nhave = true;
-            if (nj >= cur.nk) {
-                nj = 0;
-                nhave = take_item(it++, true, nxt) && nxt.nk > 0;
-            }
-            Staged sn;
-            if (nhave) load_tile(nxt, nj, sn);
-            const int b = n % G;
-            // stage b last served tile n-G; P_n-G written means it has been read
-            if (n >= G && !warp_wait(&bars[kBarPFull + b], ((n / G) - 1) & 1, abort_flag)) break;
-            MetaStage& ms = meta[b];
-            const int kt0 = cur.k0 + j * kTile;
-#pragma unroll
-            for (int u = 0; u < 8; ++u) ms.w[lane + 32 * u] = 0.5f * st.w[u];
-            int64_t tmin = INT64_MAX, tmax = INT64_MIN;
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int mm = lane + 32 * u;
-                ms.kt64[mm] = st.kt[u];
-                ms.kt32[mm] = static_cast<int32_t>(static_cast<uint64_t>(st.kt[u]));
-                ms.rts[mm] = st.rt[u];
-                ms.rstart[mm] = st.rs[u];
-                if (kt0 + mm < cur.q_end) {
-                    tmin = st.kt[u] < tmin ? st.kt[u] : tmin;
-                    tmax = st.kt[u] > tmax ? st.kt[u] : tmax;
-                }
-            }
-            __syncwarp();
-            bool mono = true;
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int mm = lane + 32 * u;
-                if (mm < 127 && kt0 + mm + 1 < cur.q_end)
-                    mono = mono && (ms.kt64[mm] <= ms.kt64[mm + 1]);
-            }
-            mono = __all_sync(0xffffffffu, mono);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const int64_t a = __shfl_xor_sync(0xffffffffu, tmin, o);
-                const int64_t c = __shfl_xor_sync(0xffffffffu, tmax, o);
-                tmin = a < tmin ? a : tmin;
-                tmax = c > tmax ? c : tmax;
-            }
-            if (lane == 0) {
-                ms.tmin = tmin;
-                ms.tmax = tmax;
-                ms.mono = mono ? 1 : 0;
-            }
-            __syncwarp();
-            mbar_arrive(&bars[kBarSFull + b]);
-            cur = nxt;
-            j = nj;
-            have = nhave;
-            st = sn;
-            ++n;
-        }
     } else {
         // ------------------------------------------------------------ pointwise stage
         const int g = warp >> 2;                            // group: tiles n = g (mod G)
         const int qd = warp & 3;                            // TMEM lane quarter
         const int r = qd * 32 + lane;                       // query row = TMEM lane
         const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
-        const MetaStage& ms = meta[g];
         const uint32_t s_col = tmem + lane_base + static_cast<uint32_t>(g * 128);
+
+        // Stage the bias data of key tile kt0 of item I (every thread of the
+        // group takes part: table entries r and r + 128, key r, and the
+        // timestamp summary of chunk qd, whose keys are this warp's lanes).
+        auto stage_tile = [&](const Item& I, int kt0, BiasStage& st, uint64_t* full) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int se = r + 128 * e;
+                if (se < 248) {
+                    uint32_t wd[4] = {0u, 0u, 0u, 0u};
+                    if (args.pos) {
+                        // R[k] = pos[h][clamp(i - j)] with i - j = q0 - kt0 + 127 - k
+                        const float* prow = args.pos + static_cast<int64_t>(I.h) * args.P;
+                        const int rel0 = I.q0 - kt0 + 127 - se;
+                        float v[8];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) v[u] = __ldg(prow + min(max(rel0 - u, 0), args.P - 1));
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) wd[u] = pack_bf16x2(0.5f * v[2 * u], 0.5f * v[2 * u + 1]);
+                    }
+                    st.wb[se] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+                }
+            }
+            const int64_t key = static_cast<int64_t>(kt0) + r;
+            const bool kvalid = key < I.q_end;
+            int64_t kv = 0, base = 0;
+            if (use_time) {
+                kv = __ldg(args.ts + (key < args.T ? key : args.T - 1));
+                base = __ldg(args.ts + kt0);
+            }
+            st.kt32[r] = static_cast<int32_t>(static_cast<uint64_t>(kv));
+            const int64_t dk = kv - base;
+            const bool near = dk > -(1ll << 30) && dk < (1ll << 30);
+            const int dmin = __reduce_min_sync(0xffffffffu, (kvalid && near) ? static_cast<int>(dk) : INT_MAX);
+            const int dmax = __reduce_max_sync(0xffffffffu, (kvalid && near) ? static_cast<int>(dk) : INT_MIN);
+            const bool all_near = __all_sync(0xffffffffu, !kvalid || near);
+            if (lane == 0) {
+                st.cmin[qd] = dmin;
+                st.cmax[qd] = dmax;
+                st.ok[qd] = all_near ? 1 : 0;
+            }
+            if (r == 0) st.base = base;
+            mbar_arrive(full);
+        };
+
         bool ok = true;
         int n = 0, it = 0, ep = 0;   // ep: outputs this group has written
+        int nt = 0;                  // tiles this group has processed (stage nt % 2)
         for (; ok; ++it) {
             Item I;
             if (!take_item(it, true, I)) {
@@ -667,30 +643,42 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
             const int64_t i = static_cast<int64_t>(I.q0) + r;
             const bool row_valid = i < I.q_end;
             const bool warp_live = __any_sync(0xffffffffu, row_valid);
-            const float tbr = tbh_s[I.h * 32 + lane];
+            // per-row values of the item: timestamp, first token of the row's
+            // sequence, and this lane's entry of the head's register time table
+            // (lane L holds time/2 of bucket min((L + 1) mod 32, NB - 1))
+            const int64_t ti = (use_time && row_valid) ? __ldg(args.ts + i) : 0;
+            const int rs = (I.packed && row_valid) ? __ldg(args.row_start + i) : I.k0;
+            const float tbr = use_time ? 0.5f * __ldg(args.tb + static_cast<int64_t>(I.h) * args.NB +
+                                                      min((lane + 1) & 31, nbm1))
+                                       : 0.f;
             const float* tbh = use_time ? args.tb + static_cast<int64_t>(I.h) * args.NB : nullptr;
+            const int32_t ti32 = static_cast<int32_t>(static_cast<uint64_t>(ti));
             for (int j = 0; j < I.nk; ++j, ++n) {
                 if (n % G != g) continue;
-                if (!warp_wait(&bars[kBarSFull + g], (n / G) & 1, abort_flag)) {
+                const int kt0 = I.k0 + j * kTile;
+                const int sb = nt & 1;
+                BiasStage& st = stages[2 * g + sb];
+                stage_tile(I, kt0, st, &bars[kBarStage + 2 * g + sb]);
+                if (!warp_wait(&bars[kBarStage + 2 * g + sb], (nt >> 1) & 1, abort_flag) ||
+                    !warp_wait(&bars[kBarSFull + g], (n / G) & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
+                ++nt;
                 tc_fence_after();
                 if (warp_live) {
-                    const int kt0 = I.k0 + j * kTile;
-                    const int lo = ms.rstart[r] - kt0;      // first key of row i's sequence
+                    const int lo = rs - kt0;                // first key of row i's sequence
                     const int hi = row_valid ? static_cast<int>(i - kt0) : -1;
-                    const int64_t ti = ms.rts[r];
-                    const int32_t ti32 = static_cast<int32_t>(static_cast<uint64_t>(ti));
                     bool fast = true;
-                    if (row_valid && use_time) {
-                        const int64_t lo_t = ti < ms.tmin ? ti : ms.tmin;
-                        const int64_t hi_t = ti > ms.tmax ? ti : ms.tmax;
-                        fast = static_cast<uint64_t>(hi_t) - static_cast<uint64_t>(lo_t) < (1ull << 31);
+                    int32_t tib = 0;                        // ti - base, when fast
+                    if (use_time) {
+                        const int64_t db = ti - st.base;
+                        fast = st.ok[0] && st.ok[1] && st.ok[2] && st.ok[3] &&
+                               (!row_valid || (db > -(1ll << 30) && db < (1ll << 30)));
+                        tib = static_cast<int32_t>(db);
                     }
                     const bool fast_w = __all_sync(0xffffffffu, fast);
-                    const bool mono = ms.mono != 0;
-                    const float* wrow = ms.w + 127 + r;
+                    const uint4* wbr = st.wb + (127 - r);        // entry k0 of chunk 0
 #pragma unroll 1
                     for (int q = 0; q < 4; ++q) {
                         const int c0 = 32 * q;
@@ -707,25 +695,24 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                         __syncwarp();
                         tmem_ld32(s_col + c0, sv);
                         const bool full = __all_sync(0xffffffffu, lo <= c0 && hi >= c0 + 31);
-                        bool done = false;
                         if (!fast_w) {
-                            if (full) pw_slow<false>(sv, c0, wrow, ms.kt64, ti, tbh, nbm1, lo, hi, pk);
-                            else pw_slow<true>(sv, c0, wrow, ms.kt64, ti, tbh, nbm1, lo, hi, pk);
-                            done = true;
-                        } else if (full && mono) {
-                            const uint32_t ef0 = log2_exponent_field(static_cast<uint32_t>(max(
-                                static_cast<int32_t>(static_cast<uint32_t>(ti32) - static_cast<uint32_t>(ms.kt32[c0])), 1)));
-                            const uint32_t ef1 = log2_exponent_field(static_cast<uint32_t>(max(
-                                static_cast<int32_t>(static_cast<uint32_t>(ti32) - static_cast<uint32_t>(ms.kt32[c0 + 31])), 1)));
-                            const float tconst = __shfl_sync(0xffffffffu, tbr, static_cast<int>(ef0));
-                            if (__all_sync(0xffffffffu, ef0 == ef1)) {
-                                pw_const<false>(sv, c0, wrow, tconst, lo, hi, pk);
-                                done = true;
+                            const int lastc = static_cast<int>(args.T - 1 - kt0);
+                            if (full) pw_slow<false>(sv, c0, wbr + c0, args.ts + kt0, lastc, ti, tbh, nbm1, lo, hi, pk);
+                            else pw_slow<true>(sv, c0, wbr + c0, args.ts + kt0, lastc, ti, tbh, nbm1, lo, hi, pk);
+                        } else if (full) {
+                            // the bucket at the chunk's largest and smallest dt
+                            float tconst = 0.f;
+                            bool cst = true;
+                            if (use_time) {
+                                const uint32_t ef_hi = log2_exponent_field(static_cast<uint32_t>(max(tib - st.cmin[q], 1)));
+                                const uint32_t ef_lo = log2_exponent_field(static_cast<uint32_t>(max(tib - st.cmax[q], 1)));
+                                tconst = __shfl_sync(0xffffffffu, tbr, static_cast<int>(ef_lo));
+                                cst = __all_sync(0xffffffffu, ef_hi == ef_lo);
                             }
-                        }
-                        if (!done) {
-                            if (full) pw_fast<false>(sv, c0, wrow, ms.kt32, ti32, tbr, lo, hi, pk);
-                            else pw_fast<true>(sv, c0, wrow, ms.kt32, ti32, tbr, lo, hi, pk);
+                            if (cst) pw_const(sv, wbr + c0, pack_bf16x2(tconst, tconst), pk);
+                            else pw_fast<false>(sv, c0, wbr + c0, st.kt32, ti32, tbr, lo, hi, pk);
+                        } else {
+                            pw_fast<true>(sv, c0, wbr + c0, st.kt32, ti32, tbr, lo, hi, pk);
                         }
                         // 32 bf16 results -> columns 32q..32q+15 of the S buffer just read
                         tmem_st16(s_col + c0, pk);

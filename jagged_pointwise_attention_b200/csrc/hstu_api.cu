@@ -151,7 +151,6 @@ hstu_status_t validate_attn(const AttnCall& c) {
     if (c.tb && (c.NB < 1 || c.NB > kMaxTimeBuckets)) return HSTU_ERR_INVALID_ARG;
     if (c.dtype == HSTU_DTYPE_BF16) {
         if (c.dqk != c.dv || (c.dqk != 64 && c.dqk != 128)) return HSTU_ERR_UNSUPPORTED;
-        if (c.H > kMaxHeadsTable) return HSTU_ERR_UNSUPPORTED;
         if (!aligned16(c.q) || !aligned16(c.k) || !aligned16(c.v) || !aligned16(c.out))
             return HSTU_ERR_INVALID_ARG;
         if (c.qs % 8 || c.ks % 8 || c.vs % 8 || c.os % 8) return HSTU_ERR_INVALID_ARG;
