@@ -93,8 +93,9 @@ constexpr uint32_t kTmemCols = 512;
 template <int D, int G>
 struct AttnCfg {
     static constexpr int kPointwiseWarps = 4 * G;
-    static constexpr int kWarpK = 4 * G, kWarpV = 4 * G + 1, kWarpMMA = 4 * G + 2;
-    static constexpr int kThreads = (4 * G + 3) * 32;
+    static constexpr int kWarpK = 4 * G, kWarpV = 4 * G + 1, kWarpMMA = 4 * G + 2,
+                         kWarpPV = 4 * G + 3;
+    static constexpr int kThreads = (4 * G + 4) * 32;
     static constexpr int kStages = D == 64 ? 3 : 2;                     // Q, K and V rings
     static constexpr int kOBufs = 128 * G + 2 * D <= static_cast<int>(kTmemCols) ? 2 : 1;
     static constexpr uint32_t kTmemO = 128 * G;
@@ -153,11 +154,15 @@ enum {
                         // is waited by one group in its own order and a waiter can
                         // never be two phases ahead of it)
     kBarOFree = 27,     // +O buffer: the 128 threads that stored the item's output
-    kBarDrain = 29,
+    kBarDrain = 29,     // the S issuer's last commit
     kBarItemFull = 30,  // +slot (8): scheduler published an item
     kBarItemFree = 38,  // +slot (8): every consumer has read it
     kBarStage = 46,     // +2g+s (up to 6): the 128 threads of group g staged stage s
+    kBarPVDone = 52,    // +buffer (up to 3): PV of the buffer's tile has completed
+    kBarDrainPV = 55,   // the PV issuer's last commit
+    kBarCount = 56,
 };
+static_assert(kBarCount == AttnSmem<64, kAttnGroups>::kNumBars, "barrier slots");
 
 // A work item as the scheduler publishes it; nk == 0 ends the stream.
 struct Item {
@@ -332,7 +337,7 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffAbort);
     BiasStage* stages = reinterpret_cast<BiasStage*>(smem + L::kOffStage);
     volatile int* items = reinterpret_cast<volatile int*>(smem + L::kOffItems);
-    constexpr int kConsumers = 2 + C::kPointwiseWarps;   // V, MMA, pointwise
+    constexpr int kConsumers = 3 + C::kPointwiseWarps;   // V, both MMA issuers, pointwise
     const bool use_time = args.ts != nullptr && args.tb != nullptr && args.NB > 0;
     const int nbm1 = use_time ? args.NB - 1 : 0;
 
@@ -359,6 +364,8 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
             mbar_init(&bars[kBarItemFree + q], kConsumers);
         }
         mbar_init(&bars[kBarDrain], 1);
+        mbar_init(&bars[kBarDrainPV], 1);
+        for (int b = 0; b < G; ++b) mbar_init(&bars[kBarPVDone + b], 1);
         mbar_fence_init();
     }
     if (warp == C::kWarpMMA) {
@@ -470,112 +477,100 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
             }
         }
         __syncwarp();
-    } else if (warp == C::kWarpMMA) {
-        // ------------------------------------------------------------ MMA issuer
-        // Two cursors over the item stream: S runs G-1 tiles ahead of PV (PV_n
-        // is issued before S_n+G reuses buffer n % G). The S cursor takes items
-        // from the ring without releasing them; the PV cursor re-reads the same
-        // slot and releases it once the item's last PV is issued, so the slot
-        // stays valid in between.
+    } else if (warp == C::kWarpMMA || warp == C::kWarpPV) {
+        // ------------------------------------------------------------ MMA issuers
+        // The MMA unit queues hardly more than one instruction, so while the
+        // issuing thread tests a barrier (a few hundred cycles for any shared
+        // memory access after an MMA) the tensor pipe runs dry. S and PV are
+        // therefore issued by two warps: while one waits, the other issues.
+        // S_n+G overwrites the buffer PV_n reads, so the S issuer waits for
+        // PV_n to complete (pv_done of the buffer) before issuing S_n+G.
         if (lane == 0) {
-            constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
-            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
             constexpr uint32_t kStageDesc = kTileBytes >> 4;      // stage stride, descriptor units
-            const uint64_t dq0 = desc_kmajor_sw128(sQ);
-            const uint64_t dk0 = desc_kmajor_sw128(sK);
-            const uint64_t dv0 = desc_mnmajor_sw128(sV, 16384);
-            auto wait_item = [&](int k, Item& I) -> bool {
-                const int slot = k % kItemRing;
-                if (!mbar_wait(&bars[kBarItemFull + slot], (k / kItemRing) & 1, abort_flag)) return false;
-                I = read_item(items + slot * 8);
-                return true;
-            };
             bool ok = true;
-            // S cursor
-            int s_it = 0, s_j = 0, ns = 0;
-            Item si;
-            si.nk = -1;
-            bool s_live = wait_item(0, si) && si.nk > 0;
-            if (si.nk < 0) ok = false;                                        // aborted
-            // PV cursor
-            int p_it = 0, p_j = 0, np = 0;
-            Item pi = si;
-            while (ok && (s_live || np < ns)) {
-                if (s_live && ns - np < G) {
-                    // ---- S_ns = Q K^T into buffer ns % G
-                    const int qs = s_it % S, ks = ns % S, b = ns % G;
-                    if (s_j == 0 && !mbar_wait(&bars[kBarQFull + qs], (s_it / S) & 1, abort_flag)) {
+            int n = 0;
+            if (warp == C::kWarpMMA) {
+                // ---- S_n = Q K_n^T into buffer n % G
+                constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
+                const uint64_t dq0 = desc_kmajor_sw128(sQ);
+                const uint64_t dk0 = desc_kmajor_sw128(sK);
+                for (int it = 0; ok; ++it) {
+                    Item I;
+                    if (!take_item(it, false, I)) {
                         ok = false;
                         break;
                     }
-                    if (!mbar_wait(&bars[kBarKFull + ks], (ns / S) & 1, abort_flag)) {
+                    if (I.nk == 0) break;
+                    const int qs = it % S;
+                    if (!mbar_wait(&bars[kBarQFull + qs], (it / S) & 1, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    tc_fence_after();
                     const uint64_t dq = dq0 + static_cast<uint64_t>(qs * kStageDesc);
-                    const uint64_t dk = dk0 + static_cast<uint64_t>(ks * kStageDesc);
-                    const uint32_t dst = tmem + b * 128;
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint64_t off = static_cast<uint64_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
-                        umma_bf16_ss(dst, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
-                    }
-                    umma_commit(&bars[kBarSFull + b]);
-                    umma_commit(&bars[kBarKFree + ks]);
-                    ++ns;
-                    if (++s_j == si.nk) {
-                        umma_commit(&bars[kBarQFree + qs]);
-                        s_j = 0;
-                        ++s_it;
-                        si.nk = -1;
-                        s_live = wait_item(s_it, si) && si.nk > 0;
-                        if (si.nk < 0) {               // aborted while waiting for an item
+                    for (int j = 0; j < I.nk; ++j, ++n) {
+                        const int ks = n % S, b = n % G;
+                        if (!mbar_wait(&bars[kBarKFull + ks], (n / S) & 1, abort_flag) ||
+                            (n >= G && !mbar_wait(&bars[kBarPVDone + b], ((n / G) - 1) & 1, abort_flag))) {
                             ok = false;
                             break;
                         }
+                        tc_fence_after();
+                        const uint64_t dk = dk0 + static_cast<uint64_t>(ks * kStageDesc);
+                        const uint32_t dst = tmem + b * 128;
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint64_t off = static_cast<uint64_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+                            umma_bf16_ss(dst, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
+                        }
+                        umma_commit(&bars[kBarSFull + b]);
+                        umma_commit(&bars[kBarKFree + ks]);
                     }
-                } else {
-                    // ---- PV_np: O += P V, A operand from TMEM
-                    const int b = np % G, vs = np % S, ob = p_it % OB;
-                    if (p_j == 0 && np > 0) {
-                        // the PV cursor enters item p_it: same ring slot the S cursor read
-                        pi = read_item(items + (p_it % kItemRing) * 8);
-                    }
-                    const bool first = p_j == 0, last = p_j == pi.nk - 1;
-                    if (!mbar_wait(&bars[kBarPFull + b], (np / G) & 1, abort_flag) ||
-                        !mbar_wait(&bars[kBarVFull + vs], (np / S) & 1, abort_flag) ||
-                        (first && p_it >= OB &&
-                         !mbar_wait(&bars[kBarOFree + ob], ((p_it / OB) - 1) & 1, abort_flag))) {
+                    if (!ok) break;
+                    umma_commit(&bars[kBarQFree + qs]);
+                }
+                umma_commit(&bars[kBarDrain]);
+                if (!mbar_wait(&bars[kBarDrain], 0, nullptr)) raise_error(kErrTimeout);
+            } else {
+                // ---- PV_n: O += P V, A operand (P) from TMEM
+                constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+                const uint64_t dv0 = desc_mnmajor_sw128(sV, 16384);
+                for (int it = 0; ok; ++it) {
+                    Item I;
+                    if (!take_item(it, false, I)) {
                         ok = false;
                         break;
                     }
-                    tc_fence_after();
-                    const uint64_t dv = dv0 + static_cast<uint64_t>(vs * kStageDesc);
-                    const uint32_t pb = tmem + b * 128;
-                    const uint32_t dst = tmem + C::kTmemO + ob * D;
+                    if (I.nk == 0) break;
+                    const int ob = it % OB;
+                    for (int j = 0; j < I.nk; ++j, ++n) {
+                        const int b = n % G, vs = n % S;
+                        const bool first = j == 0;
+                        if (!mbar_wait(&bars[kBarPFull + b], (n / G) & 1, abort_flag) ||
+                            !mbar_wait(&bars[kBarVFull + vs], (n / S) & 1, abort_flag) ||
+                            (first && it >= OB &&
+                             !mbar_wait(&bars[kBarOFree + ob], ((it / OB) - 1) & 1, abort_flag))) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint64_t dv = dv0 + static_cast<uint64_t>(vs * kStageDesc);
+                        const uint32_t pb = tmem + b * 128;
+                        const uint32_t dst = tmem + C::kTmemO + ob * D;
 #pragma unroll
-                    for (int kk = 0; kk < kTile / 16; ++kk) {
-                        // keys 16kk..16kk+15: columns 32*(kk/2) + 8*(kk%2) of the P buffer
-                        umma_bf16_ts(dst, pb + (kk >> 1) * 32 + (kk & 1) * 8,
-                                     dv + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv,
-                                     (first && kk == 0) ? 0u : 1u);
-                    }
-                    umma_commit(&bars[kBarVFree + vs]);
-                    ++np;
-                    if (last) {
-                        umma_commit(&bars[kBarOFull + b]);   // group b writes this item
-                        mbar_arrive(&bars[kBarItemFree + p_it % kItemRing]);
-                        p_j = 0;
-                        ++p_it;
-                    } else {
-                        ++p_j;
+                        for (int kk = 0; kk < kTile / 16; ++kk) {
+                            // keys 16kk..16kk+15: columns 32*(kk/2) + 8*(kk%2) of the P buffer
+                            umma_bf16_ts(dst, pb + (kk >> 1) * 32 + (kk & 1) * 8,
+                                         dv + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv,
+                                         (first && kk == 0) ? 0u : 1u);
+                        }
+                        umma_commit(&bars[kBarVFree + vs]);
+                        umma_commit(&bars[kBarPVDone + b]);
+                        if (j == I.nk - 1) umma_commit(&bars[kBarOFull + b]);   // group b writes this item
                     }
                 }
+                umma_commit(&bars[kBarDrainPV]);
+                if (!mbar_wait(&bars[kBarDrainPV], 0, nullptr)) raise_error(kErrTimeout);
             }
-            // (the end-of-stream slot is never reused, so it is not released)
-            umma_commit(&bars[kBarDrain]);
-            if (!mbar_wait(&bars[kBarDrain], 0, nullptr)) raise_error(kErrTimeout);
         }
         __syncwarp();
     } else {
