@@ -545,10 +545,12 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                     for (int j = 0; j < I.nk; ++j, ++n) {
                         const int b = n % G, vs = n % S;
                         const bool first = j == 0;
-                        if (!mbar_wait(&bars[kBarPFull + b], (n / G) & 1, abort_flag) ||
-                            !mbar_wait(&bars[kBarVFull + vs], (n / S) & 1, abort_flag) ||
+                        // resources first, right after the previous PV was issued, so
+                        // these tests overlap MMAs already in the pipe; then P_n
+                        if (!mbar_wait(&bars[kBarVFull + vs], (n / S) & 1, abort_flag) ||
                             (first && it >= OB &&
-                             !mbar_wait(&bars[kBarOFree + ob], ((it / OB) - 1) & 1, abort_flag))) {
+                             !mbar_wait(&bars[kBarOFree + ob], ((it / OB) - 1) & 1, abort_flag)) ||
+                            !mbar_wait(&bars[kBarPFull + b], (n / G) & 1, abort_flag)) {
                             ok = false;
                             break;
                         }
