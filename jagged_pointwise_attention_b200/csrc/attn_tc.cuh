@@ -70,7 +70,7 @@
 namespace hstu {
 
 struct AttnArgs {
-    const int4* units;          // plan: (q0, q_end, k0, nk | packed << 31)
+    const int4* units;          // plan: (q0, q_end, k0, nk | nt << 11 | packed << 31)
     const int* unit_count;
     int* item_counter;          // plan: zeroed; next work item to hand out
     const int* row_start;       // plan: first token of each packed row's sequence
@@ -170,16 +170,26 @@ struct Item {
     bool packed;
 };
 
+// Work item w. Items run sequence by sequence, then head, then unit: the
+// units of a sequence are consecutive (nt of them, nt stored in each), so the
+// item block of a sequence starting at unit ubase covers items
+// [H*ubase, H*(ubase + nt)), and unit w / H lies in that sequence.
 __device__ __forceinline__ Item load_item(const AttnArgs& a, int w) {
-    const int u = w / a.H;
-    const int4 wu = a.units[u];
+    const int u1 = w / a.H;
+    const int4 d1 = a.units[u1];
+    const int nk1 = d1.w & 0x7ff, nt = (d1.w >> 11) & 0x7ff;
+    const int ubase = u1 - (nt - nk1);               // units hold tiles nt-1 .. 0
+    const int r = w - a.H * ubase;
+    const int h = r / nt;
+    const int u = ubase + (r - h * nt);
+    const int4 wu = u == u1 ? d1 : a.units[u];
     Item it;
     it.q0 = wu.x;
     it.q_end = wu.y;
     it.k0 = wu.z;
-    it.nk = wu.w & 0x7fffffff;
+    it.nk = wu.w & 0x7ff;
     it.packed = (wu.w >> 31) & 1;
-    it.h = w - u * a.H;
+    it.h = h;
     return it;
 }
 

@@ -1,7 +1,8 @@
 // plan.cuh -- work list of the jagged attention.
 //
 // A work unit is a tile of at most 128 query rows with the key range it needs:
-// (q0, q_end, k0, nk | packed << 31). Two kinds:
+// (q0, q_end, k0, nk | nt << 11 | packed << 31), nt = the number of units of
+// its sequence (1 for packed units). Two kinds:
 //  * aligned: query tile t of a sequence longer than 128 tokens: rows
 //    [o + 128t, min(o + 128t + 128, o + n)), keys from the sequence start
 //    k0 = o, nk = t + 1 key tiles (tiles past the diagonal are causally empty).
@@ -10,13 +11,17 @@
 //    own sequence start is written to row_start[] so the kernel can mask pairs
 //    that cross a sequence boundary. Packing is greedy inside each 128-token
 //    bucket of sequence start positions, so buckets are packed in parallel.
-// Units are listed longest first (descending nk, aligned before packed), so
-// handing them out in list order is greedy longest-processing-time scheduling.
+// Aligned units are listed sequence by sequence, longest sequence first, and
+// inside a sequence by descending query tile (descending nk); packed units
+// follow. The attention kernel hands out work items (unit, head) in the order
+// sequence, head, tile, so the CTAs running at any time share the keys and
+// values of one or two (sequence, head) pairs, which stay in L2, while items
+// still come longest first within each pair.
 //
 // Aligned units are placed without per-unit atomics: sequences are counting-
-// sorted by their tile count nt (descending); the sequences with nt > t are
-// then a prefix of that order, so unit (b, t) goes to slot
-// start[t] + rank(b) where start[t] counts the units of all tiles above t.
+// sorted by their tile count nt (descending); a sequence of rank rho in the
+// bucket of count v starts at unit cum[v] + (rho - base[v]) * v, cum[v]
+// counting the units of all longer buckets.
 #pragma once
 
 #include "common.cuh"
@@ -35,7 +40,7 @@ plan_kernel(const int64_t* __restrict__ seq_offsets, int B, int64_t T, int max_s
     const int NT = max_tiles + 1;        // tile counts 0..max_tiles
     int* cnt = plan_smem;                // sequences with nt == v
     int* base = cnt + NT;                // first rank of nt == v in the descending order
-    int* start = base + NT;              // first slot of query tile t
+    int* cum = base + NT;                // first unit of the sequences with nt == v
     __shared__ int n_aligned, n_packed;
     const bool cache = B < kPlanSmemOffsets;
     int64_t* off_s = reinterpret_cast<int64_t*>(plan_smem + ((3 * NT + 1) & ~1));
@@ -68,34 +73,33 @@ plan_kernel(const int64_t* __restrict__ seq_offsets, int B, int64_t T, int max_s
     }
     __syncthreads();
     if (tid == 0) {
-        int rank = 0, slots = 0, ge = 0;   // ge: sequences with nt > t
+        int rank = 0, slots = 0;
         for (int v = max_tiles; v >= 1; --v) {
             base[v] = rank;
+            cum[v] = slots;
             rank += cnt[v];
-        }
-        for (int t = max_tiles - 1; t >= 0; --t) {
-            ge += cnt[t + 1];
-            start[t] = slots;
-            slots += ge;
+            slots += cnt[v] * v;
         }
         n_aligned = slots;
         for (int v = 0; v < NT; ++v) cnt[v] = 0;   // reused as fill counters
     }
     __syncthreads();
-    // aligned units: one rank per sequence, then its nt slots
+    // aligned units: one rank per sequence, then its nt consecutive slots,
+    // tile nt-1 first
     for (int b = tid; b < B; b += blockDim.x) {
         const int64_t n = length(b);
         const int nt = tiles_of(n);
         if (nt == 0) continue;
-        const int rank = base[nt] + atomicAdd(&cnt[nt], 1);
+        const int ubase = cum[nt] + atomicAdd(&cnt[nt], 1) * nt;
         const int64_t o = off[b];
-        for (int t = 0; t < nt; ++t) {
-            const int slot = start[t] + rank;
+        for (int k = 0; k < nt; ++k) {
+            const int t = nt - 1 - k;
+            const int slot = ubase + k;
             if (slot < max_units) {
                 const int64_t q0 = o + static_cast<int64_t>(t) * kTile;
                 const int64_t qe = q0 + kTile < o + n ? q0 + kTile : o + n;
                 units[slot] = make_int4(static_cast<int>(q0), static_cast<int>(qe),
-                                        static_cast<int>(o), t + 1);
+                                        static_cast<int>(o), (t + 1) | (nt << 11));
             }
         }
     }
@@ -152,7 +156,7 @@ plan_kernel(const int64_t* __restrict__ seq_offsets, int B, int64_t T, int max_s
                 const int slot = n_aligned + my0 + k;
                 if (slot < max_units)
                     units[slot] = make_int4(static_cast<int>(ts0), static_cast<int>(te),
-                                            static_cast<int>(ts0), static_cast<int>(0x80000001u));
+                                            static_cast<int>(ts0), static_cast<int>(0x80000801u));
             });
         }
     }
