@@ -284,8 +284,30 @@ def bench_attention(args, rank, world, local, peaks, peak_kind):
     if st != 0:
         raise RuntimeError("device status %d after warm-up" % st)
 
+    # Kernel-only time of the attention launch (roofline): eager steps with
+    # events around the run call, outside the timed region.
     kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        step(i, kev[i])
+    torch.cuda.synchronize(dev)
+    kernel_ms = [a.elapsed_time(b) for a, b in kev]
+
+    # The timed steps replay one CUDA graph per input copy (plan + run), so the
+    # host's launch cost is not part of the step time.
+    graphs = []
+    if not args.no_graph:
+        for i in range(ncopies):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                step(i)
+            graphs.append(g)
+        for i in range(ncopies):
+            graphs[i].replay()
+        torch.cuda.synchronize(dev)
+        stream = torch.cuda.current_stream(dev)
+
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local)
     _barrier(world)
@@ -293,13 +315,16 @@ def bench_attention(args, rank, world, local, peaks, peak_kind):
     sampler.start()
     e0.record(stream)
     for i in range(args.steps):
-        step(i, kev[i])
+        if graphs:
+            graphs[i % ncopies].replay()
+        else:
+            step(i)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     sampler.stop()
     _barrier(world)
     local_ms = e0.elapsed_time(e1)
-    kernel_ms = [a.elapsed_time(b) for a, b in kev]
+    del graphs
     st = hstu.hstu_device_status()
     if st != 0:
         raise RuntimeError("device status %d after timed steps" % st)
@@ -352,7 +377,8 @@ def bench_attention(args, rank, world, local, peaks, peak_kind):
                    int(inp.time_bias.shape[1]), "seed": seed, "parallelism": "dp%d" % world,
                    "l2": ("inputs %.0f MB > L2" % (in_bytes / 2 ** 20)) if ncopies == 1 else
                          ("rotating %d input copies (%.0f MB) > 2x L2" %
-                          (ncopies, ncopies * in_bytes / 2 ** 20))},
+                          (ncopies, ncopies * in_bytes / 2 ** 20)),
+                   "launch": "eager" if args.no_graph else "CUDA graph per step (plan + run)"},
         "pct_of_bf16_peak": {"measured_burst": round(100 * value / peaks["bf16_tflops"], 2),
                              "nominal_2250": round(100 * value / NOMINAL_BF16_TFLOPS, 2)},
         "tokens_per_s": round(total_tokens / (max_ms * 1e-3), 1),
@@ -528,6 +554,9 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--reference-budget-s", type=float, default=120.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch the timed steps one call at a time instead of replaying "
+                         "CUDA graphs")
     a = ap.parse_args(argv)
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")

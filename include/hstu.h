@@ -78,9 +78,10 @@ hstu_status_t hstu_device_status(void* stream);
 
 /* Workspace bytes that hstu_attn_plan / hstu_attn_fwd need for a batch of B
  * sequences, total_tokens tokens and the given max_seqlen (bf16 path; the
- * fp32 path needs none): a 256-byte header, 16 bytes per work unit (at most
- * min(total_tokens/128 + B + 1, B * ceil(max_seqlen/128)) units, rounded up
- * to 256 bytes) and 4 bytes per token. Returns 0 for invalid sizes. */
+ * fp32 path needs none): a 256-byte header and 32 bytes per work unit (its
+ * descriptor and the sequence-start mask of a packed tile; at most
+ * min(total_tokens/128 + B + 1, B * ceil(max_seqlen/128)) units, each array
+ * rounded up to 256 bytes). Returns 0 for invalid sizes. */
 size_t hstu_attn_workspace_bytes(int32_t B, int64_t total_tokens, int32_t max_seqlen);
 
 /* Builds the work list of the bf16 attention in `workspace` (device):
@@ -144,8 +145,8 @@ hstu_status_t hstu_attn_fwd(hstu_dtype_t dtype,
  * HSTU_NOALLOC_SCRATCH_BYTES (1 MiB), which every GPU that loads the library
  * holds until the process exits. A batch needing more than that, i.e.
  * hstu_attn_workspace_bytes(B, total_tokens, max_seqlen) > 1 MiB (the work
- * list takes 16 bytes per 128-query tile plus 4 bytes per token: roughly
- * total_tokens > 250,000), returns
+ * list takes 32 bytes per unit: roughly B + total_tokens/128 > 32,700),
+ * returns
  * HSTU_ERR_UNSUPPORTED before anything is launched; use hstu_attn_fwd then.
  * Nothing is allocated or freed by this call, including by torch or any
  * other library.

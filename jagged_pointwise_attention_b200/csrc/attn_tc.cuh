@@ -73,7 +73,7 @@ struct AttnArgs {
     const int4* units;          // plan: (q0, q_end, k0, nk | nt << 11 | packed << 31)
     const int* unit_count;
     int* item_counter;          // plan: zeroed; next work item to hand out
-    const int* row_start;       // plan: first token of each packed row's sequence
+    const uint4* starts;        // plan: per packed unit, rows where a sequence begins
     int H;
     int64_t T;
     const int64_t* ts;          // [T] or null
@@ -164,9 +164,10 @@ enum {
 };
 static_assert(kBarCount == AttnSmem<64, kAttnGroups>::kNumBars, "barrier slots");
 
-// A work item as the scheduler publishes it; nk == 0 ends the stream.
+// A work item as the scheduler publishes it; nk == 0 ends the stream. s0: the
+// unit index (packed tiles look up their sequence starts with it).
 struct Item {
-    int q0, q_end, k0, nk, h;
+    int q0, q_end, k0, nk, h, s0;
     bool packed;
 };
 
@@ -186,9 +187,10 @@ __device__ __forceinline__ Item load_item(const AttnArgs& a, int w) {
     Item it;
     it.q0 = wu.x;
     it.q_end = wu.y;
-    it.k0 = wu.z;
-    it.nk = wu.w & 0x7ff;
     it.packed = (wu.w >> 31) & 1;
+    it.k0 = wu.z;
+    it.s0 = u;
+    it.nk = wu.w & 0x7ff;
     it.h = h;
     return it;
 }
@@ -201,6 +203,7 @@ __device__ __forceinline__ Item read_item(const volatile int* slot) {
     it.nk = slot[3];
     it.h = slot[4];
     it.packed = slot[5] != 0;
+    it.s0 = slot[6];
     return it;
 }
 
@@ -318,6 +321,21 @@ __device__ __forceinline__ void pw_slow(const uint32_t* sv, int c0, const uint4*
     }
 }
 
+// First token of row q0 + r's sequence in a packed tile: the highest marked
+// row <= r of the tile's sequence-start mask (row 0 is always marked). Rows
+// past the tile's end get a start past every key.
+__device__ __forceinline__ int packed_row_start(const AttnArgs& a, const Item& I, int r) {
+    if (I.q0 + r >= I.q_end) return 0x7fffffff;
+    const uint4 m4 = __ldg(a.starts + I.s0);
+    const uint32_t m[4] = {m4.x, m4.y, m4.z, m4.w};
+    int w = r >> 5;
+    uint32_t x = m[w] & (0xffffffffu >> (31 - (r & 31)));   // marks at rows <= r of word w
+#pragma unroll
+    for (int k = 0; k < 3; ++k)
+        if (x == 0u && w > 0) x = m[--w];
+    return I.q0 + 32 * w + 31 - __clz(x);
+}
+
 template <int D, int G>
 __global__ void __launch_bounds__(AttnCfg<D, G>::kThreads, 1)
 attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
@@ -430,7 +448,7 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                     if (w < n_items) {
                         I = load_item(args, w);
                     } else {
-                        I.q0 = I.q_end = I.k0 = I.h = 0;
+                        I.q0 = I.q_end = I.k0 = I.h = I.s0 = 0;
                         I.nk = 0;
                         I.packed = false;
                     }
@@ -441,6 +459,7 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                     e[3] = I.nk;
                     e[4] = I.h;
                     e[5] = I.packed ? 1 : 0;
+                    e[6] = I.s0;
                     mbar_arrive(&bars[kBarItemFull + slot]);
                 } else if (!take_item(it, false, I)) {
                     ok = false;
@@ -654,7 +673,7 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
             // sequence, and this lane's entry of the head's register time table
             // (lane L holds time/2 of bucket min((L + 1) mod 32, NB - 1))
             const int64_t ti = (use_time && row_valid) ? __ldg(args.ts + i) : 0;
-            const int rs = (I.packed && row_valid) ? __ldg(args.row_start + i) : I.k0;
+            const int rs = I.packed ? packed_row_start(args, I, r) : I.k0;
             const float tbr = use_time ? 0.5f * __ldg(args.tb + static_cast<int64_t>(I.h) * args.NB +
                                                       min((lane + 1) & 31, nbm1))
                                        : 0.f;

@@ -92,7 +92,7 @@ int64_t max_units_of(int32_t B, int64_t T, int32_t max_seqlen) {
 
 constexpr size_t kAttnWsHeader = 256;   // unit count (int at 0), item counters (2 ints at 16)
 
-// attention workspace: [header][units: int4 x max_units][row_start: int32 x T]
+// attention workspace: [header][units: int4 x max_units][starts: uint4 x max_units]
 size_t attn_units_bytes(int32_t B, int64_t T, int32_t max_seqlen) {
     return (static_cast<size_t>(max_units_of(B, T, max_seqlen)) * 16 + 255) / 256 * 256;
 }
@@ -192,8 +192,8 @@ hstu_status_t run_attn(const AttnCall& c) {
     AttnArgs a{reinterpret_cast<const int4*>(ws + kAttnWsHeader),
                reinterpret_cast<const int*>(ws),
                reinterpret_cast<int*>(const_cast<uint8_t*>(ws) + 16),
-               reinterpret_cast<const int*>(ws + kAttnWsHeader +
-                                            attn_units_bytes(c.B, c.T, c.max_seqlen)),
+               reinterpret_cast<const uint4*>(ws + kAttnWsHeader +
+                                              attn_units_bytes(c.B, c.T, c.max_seqlen)),
                c.H,
                c.T,
                use_time ? c.ts : nullptr,
@@ -237,9 +237,9 @@ hstu_status_t plan_attn(const int64_t* off, int32_t B, int64_t T, int32_t max_se
     if (B < kPlanSmemOffsets) smem += static_cast<size_t>(B + 1) * sizeof(int64_t);
     plan_kernel<<<1, 1024, smem, stream>>>(
         off, B, T, max_seqlen, max_tiles, static_cast<int>(max_units),
-        reinterpret_cast<int4*>(w + kAttnWsHeader), reinterpret_cast<int*>(w),
-        reinterpret_cast<int*>(w + 16),
-        reinterpret_cast<int*>(w + kAttnWsHeader + attn_units_bytes(B, T, max_seqlen)));
+        reinterpret_cast<int4*>(w + kAttnWsHeader),
+        reinterpret_cast<uint4*>(w + kAttnWsHeader + attn_units_bytes(B, T, max_seqlen)),
+        reinterpret_cast<int*>(w), reinterpret_cast<int*>(w + 16));
     return launch_status();
 }
 
@@ -356,8 +356,7 @@ hstu_status_t hstu_device_status(void* stream) {
 
 size_t hstu_attn_workspace_bytes(int32_t B, int64_t total_tokens, int32_t max_seqlen) {
     if (!plan_sizes_ok(B, total_tokens, max_seqlen)) return 0;
-    return kAttnWsHeader + attn_units_bytes(B, total_tokens, max_seqlen) +
-           static_cast<size_t>(total_tokens) * sizeof(int);
+    return kAttnWsHeader + 2 * attn_units_bytes(B, total_tokens, max_seqlen);
 }
 
 hstu_status_t hstu_attn_plan(const int64_t* seq_offsets, int32_t B, int64_t total_tokens,

@@ -7,10 +7,12 @@
 //    [o + 128t, min(o + 128t + 128, o + n)), keys from the sequence start
 //    k0 = o, nk = t + 1 key tiles (tiles past the diagonal are causally empty).
 //  * packed: several whole sequences of at most 128 tokens each, consecutive in
-//    the batch, sharing one tile: rows [q0, q_end) = keys, nk = 1. Each row's
-//    own sequence start is written to row_start[] so the kernel can mask pairs
-//    that cross a sequence boundary. Packing is greedy inside each 128-token
-//    bucket of sequence start positions, so buckets are packed in parallel.
+//    the batch, sharing one tile: rows [q0, q_end) = keys, nk = 1 (k0 = q0).
+//    starts[u] marks the rows of the tile where a sequence begins (bit r of
+//    the 128-bit mask = row q0 + r), from which the kernel finds each row's
+//    own sequence start to mask pairs that cross a sequence boundary. Packing
+//    is greedy inside each 128-token bucket of sequence start positions, so
+//    buckets are packed in parallel.
 // Aligned units are listed sequence by sequence, longest sequence first, and
 // inside a sequence by descending query tile (descending nk); packed units
 // follow. The attention kernel hands out work items (unit, head) in the order
@@ -31,22 +33,25 @@ namespace hstu {
 constexpr int kPlanSmemOffsets = 4096;    // offsets cached in shared memory below this B
 
 // One block of 1024 threads. Dynamic shared memory: 3 * (max_tiles + 1) ints,
-// then (B + 1) int64 offsets when B < kPlanSmemOffsets.
-__global__ void __launch_bounds__(1024)
-plan_kernel(const int64_t* __restrict__ seq_offsets, int B, int64_t T, int max_seqlen,
-            int max_tiles, int max_units, int4* __restrict__ units, int* __restrict__ unit_count,
-            int* __restrict__ item_counter, int* __restrict__ row_start) {
-    extern __shared__ int plan_smem[];
+// then (B + 1) int64 offsets when B < kPlanSmemOffsets. The body is compiled
+// once for offsets in shared memory (kCache) and once for offsets read from
+// global memory: a pointer that may be either makes every offset load a
+// generic load, which then waits behind the thread's global stores.
+template <bool kCache>
+__device__ __forceinline__ void plan_body(const int64_t* __restrict__ seq_offsets, int B, int64_t T,
+                                          int max_seqlen, int max_tiles, int max_units,
+                                          int4* __restrict__ units, uint4* __restrict__ starts,
+                                          int* __restrict__ unit_count,
+                                          int* __restrict__ item_counter, int* plan_smem) {
     const int NT = max_tiles + 1;        // tile counts 0..max_tiles
     int* cnt = plan_smem;                // sequences with nt == v
     int* base = cnt + NT;                // first rank of nt == v in the descending order
     int* cum = base + NT;                // first unit of the sequences with nt == v
     __shared__ int n_aligned, n_packed;
-    const bool cache = B < kPlanSmemOffsets;
     int64_t* off_s = reinterpret_cast<int64_t*>(plan_smem + ((3 * NT + 1) & ~1));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
     for (int v = tid; v < NT; v += blockDim.x) cnt[v] = 0;
-    if (cache)
+    if (kCache)
         for (int b = tid; b <= B; b += blockDim.x) off_s[b] = seq_offsets[b];
     if (tid == 0) {
         n_packed = 0;
@@ -54,7 +59,7 @@ plan_kernel(const int64_t* __restrict__ seq_offsets, int B, int64_t T, int max_s
         item_counter[1] = 0;   // CTAs finished
     }
     __syncthreads();
-    const int64_t* off = cache ? off_s : seq_offsets;
+    const int64_t* __restrict__ off = kCache ? off_s : seq_offsets;
     auto length = [&](int b) -> int64_t {
         int64_t n = off[b + 1] - off[b];
         if (n < 0 || n > max_seqlen) {
@@ -122,25 +127,29 @@ plan_kernel(const int64_t* __restrict__ seq_offsets, int B, int64_t T, int max_s
                 }
             }
         }
-        // greedy pass; emit(k, ts0, te) is called for the k-th unit of the bucket
+        // greedy pass; emit(k, ts0, te, c0) is called for the k-th unit of the
+        // bucket (tokens [ts0, te), first sequence c0)
         auto pack = [&](auto emit) {
-            int k = 0;
+            int k = 0, cs = -1;
             int64_t ts0 = -1, te = -1;
             for (int c = b; c < B && off[c] / kTile == bucket; ++c) {
                 const int64_t nc = length(c);
                 if (nc == 0) continue;
                 if (nc > kTile) break;               // a long sequence ends the run
                 if (ts0 >= 0 && off[c] + nc - ts0 > kTile) {
-                    emit(k++, ts0, te);
+                    emit(k++, ts0, te, cs);
                     ts0 = -1;
                 }
-                if (ts0 < 0) ts0 = off[c];
+                if (ts0 < 0) {
+                    ts0 = off[c];
+                    cs = c;
+                }
                 te = off[c] + nc;
             }
-            if (ts0 >= 0) emit(k++, ts0, te);
+            if (ts0 >= 0) emit(k++, ts0, te, cs);
             return k;
         };
-        const int mine = first ? pack([](int, int64_t, int64_t) {}) : 0;
+        const int mine = first ? pack([](int, int64_t, int64_t, int) {}) : 0;
         int incl = mine;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -152,27 +161,39 @@ plan_kernel(const int64_t* __restrict__ seq_offsets, int B, int64_t T, int max_s
         wbase = __shfl_sync(0xffffffffu, wbase, 31);
         if (first) {
             const int my0 = wbase + incl - mine;
-            pack([&](int k, int64_t ts0, int64_t te) {
+            pack([&](int k, int64_t ts0, int64_t te, int cs) {
                 const int slot = n_aligned + my0 + k;
-                if (slot < max_units)
+                if (slot < max_units) {
                     units[slot] = make_int4(static_cast<int>(ts0), static_cast<int>(te),
                                             static_cast<int>(ts0), static_cast<int>(0x80000801u));
+                    uint32_t m[4] = {0u, 0u, 0u, 0u};
+                    for (int c = cs; c < B && off[c] < te; ++c) {
+                        const int r = static_cast<int>(off[c] - ts0);
+                        m[r >> 5] |= 1u << (r & 31);
+                    }
+                    starts[slot] = make_uint4(m[0], m[1], m[2], m[3]);
+                }
             });
         }
-    }
-    // row_start of every short sequence's tokens, one warp per sequence (coalesced)
-    for (int b = warp; b < B; b += nwarps) {
-        const int64_t o = off[b];
-        const int64_t n = length(b);
-        if (n == 0 || n > kTile) continue;
-        for (int64_t i = o + lane; i < o + n; i += 32)
-            if (i < T) row_start[i] = static_cast<int>(o);
     }
     __syncthreads();
     if (tid == 0) {
         const int total = n_aligned + n_packed;
         *unit_count = total < max_units ? total : max_units;
     }
+}
+
+__global__ void __launch_bounds__(1024)
+plan_kernel(const int64_t* __restrict__ seq_offsets, int B, int64_t T, int max_seqlen,
+            int max_tiles, int max_units, int4* __restrict__ units, uint4* __restrict__ starts,
+            int* __restrict__ unit_count, int* __restrict__ item_counter) {
+    extern __shared__ int plan_smem[];
+    if (B < kPlanSmemOffsets)
+        plan_body<true>(seq_offsets, B, T, max_seqlen, max_tiles, max_units, units, starts,
+                        unit_count, item_counter, plan_smem);
+    else
+        plan_body<false>(seq_offsets, B, T, max_seqlen, max_tiles, max_units, units, starts,
+                         unit_count, item_counter, plan_smem);
 }
 
 }  // namespace hstu

@@ -53,9 +53,10 @@ def test_library_loads_without_gpu(lib):
 def test_workspace_queries(lib):
     w = lib.hstu_attn_workspace_bytes(16, 90000, 8192)
     # header + one int4 per (sequence, query tile), bounded by T/128 + B + 1 and
-    # rounded up to 256 bytes, then one int32 sequence start per token
+    # rounded up to 256 bytes, and as much again for the per-unit sequence-start
+    # masks of packed tiles
     units = 16 * min(90000 // 128 + 16 + 1, 16 * 64)
-    assert w == 256 + (units + 255) // 256 * 256 + 4 * 90000
+    assert w == 256 + 2 * ((units + 255) // 256 * 256)
     assert lib.hstu_attn_workspace_bytes(-1, 10, 10) == 0
     assert lib.hstu_attn_workspace_bytes(1, 10, 0) == 0
     assert lib.hstu_attn_workspace_bytes(1, 10, 131073) == 0
