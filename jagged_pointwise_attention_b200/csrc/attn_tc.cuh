@@ -261,6 +261,35 @@ __device__ __forceinline__ void pw_const(const uint32_t* sv, const uint4* wbk, u
     }
 }
 
+// Two time buckets over an unmasked chunk: scores whose time difference is
+// at least thr (a power of two) take th, the others tl; the same bits as a
+// bucket per score whenever every score's bucket is one of the two.
+__device__ __forceinline__ void pw_two(const uint32_t* sv, int c0, const uint4* wbk,
+                                       const int32_t* __restrict__ kt32, int32_t ti32, int32_t thr,
+                                       float tl, float th, uint32_t* pk) {
+    const int4* k4 = reinterpret_cast<const int4*>(kt32 + c0);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint4 W = wbk[8 * q];
+        const uint32_t wv[4] = {W.x, W.y, W.z, W.w};
+        const int4 ka = k4[2 * q], kb = k4[2 * q + 1];
+        const int32_t kv[8] = {ka.x, ka.y, ka.z, ka.w, kb.x, kb.y, kb.z, kb.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            float tv[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int32_t dt = static_cast<int32_t>(static_cast<uint32_t>(ti32) -
+                                                        static_cast<uint32_t>(kv[2 * u + e]));
+                tv[e] = dt >= thr ? th : tl;
+            }
+            const int p = 4 * q + u;
+            pk[p] = silu_of_half_bf16x2(
+                half_arg_bf16x2(sv[2 * p], sv[2 * p + 1], wv[u], pack_bf16x2(tv[0], tv[1])));
+        }
+    }
+}
+
 // Bucket per score, differences exact in 32 bits. tbr: this lane's entry of
 // the register table (lane L holds time/2 of bucket min((L+1) mod 32, NB-1)).
 template <bool kMask>
@@ -725,20 +754,29 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                             const int lastc = static_cast<int>(args.T - 1 - kt0);
                             if (full) pw_slow<false>(sv, c0, wbr + c0, args.ts + kt0, lastc, ti, tbh, nbm1, lo, hi, pk);
                             else pw_slow<true>(sv, c0, wbr + c0, args.ts + kt0, lastc, ti, tbh, nbm1, lo, hi, pk);
-                        } else if (full) {
-                            // the bucket at the chunk's largest and smallest dt
-                            float tconst = 0.f;
-                            bool cst = true;
-                            if (use_time) {
-                                const uint32_t ef_hi = log2_exponent_field(static_cast<uint32_t>(max(tib - st.cmin[q], 1)));
-                                const uint32_t ef_lo = log2_exponent_field(static_cast<uint32_t>(max(tib - st.cmax[q], 1)));
-                                tconst = __shfl_sync(0xffffffffu, tbr, static_cast<int>(ef_lo));
-                                cst = __all_sync(0xffffffffu, ef_hi == ef_lo);
-                            }
-                            if (cst) pw_const(sv, wbr + c0, pack_bf16x2(tconst, tconst), pk);
-                            else pw_fast<false>(sv, c0, wbr + c0, st.kt32, ti32, tbr, lo, hi, pk);
                         } else {
-                            pw_fast<true>(sv, c0, wbr + c0, st.kt32, ti32, tbr, lo, hi, pk);
+                            // an unmasked chunk sees one or two buckets over its key range
+                            // in most rows (tested at its largest and smallest dt); the
+                            // rest take a bucket per score
+                            int path = 2;
+                            float tl = 0.f, th = 0.f;
+                            int32_t thr = 0x7fffffff;
+                            if (full) {
+                                path = 0;
+                                if (use_time) {
+                                    const uint32_t ef_hi = log2_exponent_field(static_cast<uint32_t>(max(tib - st.cmin[q], 1)));
+                                    const uint32_t ef_lo = log2_exponent_field(static_cast<uint32_t>(max(tib - st.cmax[q], 1)));
+                                    tl = __shfl_sync(0xffffffffu, tbr, static_cast<int>(ef_lo));
+                                    th = __shfl_sync(0xffffffffu, tbr, static_cast<int>(ef_hi));
+                                    // bucket ef_hi iff dt >= 2^(ef_hi - 1023) (>= 2 when ef_hi > ef_lo)
+                                    if (ef_hi > ef_lo) thr = 1 << (ef_hi - 1023u);
+                                    path = __all_sync(0xffffffffu, ef_hi == ef_lo) ? 0
+                                           : __all_sync(0xffffffffu, ef_hi - ef_lo <= 1u) ? 1 : 2;
+                                }
+                            }
+                            if (path == 0) pw_const(sv, wbr + c0, pack_bf16x2(tl, tl), pk);
+                            else if (path == 1) pw_two(sv, c0, wbr + c0, st.kt32, ti32, thr, tl, th, pk);
+                            else pw_fast<true>(sv, c0, wbr + c0, st.kt32, ti32, tbr, lo, hi, pk);
                         }
                         // 32 bf16 results -> columns 32q..32q+15 of the S buffer just read
                         tmem_st16(s_col + c0, pk);
