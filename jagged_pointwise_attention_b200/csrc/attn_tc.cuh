@@ -655,8 +655,16 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                         const float* prow = args.pos + static_cast<int64_t>(I.h) * args.P;
                         const int rel0 = I.q0 - kt0 + 127 - se;
                         float v[8];
+                        if (rel0 >= 7 && rel0 < args.P) {
+                            // the whole entry lies inside the table (all tiles but the
+                            // diagonal one and those past the table's end)
+                            const float* pe = prow + rel0;
 #pragma unroll
-                        for (int u = 0; u < 8; ++u) v[u] = __ldg(prow + min(max(rel0 - u, 0), args.P - 1));
+                            for (int u = 0; u < 8; ++u) v[u] = __ldg(pe - u);
+                        } else {
+#pragma unroll
+                            for (int u = 0; u < 8; ++u) v[u] = __ldg(prow + min(max(rel0 - u, 0), args.P - 1));
+                        }
 #pragma unroll
                         for (int u = 0; u < 4; ++u) wd[u] = pack_bf16x2(0.5f * v[2 * u], 0.5f * v[2 * u + 1]);
                     }
