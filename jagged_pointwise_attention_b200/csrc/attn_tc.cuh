@@ -665,8 +665,12 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
 #pragma unroll
                             for (int u = 0; u < 8; ++u) v[u] = __ldg(prow + min(max(rel0 - u, 0), args.P - 1));
                         }
+                        // bf16(v) / 2 is exactly bf16(v / 2) (a power-of-two scale)
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) wd[u] = pack_bf16x2(0.5f * v[2 * u], 0.5f * v[2 * u + 1]);
+                        for (int u = 0; u < 4; ++u) {
+                            const uint32_t b2 = pack_bf16x2(v[2 * u], v[2 * u + 1]);
+                            asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(wd[u]) : "r"(b2), "r"(0x3f003f00u));
+                        }
                     }
                     st.wb[se] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
                 }
@@ -742,11 +746,15 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                     }
                     const bool fast_w = __all_sync(0xffffffffu, fast);
                     const uint4* wbr = st.wb + (127 - r);        // entry k0 of chunk 0
+                    // no pair of the tile masked for any row of the warp (every tile
+                    // but the diagonal one of an aligned unit): no per-chunk tests
+                    const bool tile_full = __all_sync(0xffffffffu, lo <= 0 && hi >= 127);
 #pragma unroll 1
                     for (int q = 0; q < 4; ++q) {
                         const int c0 = 32 * q;
                         uint32_t pk[16];
-                        const bool live = __any_sync(0xffffffffu, row_valid && hi >= c0 &&
+                        const bool live = tile_full ||
+                                          __any_sync(0xffffffffu, row_valid && hi >= c0 &&
                                                                       lo <= c0 + 31 && lo <= hi);
                         if (!live) {                        // every pair of the chunk is masked
 #pragma unroll
@@ -757,7 +765,7 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                         uint32_t sv[32];
                         __syncwarp();
                         tmem_ld32(s_col + c0, sv);
-                        const bool full = __all_sync(0xffffffffu, lo <= c0 && hi >= c0 + 31);
+                        const bool full = tile_full || __all_sync(0xffffffffu, lo <= c0 && hi >= c0 + 31);
                         if (!fast_w) {
                             const int lastc = static_cast<int>(args.T - 1 - kt0);
                             if (full) pw_slow<false>(sv, c0, wbr + c0, args.ts + kt0, lastc, ti, tbh, nbm1, lo, hi, pk);
