@@ -115,6 +115,7 @@ struct AttnCfg {
 // chunk's smallest and largest key timestamp minus base.
 struct alignas(16) BiasStage {
     uint4 wb[248];         // sliding-window table of bf16 pos/2
+    uint32_t r32[128];     // its source: word m packs R[2m], R[2m+1] (R[255] = 0)
     int32_t kt32[128];     // low 32 bits of the key timestamps
     int64_t base;          // timestamp of the tile's first key
     int32_t cmin[4], cmax[4], ok[4];
@@ -131,7 +132,7 @@ struct AttnSmem {
     static constexpr int kOffStage = kOffV + C::kStages * kTileBytes;   // BiasStage[2G]
     static constexpr int kOffItems = kOffStage + 2 * G * static_cast<int>(sizeof(BiasStage));
     static constexpr int kOffBar = kOffItems + kItemRing * 32;                // int[8] per slot
-    static constexpr int kNumBars = 56;
+    static constexpr int kNumBars = 64;
     static constexpr int kOffTmem = kOffBar + kNumBars * 8;
     static constexpr int kOffAbort = kOffTmem + 8;
     static constexpr int kBytes = kOffAbort + 8;
@@ -160,7 +161,8 @@ enum {
     kBarStage = 46,     // +2g+s (up to 6): the 128 threads of group g staged stage s
     kBarPVDone = 52,    // +buffer (up to 3): PV of the buffer's tile has completed
     kBarDrainPV = 55,   // the PV issuer's last commit
-    kBarCount = 56,
+    kBarStageSrc = 56,  // +2g+s (up to 6): group g wrote the window source words of stage s
+    kBarCount = 64,
 };
 static_assert(kBarCount == AttnSmem<64, kAttnGroups>::kNumBars, "barrier slots");
 
@@ -413,6 +415,8 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
             mbar_init(&bars[kBarPFull + b], 128);
             mbar_init(&bars[kBarStage + 2 * b], 128);
             mbar_init(&bars[kBarStage + 2 * b + 1], 128);
+            mbar_init(&bars[kBarStageSrc + 2 * b], 128);
+            mbar_init(&bars[kBarStageSrc + 2 * b + 1], 128);
         }
         for (int b = 0; b < G; ++b) mbar_init(&bars[kBarOFull + b], 1);
         for (int o = 0; o < OB; ++o) mbar_init(&bars[kBarOFree + o], 128);
@@ -642,37 +646,39 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
         const uint32_t s_col = tmem + lane_base + static_cast<uint32_t>(g * 128);
 
         // Stage the bias data of key tile kt0 of item I (every thread of the
-        // group takes part: table entries r and r + 128, key r, and the
+        // group takes part: window source word r, then after the group has
+        // written all of them table entries r and r + 128; key r, and the
         // timestamp summary of chunk qd, whose keys are this warp's lanes).
-        auto stage_tile = [&](const Item& I, int kt0, BiasStage& st, uint64_t* full) {
+        auto stage_tile = [&](const Item& I, int kt0, BiasStage& st, uint64_t* full, uint64_t* src,
+                              uint32_t src_parity) -> bool {
+            {
+                // word r = (R[2r], R[2r+1]), R[k] = pos[h][clamp(i - j)] / 2 with
+                // i - j = q0 - kt0 + 127 - k, and R[255] = 0
+                uint32_t wd = 0u;
+                if (args.pos) {
+                    const float* prow = args.pos + static_cast<int64_t>(I.h) * args.P;
+                    const int rel0 = I.q0 - kt0 + 127 - 2 * r;
+                    const float v0 = __ldg(prow + min(max(rel0, 0), args.P - 1));
+                    const float v1 = r < 127 ? __ldg(prow + min(max(rel0 - 1, 0), args.P - 1)) : 0.f;
+                    // bf16(v) / 2 is exactly bf16(v / 2) (a power-of-two scale)
+                    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(wd) : "r"(pack_bf16x2(v0, v1)), "r"(0x3f003f00u));
+                }
+                st.r32[r] = wd;
+            }
+            mbar_arrive(src);
+            if (!warp_wait(src, src_parity, abort_flag)) return false;
+            // entry s = R[s..s+7]: words s/2 .. s/2+4, shifted by one half for odd s
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 const int se = r + 128 * e;
                 if (se < 248) {
-                    uint32_t wd[4] = {0u, 0u, 0u, 0u};
-                    if (args.pos) {
-                        // R[k] = pos[h][clamp(i - j)] with i - j = q0 - kt0 + 127 - k
-                        const float* prow = args.pos + static_cast<int64_t>(I.h) * args.P;
-                        const int rel0 = I.q0 - kt0 + 127 - se;
-                        float v[8];
-                        if (rel0 >= 7 && rel0 < args.P) {
-                            // the whole entry lies inside the table (all tiles but the
-                            // diagonal one and those past the table's end)
-                            const float* pe = prow + rel0;
+                    const int w0 = se >> 1;
+                    const uint32_t sel = (se & 1) ? 0x5432u : 0x3210u;
+                    uint32_t x[5];
 #pragma unroll
-                            for (int u = 0; u < 8; ++u) v[u] = __ldg(pe - u);
-                        } else {
-#pragma unroll
-                            for (int u = 0; u < 8; ++u) v[u] = __ldg(prow + min(max(rel0 - u, 0), args.P - 1));
-                        }
-                        // bf16(v) / 2 is exactly bf16(v / 2) (a power-of-two scale)
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const uint32_t b2 = pack_bf16x2(v[2 * u], v[2 * u + 1]);
-                            asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(wd[u]) : "r"(b2), "r"(0x3f003f00u));
-                        }
-                    }
-                    st.wb[se] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+                    for (int k = 0; k < 5; ++k) x[k] = st.r32[w0 + k];
+                    st.wb[se] = make_uint4(__byte_perm(x[0], x[1], sel), __byte_perm(x[1], x[2], sel),
+                                           __byte_perm(x[2], x[3], sel), __byte_perm(x[3], x[4], sel));
                 }
             }
             const int64_t key = static_cast<int64_t>(kt0) + r;
@@ -695,6 +701,7 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
             }
             if (r == 0) st.base = base;
             mbar_arrive(full);
+            return true;
         };
 
         bool ok = true;
@@ -725,8 +732,9 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                 const int kt0 = I.k0 + j * kTile;
                 const int sb = nt & 1;
                 BiasStage& st = stages[2 * g + sb];
-                stage_tile(I, kt0, st, &bars[kBarStage + 2 * g + sb]);
-                if (!warp_wait(&bars[kBarStage + 2 * g + sb], (nt >> 1) & 1, abort_flag) ||
+                if (!stage_tile(I, kt0, st, &bars[kBarStage + 2 * g + sb],
+                                &bars[kBarStageSrc + 2 * g + sb], (nt >> 1) & 1) ||
+                    !warp_wait(&bars[kBarStage + 2 * g + sb], (nt >> 1) & 1, abort_flag) ||
                     !warp_wait(&bars[kBarSFull + g], (n / G) & 1, abort_flag)) {
                     ok = false;
                     break;
