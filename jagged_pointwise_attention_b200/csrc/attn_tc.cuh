@@ -52,9 +52,9 @@
 //
 // Pointwise arithmetic per score, with h = x/2 folded into the bias adds:
 //   h = s/2 + pos/2 + time/2;  silu(x) = h + h*tanh(h)  (packed bf16x2, one
-//   MUFU op per two scores). The time bucket floor(log2(max(1, dt))) is the
-//   exponent field of dt converted exactly to double (no bit-find unit), and
-//   the bucket's bias comes from a 32-entry register table via a shuffle. The
+//   tanh.approx.bf16x2 per two scores). The time bucket floor(log2(max(1,
+//   dt))) comes from a count of leading zeros, and the bucket's bias from a
+//   32-entry register table via a shuffle. The
 //   bucket is monotone in dt, so when every row of a warp sees one bucket at
 //   the smallest and the largest key timestamp of a 32-key chunk, the bucket
 //   is constant over the chunk and the per-score bucket work is skipped.

@@ -29,20 +29,13 @@ __device__ __forceinline__ int time_bucket64(int64_t dt, int nb_minus_1) {
     return min(msb, nb_minus_1);
 }
 
-// Biased exponent of x (1 <= x < 2^32) as a double: 1023 + floor(log2(x)).
-// The double 2^52 + x is formed exactly by writing x into the low word of
-// 2^52; subtracting 2^52 leaves x exactly, so the exponent field is the bit
-// length of x minus one plus the bias. Runs on the FP64 pipe instead of the
-// shared bit-find/transcendental unit.
+// 1023 + floor(log2(x)) for 1 <= x < 2^32 (the biased exponent x would have
+// as a double), from a count of leading zeros. The time-bias register table
+// is indexed by this value modulo 32. (An earlier form built the double
+// 2^52 + x and subtracted 2^52 on the FP64 pipe; on B200 that chain sat on
+// the critical path of every 32-key chunk and cost about 9% of the kernel.)
 __device__ __forceinline__ uint32_t log2_exponent_field(uint32_t x) {
-    uint32_t hi;
-    asm("{\n\t.reg .f64 t;\n\t.reg .b32 lo;\n\t"
-        "mov.b64 t, {%1, %2};\n\t"
-        "sub.rn.f64 t, t, 0d4330000000000000;\n\t"
-        "mov.b64 {lo, %0}, t;\n\t}"
-        : "=r"(hi)
-        : "r"(x), "r"(0x43300000u));
-    return hi >> 20;
+    return 1054u - static_cast<uint32_t>(__clz(x));
 }
 
 // Same bucket for a difference already known to fit in int32.
