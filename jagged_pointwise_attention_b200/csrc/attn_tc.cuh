@@ -757,6 +757,18 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                     // no pair of the tile masked for any row of the warp (every tile
                     // but the diagonal one of an aligned unit): no per-chunk tests
                     const bool tile_full = __all_sync(0xffffffffu, lo <= 0 && hi >= 127);
+                    // one time bucket over the whole unmasked tile for every row of the
+                    // warp (most tiles away from the diagonal): no per-chunk decisions
+                    bool tile_const = tile_full && fast_w;
+                    float t_tile = 0.f;
+                    if (tile_const && use_time) {
+                        const int kmin = min(min(st.cmin[0], st.cmin[1]), min(st.cmin[2], st.cmin[3]));
+                        const int kmax = max(max(st.cmax[0], st.cmax[1]), max(st.cmax[2], st.cmax[3]));
+                        const uint32_t ef_hi = log2_exponent_field(static_cast<uint32_t>(max(tib - kmin, 1)));
+                        const uint32_t ef_lo = log2_exponent_field(static_cast<uint32_t>(max(tib - kmax, 1)));
+                        t_tile = __shfl_sync(0xffffffffu, tbr, static_cast<int>(ef_lo));
+                        tile_const = __all_sync(0xffffffffu, ef_hi == ef_lo);
+                    }
 #pragma unroll 1
                     for (int q = 0; q < 4; ++q) {
                         const int c0 = 32 * q;
@@ -787,7 +799,8 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                             int32_t thr = 0x7fffffff;
                             if (full) {
                                 path = 0;
-                                if (use_time) {
+                                tl = t_tile;
+                                if (use_time && !tile_const) {
                                     const uint32_t ef_hi = log2_exponent_field(static_cast<uint32_t>(max(tib - st.cmin[q], 1)));
                                     const uint32_t ef_lo = log2_exponent_field(static_cast<uint32_t>(max(tib - st.cmax[q], 1)));
                                     tl = __shfl_sync(0xffffffffu, tbr, static_cast<int>(ef_lo));
