@@ -109,14 +109,14 @@ struct AttnCfg {
 // 16-byte loads whose word p packs columns (c0+2p, c0+2p+1). Entry s lies in
 // 16-byte bank slot s mod 8, so the eight consecutive k0 of a quarter warp
 // never conflict.
-// Key timestamps are kept as their low 32 bits, which give exact differences
-// whenever every timestamp involved lies within 2^30 of `base` (the tile's
-// first key): ok[c] says so for the keys of chunk c, and cmin/cmax are the
-// chunk's smallest and largest key timestamp minus base.
+// Key timestamps are kept relative to `base` (the tile's first key) in 32
+// bits, exact whenever every timestamp involved lies within 2^30 of base:
+// ok[c] says so for the keys of chunk c, and cmin/cmax are the chunk's
+// smallest and largest key timestamp minus base.
 struct alignas(16) BiasStage {
     uint4 wb[248];         // sliding-window table of bf16 pos/2
     uint32_t r32[128];     // its source: word m packs R[2m], R[2m+1] (R[255] = 0)
-    int32_t kt32[128];     // low 32 bits of the key timestamps
+    int32_t kt32[128];     // key timestamps minus base (exact when ok[] holds)
     int64_t base;          // timestamp of the tile's first key
     int32_t cmin[4], cmax[4], ok[4];
     int32_t pad[2];
@@ -264,12 +264,14 @@ __device__ __forceinline__ void pw_const(const uint32_t* sv, const uint4* wbk, u
 }
 
 // Two time buckets over an unmasked chunk: scores whose time difference is
-// at least thr (a power of two) take th, the others tl; the same bits as a
-// bucket per score whenever every score's bucket is one of the two.
+// at least a power of two thr take th, the others tl; with key timestamps
+// relative to base (ktr) and the row's tib = ti - base that is
+// ktr <= kthr = tib - thr. The same bits as a bucket per score whenever every
+// score's bucket is one of the two.
 __device__ __forceinline__ void pw_two(const uint32_t* sv, int c0, const uint4* wbk,
-                                       const int32_t* __restrict__ kt32, int32_t ti32, int32_t thr,
+                                       const int32_t* __restrict__ ktr, int32_t kthr,
                                        float tl, float th, uint32_t* pk) {
-    const int4* k4 = reinterpret_cast<const int4*>(kt32 + c0);
+    const int4* k4 = reinterpret_cast<const int4*>(ktr + c0);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         const uint4 W = wbk[8 * q];
@@ -280,11 +282,7 @@ __device__ __forceinline__ void pw_two(const uint32_t* sv, int c0, const uint4* 
         for (int u = 0; u < 4; ++u) {
             float tv[2];
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int32_t dt = static_cast<int32_t>(static_cast<uint32_t>(ti32) -
-                                                        static_cast<uint32_t>(kv[2 * u + e]));
-                tv[e] = dt >= thr ? th : tl;
-            }
+            for (int e = 0; e < 2; ++e) tv[e] = kv[2 * u + e] <= kthr ? th : tl;
             const int p = 4 * q + u;
             pk[p] = silu_of_half_bf16x2(
                 half_arg_bf16x2(sv[2 * p], sv[2 * p + 1], wv[u], pack_bf16x2(tv[0], tv[1])));
@@ -292,13 +290,14 @@ __device__ __forceinline__ void pw_two(const uint32_t* sv, int c0, const uint4* 
     }
 }
 
-// Bucket per score, differences exact in 32 bits. tbr: this lane's entry of
-// the register table (lane L holds time/2 of bucket min((L+1) mod 32, NB-1)).
+// Bucket per score, differences exact in 32 bits (tib - ktr, both relative
+// to base). tbr: this lane's entry of the register table (lane L holds
+// time/2 of bucket min((L+1) mod 32, NB-1)).
 template <bool kMask>
 __device__ __forceinline__ void pw_fast(const uint32_t* sv, int c0, const uint4* wbk,
-                                        const int32_t* __restrict__ kt32, int32_t ti32, float tbr,
+                                        const int32_t* __restrict__ ktr, int32_t tib, float tbr,
                                         int lo, int hi, uint32_t* pk) {
-    const int4* k4 = reinterpret_cast<const int4*>(kt32 + c0);
+    const int4* k4 = reinterpret_cast<const int4*>(ktr + c0);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         const uint4 W = wbk[8 * q];
@@ -310,8 +309,7 @@ __device__ __forceinline__ void pw_fast(const uint32_t* sv, int c0, const uint4*
             float tv[2];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-                const int32_t dt = static_cast<int32_t>(static_cast<uint32_t>(ti32) -
-                                                        static_cast<uint32_t>(kv[2 * u + e]));
+                const int32_t dt = tib - kv[2 * u + e];
                 const uint32_t ef = log2_exponent_field(static_cast<uint32_t>(max(dt, 1)));
                 tv[e] = __shfl_sync(0xffffffffu, tbr, static_cast<int>(ef));
             }
@@ -688,8 +686,8 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                 kv = __ldg(args.ts + (key < args.T ? key : args.T - 1));
                 base = __ldg(args.ts + kt0);
             }
-            st.kt32[r] = static_cast<int32_t>(static_cast<uint64_t>(kv));
             const int64_t dk = kv - base;
+            st.kt32[r] = static_cast<int32_t>(dk);
             const bool near = dk > -(1ll << 30) && dk < (1ll << 30);
             const int dmin = __reduce_min_sync(0xffffffffu, (kvalid && near) ? static_cast<int>(dk) : INT_MAX);
             const int dmax = __reduce_max_sync(0xffffffffu, (kvalid && near) ? static_cast<int>(dk) : INT_MIN);
@@ -726,7 +724,6 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                       min((lane + 1) & 31, nbm1))
                                        : 0.f;
             const float* tbh = use_time ? args.tb + static_cast<int64_t>(I.h) * args.NB : nullptr;
-            const int32_t ti32 = static_cast<int32_t>(static_cast<uint64_t>(ti));
             for (int j = 0; j < I.nk; ++j, ++n) {
                 if (n % G != g) continue;
                 const int kt0 = I.k0 + j * kTile;
@@ -796,7 +793,7 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                             // rest take a bucket per score
                             int path = 2;
                             float tl = 0.f, th = 0.f;
-                            int32_t thr = 0x7fffffff;
+                            int32_t kthr = INT_MIN;                 // no key below it
                             if (full) {
                                 path = 0;
                                 tl = t_tile;
@@ -806,14 +803,14 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                                     tl = __shfl_sync(0xffffffffu, tbr, static_cast<int>(ef_lo));
                                     th = __shfl_sync(0xffffffffu, tbr, static_cast<int>(ef_hi));
                                     // bucket ef_hi iff dt >= 2^(ef_hi - 1023) (>= 2 when ef_hi > ef_lo)
-                                    if (ef_hi > ef_lo) thr = 1 << (ef_hi - 1023u);
+                                    if (ef_hi > ef_lo) kthr = tib - (1 << (ef_hi - 1023u));
                                     path = __all_sync(0xffffffffu, ef_hi == ef_lo) ? 0
                                            : __all_sync(0xffffffffu, ef_hi - ef_lo <= 1u) ? 1 : 2;
                                 }
                             }
                             if (path == 0) pw_const(sv, wbr + c0, pack_bf16x2(tl, tl), pk);
-                            else if (path == 1) pw_two(sv, c0, wbr + c0, st.kt32, ti32, thr, tl, th, pk);
-                            else pw_fast<true>(sv, c0, wbr + c0, st.kt32, ti32, tbr, lo, hi, pk);
+                            else if (path == 1) pw_two(sv, c0, wbr + c0, st.kt32, kthr, tl, th, pk);
+                            else pw_fast<true>(sv, c0, wbr + c0, st.kt32, tib, tbr, lo, hi, pk);
                         }
                         // 32 bf16 results -> columns 32q..32q+15 of the S buffer just read
                         tmem_st16(s_col + c0, pk);
