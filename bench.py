@@ -294,17 +294,16 @@ def bench_attention(args, rank, world, local, peaks, peak_kind):
     torch.cuda.synchronize(dev)
     kernel_ms = [a.elapsed_time(b) for a, b in kev]
 
-    # The timed steps replay one CUDA graph per input copy (plan + run), so the
-    # host's launch cost is not part of the step time.
-    graphs = []
+    # The timed steps are replayed from one CUDA graph holding all K steps
+    # (each a plan + run over its step's input copy), so neither the host's
+    # launch cost nor gaps between graph launches are part of the step time.
+    graph = None
     if not args.no_graph:
-        for i in range(ncopies):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for i in range(args.steps):
                 step(i)
-            graphs.append(g)
-        for i in range(ncopies):
-            graphs[i].replay()
+        graph.replay()
         torch.cuda.synchronize(dev)
         stream = torch.cuda.current_stream(dev)
 
@@ -314,17 +313,17 @@ def bench_attention(args, rank, world, local, peaks, peak_kind):
     torch.cuda.synchronize(dev)
     sampler.start()
     e0.record(stream)
-    for i in range(args.steps):
-        if graphs:
-            graphs[i % ncopies].replay()
-        else:
+    if graph is not None:
+        graph.replay()
+    else:
+        for i in range(args.steps):
             step(i)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     sampler.stop()
     _barrier(world)
     local_ms = e0.elapsed_time(e1)
-    del graphs
+    del graph
     st = hstu.hstu_device_status()
     if st != 0:
         raise RuntimeError("device status %d after timed steps" % st)
@@ -378,7 +377,8 @@ def bench_attention(args, rank, world, local, peaks, peak_kind):
                    "l2": ("inputs %.0f MB > L2" % (in_bytes / 2 ** 20)) if ncopies == 1 else
                          ("rotating %d input copies (%.0f MB) > 2x L2" %
                           (ncopies, ncopies * in_bytes / 2 ** 20)),
-                   "launch": "eager" if args.no_graph else "CUDA graph per step (plan + run)"},
+                   "launch": "eager" if args.no_graph else
+                             "one CUDA graph of the K steps (plan + run each)"},
         "pct_of_bf16_peak": {"measured_burst": round(100 * value / peaks["bf16_tflops"], 2),
                              "nominal_2250": round(100 * value / NOMINAL_BF16_TFLOPS, 2)},
         "tokens_per_s": round(total_tokens / (max_ms * 1e-3), 1),

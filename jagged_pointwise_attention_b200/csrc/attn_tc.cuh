@@ -387,7 +387,6 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
-    const int n_items = *args.unit_count * args.H;
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffTmem);
@@ -431,10 +430,15 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
+    // The work list comes from the plan kernel launched just before: the set-up
+    // above overlaps its tail (programmatic dependent launch); wait for it to
+    // complete, with its writes visible, before reading the list.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    const int n_items = *args.unit_count * args.H;
 
     const uint32_t sQ = smem_u32(smem + L::kOffQ);
     const uint32_t sK = smem_u32(smem + L::kOffK);

@@ -164,6 +164,28 @@ hstu_status_t validate_attn(const AttnCall& c) {
     return HSTU_OK;
 }
 
+// Launch of the attention kernel as a programmatic dependent of the kernel
+// before it in the stream (normally the plan): its set-up overlaps that
+// kernel's tail, and it waits for it (griddepcontrol.wait) before reading the
+// work list.
+template <typename Kernel>
+hstu_status_t launch_attn_pdl(Kernel kernel, unsigned grid, int threads, size_t smem,
+                              cudaStream_t stream, const CUtensorMap& tq, const CUtensorMap& tk,
+                              const CUtensorMap& tv, const AttnArgs& a) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(static_cast<unsigned>(threads));
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, tq, tk, tv, a);
+    return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
 hstu_status_t run_attn(const AttnCall& c) {
     const hstu_status_t st = validate_attn(c);
     if (st != HSTU_OK || c.B == 0 || c.T == 0) return st;
@@ -213,13 +235,13 @@ hstu_status_t run_attn(const AttnCall& c) {
     if (c.dqk == 64) {
         if (!ensure_smem(attn_fwd_bf16_kernel<64, G>, AttnSmem<64, G>::kAlloc, smem_done64))
             return HSTU_ERR_CUDA;
-        attn_fwd_bf16_kernel<64, G><<<grid, AttnCfg<64, G>::kThreads, AttnSmem<64, G>::kAlloc,
-                                      c.stream>>>(tq, tk, tv, a);
+        return launch_attn_pdl(attn_fwd_bf16_kernel<64, G>, grid, AttnCfg<64, G>::kThreads,
+                               AttnSmem<64, G>::kAlloc, c.stream, tq, tk, tv, a);
     } else {
         if (!ensure_smem(attn_fwd_bf16_kernel<128, G>, AttnSmem<128, G>::kAlloc, smem_done128))
             return HSTU_ERR_CUDA;
-        attn_fwd_bf16_kernel<128, G><<<grid, AttnCfg<128, G>::kThreads, AttnSmem<128, G>::kAlloc,
-                                       c.stream>>>(tq, tk, tv, a);
+        return launch_attn_pdl(attn_fwd_bf16_kernel<128, G>, grid, AttnCfg<128, G>::kThreads,
+                                AttnSmem<128, G>::kAlloc, c.stream, tq, tk, tv, a);
     }
     return launch_status();
 }

@@ -188,6 +188,9 @@ plan_kernel(const int64_t* __restrict__ seq_offsets, int B, int64_t T, int max_s
             int max_tiles, int max_units, int4* __restrict__ units, uint4* __restrict__ starts,
             int* __restrict__ unit_count, int* __restrict__ item_counter) {
     extern __shared__ int plan_smem[];
+    // let the attention kernel that follows start its set-up now (it waits
+    // for this grid to complete before it reads the work list)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (B < kPlanSmemOffsets)
         plan_body<true>(seq_offsets, B, T, max_seqlen, max_tiles, max_units, units, starts,
                         unit_count, item_counter, plan_smem);
