@@ -219,3 +219,40 @@ def test_bounded_wait_reports_timeout():
     assert hstu.hstu_device_status() == 0          # cleared; the context stays usable
     inp = custom_attn_inputs([33], H=1, d=64, num_pos=8, num_buckets=8, seed=13)
     assert_bf16_close(run_gpu(inp), run_oracle(inp), "after timeout")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_time_bucket_of_every_pair(d):
+    """Every pair's time bucket, read off the output: with q = k = 0 and no
+    position bias, P_ij = silu(time_bias[bucket(t_i - t_j)]) with a table whose
+    buckets differ by far more than bf16 rounding, and v is one-hot on the keys
+    of one key tile at a time, so each output element holds the P of one or
+    two pairs. The sequences are long enough for tiles that see one, two and
+    many buckets per 32-key chunk, plus packed short sequences and one with
+    timestamps too far apart for 32-bit differences."""
+    lens = [1400, 600, 90, 33, 1, 300]
+    H, NB = 2, 32
+    inp = custom_attn_inputs(lens, H=H, d=d, num_pos=8, num_buckets=NB, seed=21)
+    off = inp.seq_offsets
+    last = slice(int(off[-2]), int(off[-1]))
+    inp.timestamps[last] = np.cumsum(np.full(lens[-1], 1 << 26, np.int64)) + (1 << 40)
+    inp.q[:] = 0
+    inp.k[:] = 0
+    inp.pos_bias[:] = 0
+    b = np.arange(NB, dtype=np.float32)
+    inp.time_bias[0] = 1.0 + 0.75 * b
+    inp.time_bias[1] = 2.0 + 0.5 * b
+    T = inp.T
+    pos_in_seq = np.arange(T) - np.repeat(off[:-1], np.diff(off))
+    for kt in range((max(lens) + 127) // 128):
+        v = np.zeros((T, H, d), np.float32)
+        sel = (pos_in_seq >= 128 * kt) & (pos_in_seq < 128 * kt + 128)
+        v[np.nonzero(sel)[0], :, (pos_in_seq[sel] - 128 * kt) % d] = 1.0
+        inp.v = v
+        got = run_gpu(inp, v=dev(v, torch.bfloat16))
+        want = run_oracle(inp)
+        err = np.abs(got - want)
+        bound = 0.015 * np.abs(want) + 1e-6
+        bad = np.argwhere(err > bound)
+        assert bad.size == 0, "key tile %d: %d outputs off, first (token, head, col) %s: %g vs %g" % (
+            kt, len(bad), bad[0].tolist(), got[tuple(bad[0])], want[tuple(bad[0])])
