@@ -209,10 +209,6 @@ __device__ __forceinline__ Item read_item(const volatile int* slot) {
     return it;
 }
 
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
-    const bool ok = mbar_wait(bar, parity, abort);
-    return __all_sync(0xffffffffu, ok);
-}
 
 // Per-chunk pointwise paths. sv: 32 fp32 scores of columns c0..c0+31 of this
 // thread's row; wbk: this row's entry k0 of the pos/2 window table (entries

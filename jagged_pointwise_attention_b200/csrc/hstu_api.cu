@@ -265,6 +265,15 @@ hstu_status_t plan_attn(const int64_t* off, int32_t B, int64_t T, int32_t max_se
     return launch_status();
 }
 
+template <int EPI, int BN>
+hstu_status_t launch_gemm(unsigned grid, cudaStream_t stream, const CUtensorMap& ta,
+                          const CUtensorMap& tb, const GemmArgs& g) {
+    static int done[kMaxDevices] = {0};
+    if (!ensure_smem(gemm_bf16_kernel<EPI, BN>, GemmSmem<BN>::kAlloc, done)) return HSTU_ERR_CUDA;
+    gemm_bf16_kernel<EPI, BN><<<grid, kGemmThreads, GemmSmem<BN>::kAlloc, stream>>>(ta, tb, g);
+    return launch_status();
+}
+
 hstu_status_t run_linear(const void* x, int64_t ldx, int64_t M, int32_t K, const void* W,
                          int64_t ldw, int32_t N, const float* bias, hstu_epilogue_t epi,
                          const void* residual, int64_t ldr, void* y, int64_t ldy,
@@ -280,28 +289,29 @@ hstu_status_t run_linear(const void* x, int64_t ldx, int64_t M, int32_t K, const
     if (!aligned16(x) || !aligned16(W) || !aligned16(y)) return HSTU_ERR_INVALID_ARG;
     if (epi == HSTU_EPI_RESIDUAL && (!residual || ldr < N || ldr % 8 || !aligned16(residual)))
         return HSTU_ERR_INVALID_ARG;
+    // 128 x 256 output tiles when N allows (fewer operand bytes per FLOP),
+    // else 128 x 128
+    const int bn = N % 256 == 0 ? 256 : 128;
     CUtensorMap ta, tb;
-    if (!make_tmap_bf16(&ta, x, K, M, ldx * 2, 128) || !make_tmap_bf16(&tb, W, K, N, ldw * 2, 128))
+    if (!make_tmap_bf16(&ta, x, K, M, ldx * 2, 128) ||
+        !make_tmap_bf16(&tb, W, K, N, ldw * 2, static_cast<uint32_t>(bn)))
         return HSTU_ERR_CUDA;
     GemmArgs g{M, N, K, bias, static_cast<const __nv_bfloat16*>(residual), ldr,
                static_cast<__nv_bfloat16*>(y), ldy};
-    const dim3 grid(static_cast<unsigned>((M + 127) / 128), static_cast<unsigned>(N / 128));
-    static int done0[kMaxDevices] = {0}, done1[kMaxDevices] = {0}, done2[kMaxDevices] = {0};
-    switch (epi) {
-        case HSTU_EPI_NONE:
-            if (!ensure_smem(gemm_bf16_kernel<0>, GemmSmem::kAlloc, done0)) return HSTU_ERR_CUDA;
-            gemm_bf16_kernel<0><<<grid, kGemmThreads, GemmSmem::kAlloc, stream>>>(ta, tb, g);
-            break;
-        case HSTU_EPI_SILU:
-            if (!ensure_smem(gemm_bf16_kernel<1>, GemmSmem::kAlloc, done1)) return HSTU_ERR_CUDA;
-            gemm_bf16_kernel<1><<<grid, kGemmThreads, GemmSmem::kAlloc, stream>>>(ta, tb, g);
-            break;
-        default:
-            if (!ensure_smem(gemm_bf16_kernel<2>, GemmSmem::kAlloc, done2)) return HSTU_ERR_CUDA;
-            gemm_bf16_kernel<2><<<grid, kGemmThreads, GemmSmem::kAlloc, stream>>>(ta, tb, g);
-            break;
+    const int64_t tiles = (M + 127) / 128 * (N / bn);
+    const unsigned grid = static_cast<unsigned>(tiles < num_sms() ? tiles : num_sms());
+    if (bn == 256) {
+        switch (epi) {
+            case HSTU_EPI_NONE: return launch_gemm<0, 256>(grid, stream, ta, tb, g);
+            case HSTU_EPI_SILU: return launch_gemm<1, 256>(grid, stream, ta, tb, g);
+            default: return launch_gemm<2, 256>(grid, stream, ta, tb, g);
+        }
     }
-    return launch_status();
+    switch (epi) {
+        case HSTU_EPI_NONE: return launch_gemm<0, 128>(grid, stream, ta, tb, g);
+        case HSTU_EPI_SILU: return launch_gemm<1, 128>(grid, stream, ta, tb, g);
+        default: return launch_gemm<2, 128>(grid, stream, ta, tb, g);
+    }
 }
 
 hstu_status_t run_ln_gate(const void* a, int64_t lda, const void* u, int64_t ldu, int64_t M,

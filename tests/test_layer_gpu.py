@@ -46,6 +46,25 @@ def test_linear_projection_shapes():
                       "f1 shape")
 
 
+@pytest.mark.parametrize("N,epi", [(2048, "silu"), (512, "residual"), (384, "none")])
+def test_linear_persistent_tiles(N, epi):
+    """More output tiles than two per SM, so every CTA reuses both TMEM
+    accumulators and several k-block rings; ragged last row block."""
+    rng = np.random.default_rng(3)
+    M, K = 41000 if N != 2048 else 5300, 512
+    x = round_to_bf16(rng.standard_normal((M, K)).astype(np.float32))
+    W = round_to_bf16((rng.standard_normal((N, K)) / np.sqrt(K)).astype(np.float32))
+    b = (0.1 * rng.standard_normal(N)).astype(np.float32)
+    r = round_to_bf16(rng.standard_normal((M, N)).astype(np.float32)) if epi == "residual" else None
+    got = hstu.hstu_linear_fwd(bf(x), bf(W), dev(b), epi,
+                               residual=None if r is None else bf(r))
+    assert hstu.hstu_device_status() == 0
+    rows = np.concatenate([np.arange(0, M, 97), np.arange(M - 130, M)])
+    want = oracle.linear(x[rows], W, b, act_silu=epi == "silu",
+                         residual=None if r is None else r[rows])
+    assert_bf16_close(got.float().cpu().numpy()[rows], want, f"{epi} N={N}")
+
+
 def test_layernorm_gate():
     rng = np.random.default_rng(2)
     M, F = 517, 512
