@@ -649,6 +649,14 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
         // timestamp summary of chunk qd, whose keys are this warp's lanes).
         auto stage_tile = [&](const Item& I, int kt0, BiasStage& st, uint64_t* full, uint64_t* src,
                               uint32_t src_parity) -> bool {
+            // every global load first, so that their latencies overlap
+            const int64_t key = static_cast<int64_t>(kt0) + r;
+            const bool kvalid = key < I.q_end;
+            int64_t kv = 0, base = 0;
+            if (use_time) {
+                kv = __ldg(args.ts + (key < args.T ? key : args.T - 1));
+                base = __ldg(args.ts + kt0);
+            }
             {
                 // word r = (R[2r], R[2r+1]), R[k] = pos[h][clamp(i - j)] / 2 with
                 // i - j = q0 - kt0 + 127 - k, and R[255] = 0
@@ -678,13 +686,6 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                     st.wb[se] = make_uint4(__byte_perm(x[0], x[1], sel), __byte_perm(x[1], x[2], sel),
                                            __byte_perm(x[2], x[3], sel), __byte_perm(x[3], x[4], sel));
                 }
-            }
-            const int64_t key = static_cast<int64_t>(kt0) + r;
-            const bool kvalid = key < I.q_end;
-            int64_t kv = 0, base = 0;
-            if (use_time) {
-                kv = __ldg(args.ts + (key < args.T ? key : args.T - 1));
-                base = __ldg(args.ts + kt0);
             }
             const int64_t dk = kv - base;
             st.kt32[r] = static_cast<int32_t>(dk);
@@ -776,7 +777,7 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                         if (!live) {                        // every pair of the chunk is masked
 #pragma unroll
                             for (int e = 0; e < 16; ++e) pk[e] = 0u;
-                            tmem_st16(s_col + c0, pk);
+                            tmem_st16_async(s_col + c0, pk);
                             continue;
                         }
                         uint32_t sv[32];
@@ -813,9 +814,10 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                             else pw_fast<true>(sv, c0, wbr + c0, st.kt32, tib, tbr, lo, hi, pk);
                         }
                         // 32 bf16 results -> columns 32q..32q+15 of the S buffer just read
-                        tmem_st16(s_col + c0, pk);
+                        tmem_st16_async(s_col + c0, pk);
                     }
                 }
+                tmem_wait_st();     // every P store of the tile has landed
                 tc_fence_before();
                 mbar_arrive(&bars[kBarPFull + g]);
                 if (j == I.nk - 1) {
