@@ -8,7 +8,10 @@
 // ring; the fp32 accumulator of a tile lives in TMEM, two buffers of BN
 // columns, so the epilogue of one tile overlaps the main loop of the next.
 // Warp roles: 0-7 epilogue (two per TMEM lane quarter, one row per thread,
-// BN/2 columns each), 8 TMA producer, 9 MMA issuer and TMEM owner.
+// BN/2 columns each), 8 TMA producer, 9 MMA issuer and TMEM owner. The
+// epilogue writes each 32 x 32 block of results into shared memory (64-byte
+// swizzle, conflict-free) and one lane stores it with a TMA bulk store, two
+// staging buffers per warp; the store clips rows past M.
 #pragma once
 
 #include "common.cuh"
@@ -36,7 +39,8 @@ struct GemmSmem {
     static constexpr int kStageBytes = 16384 + kBBytes;
     static constexpr int kOffA = 0;                                   // [stage] 16 KB
     static constexpr int kOffB = kOffA + kGemmStages * 16384;         // [stage] BN x 128 B
-    static constexpr int kOffBar = kOffB + kGemmStages * kBBytes;
+    static constexpr int kOffOut = kOffB + kGemmStages * kBBytes;     // [warp][2] 32 x 64 B
+    static constexpr int kOffBar = kOffOut + kGemmEpiWarps * 2 * 2048;
     static constexpr int kOffTmem = kOffBar + 16 * 8;
     static constexpr int kOffAbort = kOffTmem + 8;
     static constexpr int kBytes = kOffAbort + 8;
@@ -47,7 +51,7 @@ struct GemmSmem {
 template <int EPI, int BN>   // EPI: hstu_epilogue_t (0 none, 1 silu, 2 residual)
 __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 const GemmArgs g) {
+                 const __grid_constant__ CUtensorMap tmY, const GemmArgs g) {
     using L = GemmSmem<BN>;
     constexpr int S = kGemmStages;
     constexpr int kWarpTMA = kGemmEpiWarps, kWarpMMA = kGemmEpiWarps + 1;
@@ -157,6 +161,9 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3, h = warp >> 2;          // lane quarter, column half
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+        uint8_t* stage_out = smem + L::kOffOut + warp * 2 * 2048;
+        if (lane == 0) tma_prefetch_desc(&tmY);
+        int nst = 0;                                    // blocks this warp has stored
         int tl = 0;
         for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tl) {
             const int buf = tl & 1;
@@ -165,13 +172,17 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             tc_fence_after();
             const int64_t row = static_cast<int64_t>(m0) + q * 32 + lane;
 #pragma unroll 1
-            for (int ch = 0; ch < BN / 64; ++ch) {
+            for (int ch = 0; ch < BN / 64; ++ch, ++nst) {
                 const int c = h * (BN / 2) + ch * 32;   // column within the tile
+                const int col0 = n0 + c;
                 uint32_t v[32];
                 __syncwarp();
                 tmem_ld32(tmem + lane_base + static_cast<uint32_t>(buf * BN + c), v);
-                if (row < g.M) {
-                    const int col0 = n0 + c;
+                // the store that last read this staging buffer is done with it
+                if (lane == 0) bulk_wait_group_read<1>();
+                __syncwarp();
+                uint8_t* sb = stage_out + (nst & 1) * 2048;
+                {
                     float f[32];
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
@@ -179,7 +190,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                         if (g.bias) f[e] += __ldg(g.bias + col0 + e);
                         if (EPI == 1) f[e] = silu_tanh(f[e]);
                     }
-                    if (EPI == 2) {
+                    if (EPI == 2 && row < g.M) {
                         const uint4* rp =
                             reinterpret_cast<const uint4*>(g.residual + row * g.ldr + col0);
 #pragma unroll
@@ -193,18 +204,27 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                             }
                         }
                     }
-                    uint4* dst = reinterpret_cast<uint4*>(g.y + row * g.ldy + col0);
+                    // row `lane` of the block: 16-byte unit qq at qq ^ ((lane >> 1) & 3)
 #pragma unroll
                     for (int qq = 0; qq < 4; ++qq)
-                        dst[qq] = make_uint4(pack_bf16x2(f[8 * qq], f[8 * qq + 1]),
-                                             pack_bf16x2(f[8 * qq + 2], f[8 * qq + 3]),
-                                             pack_bf16x2(f[8 * qq + 4], f[8 * qq + 5]),
-                                             pack_bf16x2(f[8 * qq + 6], f[8 * qq + 7]));
+                        *reinterpret_cast<uint4*>(sb + lane * 64 + ((qq ^ ((lane >> 1) & 3)) << 4)) =
+                            make_uint4(pack_bf16x2(f[8 * qq], f[8 * qq + 1]),
+                                       pack_bf16x2(f[8 * qq + 2], f[8 * qq + 3]),
+                                       pack_bf16x2(f[8 * qq + 4], f[8 * qq + 5]),
+                                       pack_bf16x2(f[8 * qq + 6], f[8 * qq + 7]));
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmY, sb, col0, m0 + q * 32);
+                    bulk_commit_group();
                 }
             }
             tc_fence_before();
             mbar_arrive(&acc_empty[buf]);
         }
+        if (lane == 0) bulk_wait_group_all();
+        __syncwarp();
     }
     tc_fence_before();
     __syncthreads();

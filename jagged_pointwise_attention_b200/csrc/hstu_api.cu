@@ -48,19 +48,26 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // 2-D bf16 tensor map over a row-major [rows, inner] view with the given row
 // stride (bytes); 64 x 128 boxes with the 128-byte swizzle the UMMA
 // descriptors expect.
-bool make_tmap_bf16(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t rows,
-                    uint64_t row_stride_bytes, uint32_t box_rows) {
+bool make_tmap_bf16_box(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t rows,
+                        uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows,
+                        CUtensorMapSwizzle swizzle) {
     auto fn = encode_fn();
     if (fn == nullptr) return false;
     cuuint64_t dims[2] = {inner, rows};
     cuuint64_t strides[1] = {row_stride_bytes};
-    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t box[2] = {box_inner, box_rows};
     cuuint32_t estr[2] = {1, 1};
     const CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
-                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+// Boxes of 64 columns (128 bytes, 128-byte swizzle) x box_rows: MMA operands.
+bool make_tmap_bf16(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t rows,
+                    uint64_t row_stride_bytes, uint32_t box_rows) {
+    return make_tmap_bf16_box(tm, base, inner, rows, row_stride_bytes, 64, box_rows,
+                              CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // Raise a kernel's dynamic shared-memory limit once per device.
@@ -267,10 +274,10 @@ hstu_status_t plan_attn(const int64_t* off, int32_t B, int64_t T, int32_t max_se
 
 template <int EPI, int BN>
 hstu_status_t launch_gemm(unsigned grid, cudaStream_t stream, const CUtensorMap& ta,
-                          const CUtensorMap& tb, const GemmArgs& g) {
+                          const CUtensorMap& tb, const CUtensorMap& ty, const GemmArgs& g) {
     static int done[kMaxDevices] = {0};
     if (!ensure_smem(gemm_bf16_kernel<EPI, BN>, GemmSmem<BN>::kAlloc, done)) return HSTU_ERR_CUDA;
-    gemm_bf16_kernel<EPI, BN><<<grid, kGemmThreads, GemmSmem<BN>::kAlloc, stream>>>(ta, tb, g);
+    gemm_bf16_kernel<EPI, BN><<<grid, kGemmThreads, GemmSmem<BN>::kAlloc, stream>>>(ta, tb, ty, g);
     return launch_status();
 }
 
@@ -292,9 +299,11 @@ hstu_status_t run_linear(const void* x, int64_t ldx, int64_t M, int32_t K, const
     // 128 x 256 output tiles when N allows (fewer operand bytes per FLOP),
     // else 128 x 128
     const int bn = N % 256 == 0 ? 256 : 128;
-    CUtensorMap ta, tb;
+    // output in 32 x 32 blocks (64-byte rows, 64-byte swizzle)
+    CUtensorMap ta, tb, ty;
     if (!make_tmap_bf16(&ta, x, K, M, ldx * 2, 128) ||
-        !make_tmap_bf16(&tb, W, K, N, ldw * 2, static_cast<uint32_t>(bn)))
+        !make_tmap_bf16(&tb, W, K, N, ldw * 2, static_cast<uint32_t>(bn)) ||
+        !make_tmap_bf16_box(&ty, y, N, M, ldy * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
         return HSTU_ERR_CUDA;
     GemmArgs g{M, N, K, bias, static_cast<const __nv_bfloat16*>(residual), ldr,
                static_cast<__nv_bfloat16*>(y), ldy};
@@ -302,15 +311,15 @@ hstu_status_t run_linear(const void* x, int64_t ldx, int64_t M, int32_t K, const
     const unsigned grid = static_cast<unsigned>(tiles < num_sms() ? tiles : num_sms());
     if (bn == 256) {
         switch (epi) {
-            case HSTU_EPI_NONE: return launch_gemm<0, 256>(grid, stream, ta, tb, g);
-            case HSTU_EPI_SILU: return launch_gemm<1, 256>(grid, stream, ta, tb, g);
-            default: return launch_gemm<2, 256>(grid, stream, ta, tb, g);
+            case HSTU_EPI_NONE: return launch_gemm<0, 256>(grid, stream, ta, tb, ty, g);
+            case HSTU_EPI_SILU: return launch_gemm<1, 256>(grid, stream, ta, tb, ty, g);
+            default: return launch_gemm<2, 256>(grid, stream, ta, tb, ty, g);
         }
     }
     switch (epi) {
-        case HSTU_EPI_NONE: return launch_gemm<0, 128>(grid, stream, ta, tb, g);
-        case HSTU_EPI_SILU: return launch_gemm<1, 128>(grid, stream, ta, tb, g);
-        default: return launch_gemm<2, 128>(grid, stream, ta, tb, g);
+        case HSTU_EPI_NONE: return launch_gemm<0, 128>(grid, stream, ta, tb, ty, g);
+        case HSTU_EPI_SILU: return launch_gemm<1, 128>(grid, stream, ta, tb, ty, g);
+        default: return launch_gemm<2, 128>(grid, stream, ta, tb, ty, g);
     }
 }
 
