@@ -11,7 +11,9 @@
 // BN/2 columns each), 8 TMA producer, 9 MMA issuer and TMEM owner. The
 // epilogue writes each 32 x 32 block of results into shared memory (64-byte
 // swizzle, conflict-free) and one lane stores it with a TMA bulk store, two
-// staging buffers per warp; the store clips rows past M.
+// staging buffers per warp; the store clips rows past M. With the residual
+// epilogue the block's residual is first loaded into the same buffer by TMA,
+// one block ahead.
 #pragma once
 
 #include "common.cuh"
@@ -41,7 +43,7 @@ struct GemmSmem {
     static constexpr int kOffB = kOffA + kGemmStages * 16384;         // [stage] BN x 128 B
     static constexpr int kOffOut = kOffB + kGemmStages * kBBytes;     // [warp][2] 32 x 64 B
     static constexpr int kOffBar = kOffOut + kGemmEpiWarps * 2 * 2048;
-    static constexpr int kOffTmem = kOffBar + 16 * 8;
+    static constexpr int kOffTmem = kOffBar + 32 * 8;
     static constexpr int kOffAbort = kOffTmem + 8;
     static constexpr int kBytes = kOffAbort + 8;
     static constexpr int kAlloc = kBytes + 1024;
@@ -51,7 +53,8 @@ struct GemmSmem {
 template <int EPI, int BN>   // EPI: hstu_epilogue_t (0 none, 1 silu, 2 residual)
 __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 const __grid_constant__ CUtensorMap tmY, const GemmArgs g) {
+                 const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmR,
+                 const GemmArgs g) {
     using L = GemmSmem<BN>;
     constexpr int S = kGemmStages;
     constexpr int kWarpTMA = kGemmEpiWarps, kWarpMMA = kGemmEpiWarps + 1;
@@ -69,6 +72,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     uint64_t* acc_full = empty + S;      // [2]
     uint64_t* acc_empty = acc_full + 2;  // [2]
     uint64_t* drain = acc_empty + 2;
+    uint64_t* res_full = drain + 1;      // [epilogue warp][2]: residual block landed
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffTmem);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffAbort);
 
@@ -83,6 +87,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             mbar_init(&acc_empty[b], 32 * kGemmEpiWarps);
         }
         mbar_init(drain, 1);
+        for (int b = 0; b < 2 * kGemmEpiWarps; ++b) mbar_init(&res_full[b], 1);
         mbar_fence_init();
     }
     if (warp == kWarpMMA) {
@@ -162,10 +167,26 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         const int q = warp & 3, h = warp >> 2;          // lane quarter, column half
         const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
         uint8_t* stage_out = smem + L::kOffOut + warp * 2 * 2048;
-        if (lane == 0) tma_prefetch_desc(&tmY);
+        uint64_t* rbar = res_full + 2 * warp;
+        constexpr int kBlocks = BN / 64;                // 32-column blocks per warp and tile
+        // residual block ch of tile t into staging buffer b (lane 0)
+        auto load_res = [&](int t, int ch, int b) {
+            mbar_arrive_expect_tx(&rbar[b], 2048);
+            tma_load_2d(stage_out + b * 2048, &tmR, &rbar[b],
+                        (t % tiles_n) * BN + h * (BN / 2) + ch * 32, (t / tiles_n) * 128 + q * 32);
+        };
+        if (lane == 0) {
+            tma_prefetch_desc(&tmY);
+            if (EPI == 2) {
+                tma_prefetch_desc(&tmR);
+                if (static_cast<int>(blockIdx.x) < tiles) load_res(blockIdx.x, 0, 0);
+            }
+        }
         int nst = 0;                                    // blocks this warp has stored
+        int nres = EPI == 2 && static_cast<int>(blockIdx.x) < tiles ? 1 : 0;  // residual loads issued
+        bool eok = true;
         int tl = 0;
-        for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tl) {
+        for (int t = blockIdx.x; eok && t < tiles; t += gridDim.x, ++tl) {
             const int buf = tl & 1;
             const int m0 = (t / tiles_n) * 128, n0 = (t % tiles_n) * BN;
             if (!warp_wait(&acc_full[buf], (tl >> 1) & 1, abort_flag)) break;
@@ -178,10 +199,18 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 uint32_t v[32];
                 __syncwarp();
                 tmem_ld32(tmem + lane_base + static_cast<uint32_t>(buf * BN + c), v);
-                // the store that last read this staging buffer is done with it
-                if (lane == 0) bulk_wait_group_read<1>();
-                __syncwarp();
                 uint8_t* sb = stage_out + (nst & 1) * 2048;
+                if (EPI == 2) {
+                    // this block's residual (loaded one block ahead)
+                    if (!warp_wait(&rbar[nst & 1], (nst >> 1) & 1, abort_flag)) {
+                        eok = false;
+                        break;
+                    }
+                } else {
+                    // the store that last read this staging buffer is done with it
+                    if (lane == 0) bulk_wait_group_read<1>();
+                    __syncwarp();
+                }
                 {
                     float f[32];
 #pragma unroll
@@ -190,12 +219,11 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                         if (g.bias) f[e] += __ldg(g.bias + col0 + e);
                         if (EPI == 1) f[e] = silu_tanh(f[e]);
                     }
-                    if (EPI == 2 && row < g.M) {
-                        const uint4* rp =
-                            reinterpret_cast<const uint4*>(g.residual + row * g.ldr + col0);
+                    if (EPI == 2) {
 #pragma unroll
                         for (int qq = 0; qq < 4; ++qq) {
-                            const uint4 w = rp[qq];
+                            const uint4 w = *reinterpret_cast<const uint4*>(
+                                sb + lane * 64 + ((qq ^ ((lane >> 1) & 3)) << 4));
                             const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                             for (int u = 0; u < 4; ++u) {
@@ -218,12 +246,28 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 if (lane == 0) {
                     tma_store_2d(&tmY, sb, col0, m0 + q * 32);
                     bulk_commit_group();
+                    if (EPI == 2) {
+                        // the next block's residual into the other buffer, once the
+                        // store that last read it is done
+                        const int nt = ch + 1 < kBlocks ? t : t + static_cast<int>(gridDim.x);
+                        if (nt < tiles) {
+                            bulk_wait_group_read<1>();
+                            load_res(nt, ch + 1 < kBlocks ? ch + 1 : 0, (nst + 1) & 1);
+                            ++nres;
+                        }
+                    }
                 }
             }
+            if (!eok) break;
             tc_fence_before();
             mbar_arrive(&acc_empty[buf]);
         }
-        if (lane == 0) bulk_wait_group_all();
+        if (lane == 0) {
+            bulk_wait_group_all();
+            // a residual load issued for a block never reached (an early exit)
+            if (nres > nst && !mbar_wait(&rbar[nst & 1], (nst >> 1) & 1, nullptr))
+                raise_error(kErrTimeout);
+        }
         __syncwarp();
     }
     tc_fence_before();

@@ -274,10 +274,12 @@ hstu_status_t plan_attn(const int64_t* off, int32_t B, int64_t T, int32_t max_se
 
 template <int EPI, int BN>
 hstu_status_t launch_gemm(unsigned grid, cudaStream_t stream, const CUtensorMap& ta,
-                          const CUtensorMap& tb, const CUtensorMap& ty, const GemmArgs& g) {
+                          const CUtensorMap& tb, const CUtensorMap& ty, const CUtensorMap& tr,
+                          const GemmArgs& g) {
     static int done[kMaxDevices] = {0};
     if (!ensure_smem(gemm_bf16_kernel<EPI, BN>, GemmSmem<BN>::kAlloc, done)) return HSTU_ERR_CUDA;
-    gemm_bf16_kernel<EPI, BN><<<grid, kGemmThreads, GemmSmem<BN>::kAlloc, stream>>>(ta, tb, ty, g);
+    gemm_bf16_kernel<EPI, BN>
+        <<<grid, kGemmThreads, GemmSmem<BN>::kAlloc, stream>>>(ta, tb, ty, tr, g);
     return launch_status();
 }
 
@@ -299,27 +301,33 @@ hstu_status_t run_linear(const void* x, int64_t ldx, int64_t M, int32_t K, const
     // 128 x 256 output tiles when N allows (fewer operand bytes per FLOP),
     // else 128 x 128
     const int bn = N % 256 == 0 ? 256 : 128;
-    // output in 32 x 32 blocks (64-byte rows, 64-byte swizzle)
-    CUtensorMap ta, tb, ty;
+    // output and residual in 32 x 32 blocks (64-byte rows, 64-byte swizzle)
+    CUtensorMap ta, tb, ty, tr;
     if (!make_tmap_bf16(&ta, x, K, M, ldx * 2, 128) ||
         !make_tmap_bf16(&tb, W, K, N, ldw * 2, static_cast<uint32_t>(bn)) ||
         !make_tmap_bf16_box(&ty, y, N, M, ldy * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
         return HSTU_ERR_CUDA;
+    if (epi == HSTU_EPI_RESIDUAL) {
+        if (!make_tmap_bf16_box(&tr, residual, N, M, ldr * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+            return HSTU_ERR_CUDA;
+    } else {
+        tr = ty;    // not read
+    }
     GemmArgs g{M, N, K, bias, static_cast<const __nv_bfloat16*>(residual), ldr,
                static_cast<__nv_bfloat16*>(y), ldy};
     const int64_t tiles = (M + 127) / 128 * (N / bn);
     const unsigned grid = static_cast<unsigned>(tiles < num_sms() ? tiles : num_sms());
     if (bn == 256) {
         switch (epi) {
-            case HSTU_EPI_NONE: return launch_gemm<0, 256>(grid, stream, ta, tb, ty, g);
-            case HSTU_EPI_SILU: return launch_gemm<1, 256>(grid, stream, ta, tb, ty, g);
-            default: return launch_gemm<2, 256>(grid, stream, ta, tb, ty, g);
+            case HSTU_EPI_NONE: return launch_gemm<0, 256>(grid, stream, ta, tb, ty, tr, g);
+            case HSTU_EPI_SILU: return launch_gemm<1, 256>(grid, stream, ta, tb, ty, tr, g);
+            default: return launch_gemm<2, 256>(grid, stream, ta, tb, ty, tr, g);
         }
     }
     switch (epi) {
-        case HSTU_EPI_NONE: return launch_gemm<0, 128>(grid, stream, ta, tb, ty, g);
-        case HSTU_EPI_SILU: return launch_gemm<1, 128>(grid, stream, ta, tb, ty, g);
-        default: return launch_gemm<2, 128>(grid, stream, ta, tb, ty, g);
+        case HSTU_EPI_NONE: return launch_gemm<0, 128>(grid, stream, ta, tb, ty, tr, g);
+        case HSTU_EPI_SILU: return launch_gemm<1, 128>(grid, stream, ta, tb, ty, tr, g);
+        default: return launch_gemm<2, 128>(grid, stream, ta, tb, ty, tr, g);
     }
 }
 
