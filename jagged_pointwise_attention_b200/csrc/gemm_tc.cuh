@@ -191,7 +191,6 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             const int m0 = (t / tiles_n) * 128, n0 = (t % tiles_n) * BN;
             if (!warp_wait(&acc_full[buf], (tl >> 1) & 1, abort_flag)) break;
             tc_fence_after();
-            const int64_t row = static_cast<int64_t>(m0) + q * 32 + lane;
 #pragma unroll 1
             for (int ch = 0; ch < BN / 64; ++ch, ++nst) {
                 const int c = h * (BN / 2) + ch * 32;   // column within the tile
