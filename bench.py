@@ -264,7 +264,8 @@ def bench_attention(args, rank, world, local, peaks, peak_kind):
     ts = to_dev(inp.timestamps)
     pos = to_dev(inp.pos_bias)
     tb = to_dev(inp.time_bias)
-    ws = torch.empty(max(16, hstu.hstu_attn_workspace_bytes(inp.B, inp.T, inp.max_seqlen)),
+    ws = torch.empty(max(16, hstu.hstu_attn_workspace_bytes(inp.B, inp.T, inp.max_seqlen, inp.H,
+                                                                inp.pos_bias.shape[1])),
                      dtype=torch.uint8, device=dev)
 
     def step(i, ev=None):
@@ -277,7 +278,7 @@ def bench_attention(args, rank, world, local, peaks, peak_kind):
         if ev is not None:
             ev[1].record(stream)
 
-    launches_per_step = 2 if bf == torch.bfloat16 else 1
+    launches_per_step = 3 if bf == torch.bfloat16 else 1   # plan, bias tables, attention
     for i in range(args.warmup):
         step(i)
     st = hstu.hstu_device_status()
@@ -413,7 +414,8 @@ def e2e_attention(args, inp, dev, stream, flops, world):
     devb = [{k: torch.empty_like(v, device=dev) for k, v in host.items()} for _ in range(2)]
     out_dev = [torch.empty(shape, dtype=bf, device=dev) for _ in range(2)]
     out_host = [torch.empty(shape, dtype=bf).pin_memory() for _ in range(2)]
-    ws = torch.empty(max(16, hstu.hstu_attn_workspace_bytes(inp.B, inp.T, inp.max_seqlen)),
+    ws = torch.empty(max(16, hstu.hstu_attn_workspace_bytes(inp.B, inp.T, inp.max_seqlen, inp.H,
+                                                                inp.pos_bias.shape[1])),
                      dtype=torch.uint8, device=dev)
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = out_host[0].numel() * out_host[0].element_size()

@@ -76,13 +76,22 @@ hstu_status_t hstu_device_status(void* stream);
 
 /* ---------------------------------------------------------------- attention */
 
-/* Workspace bytes that hstu_attn_plan / hstu_attn_fwd need for a batch of B
- * sequences, total_tokens tokens and the given max_seqlen (bf16 path; the
- * fp32 path needs none): a 256-byte header and 32 bytes per work unit (its
- * descriptor and the sequence-start mask of a packed tile; at most
- * min(total_tokens/128 + B + 1, B * ceil(max_seqlen/128)) units, each array
- * rounded up to 256 bytes). Returns 0 for invalid sizes. */
-size_t hstu_attn_workspace_bytes(int32_t B, int64_t total_tokens, int32_t max_seqlen);
+/* Workspace bytes that hstu_attn_plan + hstu_attn_run (or hstu_attn_fwd)
+ * need for a batch of B sequences, total_tokens tokens, the given
+ * max_seqlen, H heads and a position table of num_pos entries per head
+ * (pass the same num_pos as the run, or 1 when it has no position term; bf16
+ * path, the fp32 path needs none). Layout:
+ *  - the plan's part: a 256-byte header and 32 bytes per work unit (its
+ *    descriptor and the sequence-start mask of a packed tile; at most
+ *    U = min(total_tokens/128 + B + 1, B * ceil(max_seqlen/128)) units, each
+ *    array rounded up to 256 bytes);
+ *  - the run's bias tables: 3968 bytes per head and distinct 128-token
+ *    diagonal offset of the position window (min(ceil(max_seqlen/128),
+ *    ceil((num_pos + 126)/128) + 1) offsets), and 576 bytes per unit for the
+ *    key-timestamp summary of its tile.
+ * hstu_attn_plan needs only the plan's part. Returns 0 for invalid sizes. */
+size_t hstu_attn_workspace_bytes(int32_t B, int64_t total_tokens, int32_t max_seqlen, int32_t H,
+                                 int32_t num_pos);
 
 /* Builds the work list of the bf16 attention in `workspace` (device):
  * one entry per (sequence, 128-query tile), ordered longest-first (a query
@@ -106,6 +115,10 @@ hstu_status_t hstu_attn_plan(const int64_t* seq_offsets, int32_t B, int64_t tota
  *   max_seqlen : N of the 1/N scale
  *   out  : device [T, H, d_v] of `dtype`, token stride out_tok_stride; every row
  *          of every sequence is written, nothing else is touched
+ *   workspace : the plan's workspace, hstu_attn_workspace_bytes(B, total_tokens,
+ *          max_seqlen, H, num_pos or 1) bytes; the run reads the plan's part
+ *          and rewrites the bias tables behind it (two launches: the tables,
+ *          then the attention)
  * Supported: bf16 with d_qk == d_v in {64, 128}; fp32 with d_qk, d_v <= 128. */
 hstu_status_t hstu_attn_run(hstu_dtype_t dtype,
                             const void* q, int64_t q_tok_stride,
@@ -118,9 +131,9 @@ hstu_status_t hstu_attn_run(hstu_dtype_t dtype,
                             const float* time_bias, int32_t num_time_buckets,
                             int32_t max_seqlen,
                             void* out, int64_t out_tok_stride,
-                            const void* workspace, size_t workspace_bytes, void* stream);
+                            void* workspace, size_t workspace_bytes, void* stream);
 
-/* hstu_attn_plan followed by hstu_attn_run (two launches for bf16, one for fp32). */
+/* hstu_attn_plan followed by hstu_attn_run (three launches for bf16, one for fp32). */
 hstu_status_t hstu_attn_fwd(hstu_dtype_t dtype,
                             const void* q, int64_t q_tok_stride,
                             const void* k, int64_t k_tok_stride,
@@ -141,12 +154,12 @@ hstu_status_t hstu_attn_fwd(hstu_dtype_t dtype,
  * counterpart: this is an interface convenience of this library.
  *
  * Same arguments, layouts and results as hstu_attn_fwd, minus the workspace:
- * the bf16 path keeps its work list in a file-scope device array of
- * HSTU_NOALLOC_SCRATCH_BYTES (1 MiB), which every GPU that loads the library
- * holds until the process exits. A batch needing more than that, i.e.
- * hstu_attn_workspace_bytes(B, total_tokens, max_seqlen) > 1 MiB (the work
- * list takes 32 bytes per unit: roughly B + total_tokens/128 > 32,700),
- * returns
+ * the bf16 path keeps its work list and bias tables in a file-scope device
+ * array of HSTU_NOALLOC_SCRATCH_BYTES (16 MiB), which every GPU that loads
+ * the library holds until the process exits. A batch needing more than that,
+ * i.e. hstu_attn_workspace_bytes(B, total_tokens, max_seqlen, H, num_pos) >
+ * 16 MiB (about 600 bytes per work unit, plus 3968 bytes per head and
+ * 128-token diagonal offset of the position window), returns
  * HSTU_ERR_UNSUPPORTED before anything is launched; use hstu_attn_fwd then.
  * Nothing is allocated or freed by this call, including by torch or any
  * other library.
@@ -158,7 +171,7 @@ hstu_status_t hstu_attn_fwd(hstu_dtype_t dtype,
  * before the attention kernel reads them, so nothing has to be cleared. Calls
  * whose executions overlap on the GPU (other streams, or graphs replayed
  * concurrently) race on the array. */
-#define HSTU_NOALLOC_SCRATCH_BYTES 1048576
+#define HSTU_NOALLOC_SCRATCH_BYTES 16777216
 hstu_status_t hstu_attn_fwd_noalloc(hstu_dtype_t dtype,
                                     const void* q, int64_t q_tok_stride,
                                     const void* k, int64_t k_tok_stride,

@@ -77,8 +77,12 @@ def hstu_device_status(stream=None) -> int:
     return _lib().hstu_device_status(_stream(stream))
 
 
-def hstu_attn_workspace_bytes(B: int, total_tokens: int, max_seqlen: int) -> int:
-    return int(_lib().hstu_attn_workspace_bytes(B, total_tokens, max_seqlen))
+def hstu_attn_workspace_bytes(B: int, total_tokens: int, max_seqlen: int, H: int,
+                              num_pos: int = 1) -> int:
+    """Workspace of hstu_attn_plan + hstu_attn_run (bf16): the plan's work list,
+    then the run's bias tables (num_pos: the position table's length, or 1
+    without a position term)."""
+    return int(_lib().hstu_attn_workspace_bytes(B, total_tokens, max_seqlen, H, max(num_pos, 1)))
 
 
 def _workspace(nbytes: int, device) -> torch.Tensor:
@@ -145,7 +149,8 @@ def hstu_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, seq_offsets
         out = torch.empty((T, H, v.shape[2]), dtype=q.dtype, device=q.device)
     a = _attn_args(q, k, v, seq_offsets, timestamps, pos_bias, time_bias, max_seqlen, out)
     if workspace is None and a["dtype"] == _native.HSTU_DTYPE_BF16:
-        workspace = _workspace(hstu_attn_workspace_bytes(a["B"], T, max_seqlen), q.device)
+        workspace = _workspace(hstu_attn_workspace_bytes(a["B"], T, max_seqlen, a["H"], a["P"]),
+                               q.device)
     _native.check("hstu_attn_fwd", _lib().hstu_attn_fwd(
         a["dtype"], a["q"], a["qs"], a["k"], a["ks"], a["v"], a["vs"], a["off"], a["B"], a["T"],
         a["H"], a["dqk"], a["dv"], a["ts"], a["pos"], a["P"], a["tb"], a["NB"], a["N"], a["out"],

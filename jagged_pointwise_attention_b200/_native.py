@@ -17,7 +17,7 @@ SIGNATURES = {
     "hstu_abi_version": (c_i32, []),
     "hstu_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "hstu_device_status": (ctypes.c_int, [c_p]),
-    "hstu_attn_workspace_bytes": (c_sz, [c_i32, c_i64, c_i32]),
+    "hstu_attn_workspace_bytes": (c_sz, [c_i32, c_i64, c_i32, c_i32, c_i32]),
     "hstu_attn_plan": (ctypes.c_int, [c_p, c_i32, c_i64, c_i32, c_p, c_sz, c_p]),
     "hstu_attn_run": (ctypes.c_int, [ctypes.c_int, c_p, c_i64, c_p, c_i64, c_p, c_i64, c_p, c_i32,
                                      c_i64, c_i32, c_i32, c_i32, c_p, c_p, c_i32, c_p, c_i32,

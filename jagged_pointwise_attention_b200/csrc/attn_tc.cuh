@@ -69,11 +69,16 @@
 
 namespace hstu {
 
+struct KeySummary;
+
 struct AttnArgs {
     const int4* units;          // plan: (q0, q_end, k0, nk | nt << 11 | packed << 31)
     const int* unit_count;
     int* item_counter;          // plan: zeroed; next work item to hand out
     const uint4* starts;        // plan: per packed unit, rows where a sequence begins
+    const uint4* ptab;          // bias prep: [H][DD][248] window tables (see BiasStage)
+    int DD;                     // window tables per head (diagonal offsets 0..DD-1)
+    const KeySummary* ksum;     // bias prep: per unit, its 128 tokens as keys; null without time
     int H;
     int64_t T;
     const int64_t* ts;          // [T] or null
@@ -108,19 +113,31 @@ struct AttnCfg {
 // c0..c0+31 as entries k0, k0+8, k0+16, k0+24 (k0 = 127 - r + c0), four
 // 16-byte loads whose word p packs columns (c0+2p, c0+2p+1). Entry s lies in
 // 16-byte bank slot s mod 8, so the eight consecutive k0 of a quarter warp
-// never conflict.
+// never conflict. The window depends only on the head and on the tile's
+// diagonal offset (q0 - kt0) / 128, so the tables are built once per launch
+// (bias_prep_kernel) and copied in per tile.
 // Key timestamps are kept relative to `base` (the tile's first key) in 32
 // bits, exact whenever every timestamp involved lies within 2^30 of base:
 // ok[c] says so for the keys of chunk c, and cmin/cmax are the chunk's
-// smallest and largest key timestamp minus base.
-struct alignas(16) BiasStage {
-    uint4 wb[248];         // sliding-window table of bf16 pos/2
-    uint32_t r32[128];     // its source: word m packs R[2m], R[2m+1] (R[255] = 0)
+// smallest and largest key timestamp minus base. They depend only on the
+// key tile, i.e. on the unit whose rows are those keys, and are also built
+// once per launch.
+constexpr int kWinEntries = 248;
+constexpr int kWinBytes = kWinEntries * 16;
+
+struct alignas(16) KeySummary {
     int32_t kt32[128];     // key timestamps minus base (exact when ok[] holds)
     int64_t base;          // timestamp of the tile's first key
     int32_t cmin[4], cmax[4], ok[4];
     int32_t pad[2];
 };
+static_assert(sizeof(KeySummary) == 576, "key summary copy size");
+
+struct alignas(16) BiasStage {
+    uint4 wb[kWinEntries]; // sliding-window table of bf16 pos/2
+    KeySummary keys;
+};
+static_assert(sizeof(BiasStage) == kWinBytes + sizeof(KeySummary), "stage layout");
 
 template <int D, int G>
 struct AttnSmem {
@@ -158,10 +175,10 @@ enum {
     kBarDrain = 29,     // the S issuer's last commit
     kBarItemFull = 30,  // +slot (8): scheduler published an item
     kBarItemFree = 38,  // +slot (8): every consumer has read it
-    kBarStage = 46,     // +2g+s (up to 6): the 128 threads of group g staged stage s
+    kBarStage = 46,     // +2g+s (up to 6): the copies into stage s of group g landed
     kBarPVDone = 52,    // +buffer (up to 3): PV of the buffer's tile has completed
     kBarDrainPV = 55,   // the PV issuer's last commit
-    kBarStageSrc = 56,  // +2g+s (up to 6): group g wrote the window source words of stage s
+    kBarStageFree = 56, // +2g+s (up to 6): the four warps of group g are done with stage s
     kBarCount = 64,
 };
 static_assert(kBarCount == AttnSmem<64, kAttnGroups>::kNumBars, "barrier slots");
@@ -170,6 +187,7 @@ static_assert(kBarCount == AttnSmem<64, kAttnGroups>::kNumBars, "barrier slots")
 // unit index (packed tiles look up their sequence starts with it).
 struct Item {
     int q0, q_end, k0, nk, h, s0;
+    int kb;   // unit whose rows are key tile 0 (key tile j: unit kb - j)
     bool packed;
 };
 
@@ -194,6 +212,7 @@ __device__ __forceinline__ Item load_item(const AttnArgs& a, int w) {
     it.s0 = u;
     it.nk = wu.w & 0x7ff;
     it.h = h;
+    it.kb = ubase + nt - 1;   // units hold tiles nt-1 .. 0
     return it;
 }
 
@@ -206,6 +225,7 @@ __device__ __forceinline__ Item read_item(const volatile int* slot) {
     it.h = slot[4];
     it.packed = slot[5] != 0;
     it.s0 = slot[6];
+    it.kb = slot[7];
     return it;
 }
 
@@ -406,10 +426,10 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
         for (int b = 0; b < G; ++b) {
             mbar_init(&bars[kBarSFull + b], 1);
             mbar_init(&bars[kBarPFull + b], 128);
-            mbar_init(&bars[kBarStage + 2 * b], 128);
-            mbar_init(&bars[kBarStage + 2 * b + 1], 128);
-            mbar_init(&bars[kBarStageSrc + 2 * b], 128);
-            mbar_init(&bars[kBarStageSrc + 2 * b + 1], 128);
+            mbar_init(&bars[kBarStage + 2 * b], 1);
+            mbar_init(&bars[kBarStage + 2 * b + 1], 1);
+            mbar_init(&bars[kBarStageFree + 2 * b], 4);
+            mbar_init(&bars[kBarStageFree + 2 * b + 1], 4);
         }
         for (int b = 0; b < G; ++b) mbar_init(&bars[kBarOFull + b], 1);
         for (int o = 0; o < OB; ++o) mbar_init(&bars[kBarOFree + o], 128);
@@ -479,7 +499,7 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                     if (w < n_items) {
                         I = load_item(args, w);
                     } else {
-                        I.q0 = I.q_end = I.k0 = I.h = I.s0 = 0;
+                        I.q0 = I.q_end = I.k0 = I.h = I.s0 = I.kb = 0;
                         I.nk = 0;
                         I.packed = false;
                     }
@@ -491,6 +511,7 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                     e[4] = I.h;
                     e[5] = I.packed ? 1 : 0;
                     e[6] = I.s0;
+                    e[7] = I.kb;
                     mbar_arrive(&bars[kBarItemFull + slot]);
                 } else if (!take_item(it, false, I)) {
                     ok = false;
@@ -511,7 +532,13 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                 }
                 for (int j = 0; j < I.nk; ++j, ++n) {
                     const int ks = n % S;
-                    if (n >= S && !mbar_wait(&freeb[ks], ((n / S) - 1) & 1, abort_flag)) {
+                    // with K: the tile's bias data goes into stage (n / G) & 1 of group
+                    // n % G, once the group is done with that stage's previous tile
+                    const int sidx = 2 * (n % G) + ((n / G) & 1);
+                    const int use = n / (2 * G);
+                    if ((n >= S && !mbar_wait(&freeb[ks], ((n / S) - 1) & 1, abort_flag)) ||
+                        (is_k && use > 0 &&
+                         !mbar_wait(&bars[kBarStageFree + sidx], (use - 1) & 1, abort_flag))) {
                         ok = false;
                         break;
                     }
@@ -520,6 +547,17 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                     for (int kb = 0; kb < kKB; ++kb)
                         tma_load_2d(smem + ring + ks * kTileBytes + kb * 16384, tm, &full[ks],
                                     I.h * D + kb * 64, I.k0 + j * kTile);
+                    if (is_k) {
+                        BiasStage& st = stages[sidx];
+                        const int dd = min(I.nk - 1 - j, args.DD - 1);     // diagonal offset
+                        mbar_arrive_expect_tx(&bars[kBarStage + sidx],
+                                              kWinBytes + (args.ksum ? sizeof(KeySummary) : 0));
+                        bulk_load(st.wb, args.ptab + (static_cast<int64_t>(I.h) * args.DD + dd) * kWinEntries,
+                                  kWinBytes, &bars[kBarStage + sidx]);
+                        if (args.ksum)
+                            bulk_load(&st.keys, args.ksum + (I.kb - j), sizeof(KeySummary),
+                                      &bars[kBarStage + sidx]);
+                    }
                 }
                 if (!ok) {
                     ++it;   // this item's Q load was issued
@@ -534,6 +572,15 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                 if (is_k && cq > 0 && !mbar_wait(&bars[kBarQFull + s], (cq - 1) & 1, nullptr))
                     raise_error(kErrTimeout);
                 if (ck > 0 && !mbar_wait(&full[s], (ck - 1) & 1, nullptr)) raise_error(kErrTimeout);
+            }
+            // stage (g, b) took the tiles g + G k, k even (b = 0) or odd (b = 1), k < K_g
+            for (int g = 0; is_k && g < G; ++g) {
+                const int kg = n > g ? (n - g + G - 1) / G : 0;
+                for (int b = 0; b < 2; ++b) {
+                    const int c = kg > b ? (kg - b + 1) / 2 : 0;
+                    if (c > 0 && !mbar_wait(&bars[kBarStage + 2 * g + b], (c - 1) & 1, nullptr))
+                        raise_error(kErrTimeout);
+                }
             }
         }
         __syncwarp();
@@ -643,66 +690,6 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
         const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
         const uint32_t s_col = tmem + lane_base + static_cast<uint32_t>(g * 128);
 
-        // Stage the bias data of key tile kt0 of item I (every thread of the
-        // group takes part: window source word r, then after the group has
-        // written all of them table entries r and r + 128; key r, and the
-        // timestamp summary of chunk qd, whose keys are this warp's lanes).
-        auto stage_tile = [&](const Item& I, int kt0, BiasStage& st, uint64_t* full, uint64_t* src,
-                              uint32_t src_parity) -> bool {
-            // every global load first, so that their latencies overlap
-            const int64_t key = static_cast<int64_t>(kt0) + r;
-            const bool kvalid = key < I.q_end;
-            int64_t kv = 0, base = 0;
-            if (use_time) {
-                kv = __ldg(args.ts + (key < args.T ? key : args.T - 1));
-                base = __ldg(args.ts + kt0);
-            }
-            {
-                // word r = (R[2r], R[2r+1]), R[k] = pos[h][clamp(i - j)] / 2 with
-                // i - j = q0 - kt0 + 127 - k, and R[255] = 0
-                uint32_t wd = 0u;
-                if (args.pos) {
-                    const float* prow = args.pos + static_cast<int64_t>(I.h) * args.P;
-                    const int rel0 = I.q0 - kt0 + 127 - 2 * r;
-                    const float v0 = __ldg(prow + min(max(rel0, 0), args.P - 1));
-                    const float v1 = r < 127 ? __ldg(prow + min(max(rel0 - 1, 0), args.P - 1)) : 0.f;
-                    // bf16(v) / 2 is exactly bf16(v / 2) (a power-of-two scale)
-                    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(wd) : "r"(pack_bf16x2(v0, v1)), "r"(0x3f003f00u));
-                }
-                st.r32[r] = wd;
-            }
-            mbar_arrive(src);
-            if (!warp_wait(src, src_parity, abort_flag)) return false;
-            // entry s = R[s..s+7]: words s/2 .. s/2+4, shifted by one half for odd s
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int se = r + 128 * e;
-                if (se < 248) {
-                    const int w0 = se >> 1;
-                    const uint32_t sel = (se & 1) ? 0x5432u : 0x3210u;
-                    uint32_t x[5];
-#pragma unroll
-                    for (int k = 0; k < 5; ++k) x[k] = st.r32[w0 + k];
-                    st.wb[se] = make_uint4(__byte_perm(x[0], x[1], sel), __byte_perm(x[1], x[2], sel),
-                                           __byte_perm(x[2], x[3], sel), __byte_perm(x[3], x[4], sel));
-                }
-            }
-            const int64_t dk = kv - base;
-            st.kt32[r] = static_cast<int32_t>(dk);
-            const bool near = dk > -(1ll << 30) && dk < (1ll << 30);
-            const int dmin = __reduce_min_sync(0xffffffffu, (kvalid && near) ? static_cast<int>(dk) : INT_MAX);
-            const int dmax = __reduce_max_sync(0xffffffffu, (kvalid && near) ? static_cast<int>(dk) : INT_MIN);
-            const bool all_near = __all_sync(0xffffffffu, !kvalid || near);
-            if (lane == 0) {
-                st.cmin[qd] = dmin;
-                st.cmax[qd] = dmax;
-                st.ok[qd] = all_near ? 1 : 0;
-            }
-            if (r == 0) st.base = base;
-            mbar_arrive(full);
-            return true;
-        };
-
         bool ok = true;
         int n = 0, it = 0, ep = 0;   // ep: outputs this group has written
         int nt = 0;                  // tiles this group has processed (stage nt % 2)
@@ -729,10 +716,8 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                 if (n % G != g) continue;
                 const int kt0 = I.k0 + j * kTile;
                 const int sb = nt & 1;
-                BiasStage& st = stages[2 * g + sb];
-                if (!stage_tile(I, kt0, st, &bars[kBarStage + 2 * g + sb],
-                                &bars[kBarStageSrc + 2 * g + sb], (nt >> 1) & 1) ||
-                    !warp_wait(&bars[kBarStage + 2 * g + sb], (nt >> 1) & 1, abort_flag) ||
+                const BiasStage& st = stages[2 * g + sb];   // copied in by the K producer
+                if (!warp_wait(&bars[kBarStage + 2 * g + sb], (nt >> 1) & 1, abort_flag) ||
                     !warp_wait(&bars[kBarSFull + g], (n / G) & 1, abort_flag)) {
                     ok = false;
                     break;
@@ -745,8 +730,8 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                     bool fast = true;
                     int32_t tib = 0;                        // ti - base, when fast
                     if (use_time) {
-                        const int64_t db = ti - st.base;
-                        fast = st.ok[0] && st.ok[1] && st.ok[2] && st.ok[3] &&
+                        const int64_t db = ti - st.keys.base;
+                        fast = st.keys.ok[0] && st.keys.ok[1] && st.keys.ok[2] && st.keys.ok[3] &&
                                (!row_valid || (db > -(1ll << 30) && db < (1ll << 30)));
                         tib = static_cast<int32_t>(db);
                     }
@@ -760,8 +745,8 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                     bool tile_const = tile_full && fast_w;
                     float t_tile = 0.f;
                     if (tile_const && use_time) {
-                        const int kmin = min(min(st.cmin[0], st.cmin[1]), min(st.cmin[2], st.cmin[3]));
-                        const int kmax = max(max(st.cmax[0], st.cmax[1]), max(st.cmax[2], st.cmax[3]));
+                        const int kmin = min(min(st.keys.cmin[0], st.keys.cmin[1]), min(st.keys.cmin[2], st.keys.cmin[3]));
+                        const int kmax = max(max(st.keys.cmax[0], st.keys.cmax[1]), max(st.keys.cmax[2], st.keys.cmax[3]));
                         const uint32_t ef_hi = log2_exponent_field(static_cast<uint32_t>(max(tib - kmin, 1)));
                         const uint32_t ef_lo = log2_exponent_field(static_cast<uint32_t>(max(tib - kmax, 1)));
                         t_tile = __shfl_sync(0xffffffffu, tbr, static_cast<int>(ef_lo));
@@ -799,8 +784,8 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                                 path = 0;
                                 tl = t_tile;
                                 if (use_time && !tile_const) {
-                                    const uint32_t ef_hi = log2_exponent_field(static_cast<uint32_t>(max(tib - st.cmin[q], 1)));
-                                    const uint32_t ef_lo = log2_exponent_field(static_cast<uint32_t>(max(tib - st.cmax[q], 1)));
+                                    const uint32_t ef_hi = log2_exponent_field(static_cast<uint32_t>(max(tib - st.keys.cmin[q], 1)));
+                                    const uint32_t ef_lo = log2_exponent_field(static_cast<uint32_t>(max(tib - st.keys.cmax[q], 1)));
                                     tl = __shfl_sync(0xffffffffu, tbr, static_cast<int>(ef_lo));
                                     th = __shfl_sync(0xffffffffu, tbr, static_cast<int>(ef_hi));
                                     // bucket ef_hi iff dt >= 2^(ef_hi - 1023) (>= 2 when ef_hi > ef_lo)
@@ -810,8 +795,8 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                                 }
                             }
                             if (path == 0) pw_const(sv, wbr + c0, pack_bf16x2(tl, tl), pk);
-                            else if (path == 1) pw_two(sv, c0, wbr + c0, st.kt32, kthr, tl, th, pk);
-                            else pw_fast<true>(sv, c0, wbr + c0, st.kt32, tib, tbr, lo, hi, pk);
+                            else if (path == 1) pw_two(sv, c0, wbr + c0, st.keys.kt32, kthr, tl, th, pk);
+                            else pw_fast<true>(sv, c0, wbr + c0, st.keys.kt32, tib, tbr, lo, hi, pk);
                         }
                         // 32 bf16 results -> columns 32q..32q+15 of the S buffer just read
                         tmem_st16_async(s_col + c0, pk);
@@ -820,6 +805,8 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                 tmem_wait_st();     // every P store of the tile has landed
                 tc_fence_before();
                 mbar_arrive(&bars[kBarPFull + g]);
+                __syncwarp();       // the warp's last read of the stage is behind it
+                if (lane == 0) mbar_arrive(&bars[kBarStageFree + 2 * g + sb]);
                 if (j == I.nk - 1) {
                     // this group handled the item's last tile: store its output
                     const int ob = it % OB;

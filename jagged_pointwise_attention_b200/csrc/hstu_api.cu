@@ -13,6 +13,7 @@
 #include "hstu.h"
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
+#include "bias_prep.cuh"
 #include "common.cuh"
 #include "debug.cuh"
 #include "gemm_tc.cuh"
@@ -100,8 +101,27 @@ int64_t max_units_of(int32_t B, int64_t T, int32_t max_seqlen) {
 constexpr size_t kAttnWsHeader = 256;   // unit count (int at 0), item counters (2 ints at 16)
 
 // attention workspace: [header][units: int4 x max_units][starts: uint4 x max_units]
+// (the plan's part), then [window tables: H x DD x 3968 B][key summaries:
+// 576 B x max_units] (built per run by the bias prep kernel)
 size_t attn_units_bytes(int32_t B, int64_t T, int32_t max_seqlen) {
     return (static_cast<size_t>(max_units_of(B, T, max_seqlen)) * 16 + 255) / 256 * 256;
+}
+
+size_t attn_plan_bytes(int32_t B, int64_t T, int32_t max_seqlen) {
+    return kAttnWsHeader + 2 * attn_units_bytes(B, T, max_seqlen);
+}
+
+// window tables of a run: P = num_pos (1 when there is no position term)
+int attn_window_tables(int32_t P, int32_t max_seqlen) {
+    return window_tables(P > 0 ? P : 1, max_tiles_of(max_seqlen));
+}
+
+size_t attn_tables_bytes(int32_t H, int32_t P, int32_t max_seqlen) {
+    return static_cast<size_t>(H) * attn_window_tables(P, max_seqlen) * kWinBytes;
+}
+
+size_t attn_keys_bytes(int32_t B, int64_t T, int32_t max_seqlen) {
+    return static_cast<size_t>(max_units_of(B, T, max_seqlen)) * sizeof(KeySummary);
 }
 
 int num_sms() {
@@ -140,7 +160,7 @@ struct AttnCall {
     int32_t max_seqlen;
     void* out;
     int64_t os;
-    const void* ws;
+    void* ws;
     size_t ws_bytes;
     cudaStream_t stream;
 };
@@ -161,7 +181,8 @@ hstu_status_t validate_attn(const AttnCall& c) {
         if (!aligned16(c.q) || !aligned16(c.k) || !aligned16(c.v) || !aligned16(c.out))
             return HSTU_ERR_INVALID_ARG;
         if (c.qs % 8 || c.ks % 8 || c.vs % 8 || c.os % 8) return HSTU_ERR_INVALID_ARG;
-        if (!c.ws || c.ws_bytes < hstu_attn_workspace_bytes(c.B, c.T, c.max_seqlen))
+        if (!c.ws || c.ws_bytes < hstu_attn_workspace_bytes(c.B, c.T, c.max_seqlen, c.H,
+                                                            c.pos ? c.P : 1))
             return HSTU_ERR_INVALID_ARG;
         if (!aligned16(c.ws)) return HSTU_ERR_INVALID_ARG;
     } else {
@@ -217,12 +238,40 @@ hstu_status_t run_attn(const AttnCall& c) {
         !make_tmap_bf16(&tv, c.v, inner, c.T, c.vs * 2, 128))
         return HSTU_ERR_CUDA;
     const int64_t max_units = max_units_of(c.B, c.T, c.max_seqlen);
-    const uint8_t* ws = static_cast<const uint8_t*>(c.ws);
+    uint8_t* ws = static_cast<uint8_t*>(c.ws);
+    const int P = c.pos ? c.P : 1;
+    const int DD = attn_window_tables(P, c.max_seqlen);
+    uint4* ptab = reinterpret_cast<uint4*>(ws + attn_plan_bytes(c.B, c.T, c.max_seqlen));
+    KeySummary* ksum = reinterpret_cast<KeySummary*>(
+        ws + attn_plan_bytes(c.B, c.T, c.max_seqlen) + attn_tables_bytes(c.H, P, c.max_seqlen));
+    // bias tables of this run (programmatic dependent of the plan)
+    {
+        const int64_t entries = static_cast<int64_t>(c.H) * DD * kWinEntries;
+        const int table_blocks = static_cast<int>((entries + 127) / 128);
+        BiasPrepArgs pa{c.pos, P, c.H, DD, ptab, reinterpret_cast<const int4*>(ws + kAttnWsHeader),
+                        reinterpret_cast<const int*>(ws), static_cast<int>(max_units),
+                        use_time ? c.ts : nullptr, c.T, ksum, table_blocks};
+        const int64_t blocks = table_blocks + (use_time ? max_units : 0);
+        if (blocks > 0x7fffffff) return HSTU_ERR_UNSUPPORTED;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+        cfg.blockDim = dim3(128);
+        cfg.stream = c.stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, bias_prep_kernel, pa) != cudaSuccess) return HSTU_ERR_CUDA;
+    }
     AttnArgs a{reinterpret_cast<const int4*>(ws + kAttnWsHeader),
                reinterpret_cast<const int*>(ws),
-               reinterpret_cast<int*>(const_cast<uint8_t*>(ws) + 16),
+               reinterpret_cast<int*>(ws + 16),
                reinterpret_cast<const uint4*>(ws + kAttnWsHeader +
                                               attn_units_bytes(c.B, c.T, c.max_seqlen)),
+               ptab,
+               DD,
+               use_time ? ksum : nullptr,
                c.H,
                c.T,
                use_time ? c.ts : nullptr,
@@ -257,7 +306,7 @@ hstu_status_t plan_attn(const int64_t* off, int32_t B, int64_t T, int32_t max_se
                         size_t ws_bytes, cudaStream_t stream) {
     if (!plan_sizes_ok(B, T, max_seqlen)) return HSTU_ERR_INVALID_ARG;
     if (B == 0 || T == 0) return HSTU_OK;
-    if (!off || !ws || !aligned16(ws) || ws_bytes < hstu_attn_workspace_bytes(B, T, max_seqlen))
+    if (!off || !ws || !aligned16(ws) || ws_bytes < attn_plan_bytes(B, T, max_seqlen))
         return HSTU_ERR_INVALID_ARG;
     const int max_tiles = max_tiles_of(max_seqlen);
     const int64_t max_units = max_units_of(B, T, max_seqlen);
@@ -367,7 +416,8 @@ LayerWs layer_ws(int64_t T, int32_t B, int32_t H, int32_t d, int32_t max_seqlen)
     w.attn = round_up(w.uvqk + static_cast<size_t>(T) * 4 * F * 2, 256);
     w.y = round_up(w.attn + static_cast<size_t>(T) * F * 2, 256);
     w.plan = round_up(w.y + static_cast<size_t>(T) * F * 2, 256);
-    w.total = w.plan + hstu_attn_workspace_bytes(B, T, max_seqlen);
+    // window tables for any num_pos: at most one per 128-token diagonal offset
+    w.total = w.plan + hstu_attn_workspace_bytes(B, T, max_seqlen, H, 128 * max_tiles_of(max_seqlen));
     return w;
 }
 
@@ -403,9 +453,12 @@ hstu_status_t hstu_device_status(void* stream) {
     return HSTU_OK;
 }
 
-size_t hstu_attn_workspace_bytes(int32_t B, int64_t total_tokens, int32_t max_seqlen) {
-    if (!plan_sizes_ok(B, total_tokens, max_seqlen)) return 0;
-    return kAttnWsHeader + 2 * attn_units_bytes(B, total_tokens, max_seqlen);
+size_t hstu_attn_workspace_bytes(int32_t B, int64_t total_tokens, int32_t max_seqlen, int32_t H,
+                                 int32_t num_pos) {
+    if (!plan_sizes_ok(B, total_tokens, max_seqlen) || H < 1 || num_pos < 0) return 0;
+    return attn_plan_bytes(B, total_tokens, max_seqlen) +
+           attn_tables_bytes(H, num_pos > 0 ? num_pos : 1, max_seqlen) +
+           attn_keys_bytes(B, total_tokens, max_seqlen);
 }
 
 hstu_status_t hstu_attn_plan(const int64_t* seq_offsets, int32_t B, int64_t total_tokens,
@@ -421,7 +474,7 @@ hstu_status_t hstu_attn_run(hstu_dtype_t dtype, const void* q, int64_t q_tok_str
                             int64_t total_tokens, int32_t H, int32_t d_qk, int32_t d_v,
                             const int64_t* timestamps, const float* pos_bias, int32_t num_pos,
                             const float* time_bias, int32_t num_time_buckets, int32_t max_seqlen,
-                            void* out, int64_t out_tok_stride, const void* workspace,
+                            void* out, int64_t out_tok_stride, void* workspace,
                             size_t workspace_bytes, void* stream) {
     AttnCall c{dtype, q, k, v, q_tok_stride, k_tok_stride, v_tok_stride, seq_offsets, B,
                total_tokens, H, d_qk, d_v, timestamps, pos_bias, num_pos, time_bias,
@@ -582,7 +635,8 @@ extern "C" hstu_status_t hstu_attn_fwd_noalloc(
     int32_t max_seqlen, void* out, int64_t out_tok_stride, void* stream) {
     void* scratch = nullptr;
     if (dtype == HSTU_DTYPE_BF16 && B > 0 && total_tokens > 0) {
-        const size_t need = hstu_attn_workspace_bytes(B, total_tokens, max_seqlen);
+        const size_t need = hstu_attn_workspace_bytes(B, total_tokens, max_seqlen, H,
+                                                      pos_bias ? num_pos : 1);
         if (need == 0) return HSTU_ERR_INVALID_ARG;
         if (need > HSTU_NOALLOC_SCRATCH_BYTES) return HSTU_ERR_UNSUPPORTED;
         const hstu_status_t st = noalloc_scratch(&scratch);

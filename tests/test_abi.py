@@ -51,15 +51,23 @@ def test_library_loads_without_gpu(lib):
 
 
 def test_workspace_queries(lib):
-    w = lib.hstu_attn_workspace_bytes(16, 90000, 8192)
-    # header + one int4 per (sequence, query tile), bounded by T/128 + B + 1 and
-    # rounded up to 256 bytes, and as much again for the per-unit sequence-start
-    # masks of packed tiles
-    units = 16 * min(90000 // 128 + 16 + 1, 16 * 64)
-    assert w == 256 + 2 * ((units + 255) // 256 * 256)
-    assert lib.hstu_attn_workspace_bytes(-1, 10, 10) == 0
-    assert lib.hstu_attn_workspace_bytes(1, 10, 0) == 0
-    assert lib.hstu_attn_workspace_bytes(1, 10, 131073) == 0
+    # the plan's part: header + one int4 per (sequence, query tile), bounded by
+    # T/128 + B + 1 and rounded up to 256 bytes, and as much again for the
+    # per-unit sequence-start masks of packed tiles; then the run's bias
+    # tables: 3968 bytes per head and distinct diagonal offset of the
+    # position window, 576 bytes per unit of key summary
+    units = min(90000 // 128 + 16 + 1, 16 * 64)
+    plan = 256 + 2 * ((16 * units + 255) // 256 * 256)
+    # 8192 positions: offsets 0 .. ceil((8192 + 126) / 128) = 65, capped at 64 tiles
+    assert lib.hstu_attn_workspace_bytes(16, 90000, 8192, 4, 8192) == \
+        plan + 4 * 64 * 3968 + 576 * units
+    # 200 positions: offsets 0 .. ceil(326 / 128) = 3
+    assert lib.hstu_attn_workspace_bytes(16, 90000, 8192, 2, 200) == \
+        plan + 2 * 4 * 3968 + 576 * units
+    assert lib.hstu_attn_workspace_bytes(-1, 10, 10, 1, 1) == 0
+    assert lib.hstu_attn_workspace_bytes(1, 10, 0, 1, 1) == 0
+    assert lib.hstu_attn_workspace_bytes(1, 10, 131073, 1, 1) == 0
+    assert lib.hstu_attn_workspace_bytes(1, 10, 10, 0, 1) == 0
     lw = lib.hstu_layer_workspace_bytes(1000, 4, 4, 128, 512)
     assert lw >= 1000 * 512 * 2 * 6
 

@@ -170,7 +170,8 @@ def test_causality_on_gpu():
 def test_plan_then_run_matches_fwd():
     inp = make_attn_inputs(2)
     t = attn_tensors(inp)
-    ws = torch.empty(hstu.hstu_attn_workspace_bytes(inp.B, inp.T, inp.max_seqlen),
+    ws = torch.empty(hstu.hstu_attn_workspace_bytes(inp.B, inp.T, inp.max_seqlen, inp.H,
+                                                    inp.pos_bias.shape[1]),
                      dtype=torch.uint8, device="cuda")
     hstu.hstu_attn_plan(t["seq_offsets"], inp.max_seqlen, inp.T, ws)
     out = torch.empty_like(t["q"])
