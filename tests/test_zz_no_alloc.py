@@ -50,8 +50,9 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
 
 def test_noalloc_rejects_batches_beyond_its_scratch():
     lib = _native.load()
-    # 70000 sequences need more than the 1 MiB work-list array: refused on the
-    # host before anything is launched
+    # 70000 sequences (70000 work units: 2.2 MB of work list, 40 MB of key
+    # summaries) need more than the 16 MiB scratch array: refused on the host
+    # before anything is launched
     B, T = 70000, 70000 * 4
     st = lib.hstu_attn_fwd_noalloc(_native.HSTU_DTYPE_BF16, 16, 512, 16, 512, 16, 512, 16, B, T,
                                    4, 128, 128, None, None, 0, None, 0, 4, 16, 512, None)
