@@ -12,7 +12,7 @@
 //    the 128-bit mask = row q0 + r), from which the kernel finds each row's
 //    own sequence start to mask pairs that cross a sequence boundary. Packing
 //    is greedy inside each 128-token bucket of sequence start positions, so
-//    buckets are packed in parallel.
+//    buckets are packed in parallel, each in one pass by one thread.
 // Aligned units are listed sequence by sequence, longest sequence first, and
 // inside a sequence by descending query tile (descending nk); packed units
 // follow. The attention kernel hands out work items (unit, head) in the order
@@ -109,8 +109,8 @@ __device__ __forceinline__ void plan_body(const int64_t* __restrict__ seq_offset
         }
     }
     // packed units. The first non-empty short sequence of each 128-token start
-    // bucket packs the short sequences of its bucket greedily: once to count
-    // (slots reserved with one atomic per warp), once to write.
+    // bucket packs the short sequences of its bucket greedily in one pass;
+    // each unit takes its slot with a shared-memory atomic as it closes.
     for (int b0 = warp * 32; b0 < B; b0 += nwarps * 32) {
         const int b = b0 + lane;
         bool first = false;
@@ -127,54 +127,40 @@ __device__ __forceinline__ void plan_body(const int64_t* __restrict__ seq_offset
                 }
             }
         }
-        // greedy pass; emit(k, ts0, te, c0) is called for the k-th unit of the
-        // bucket (tokens [ts0, te), first sequence c0)
-        auto pack = [&](auto emit) {
-            int k = 0, cs = -1;
-            int64_t ts0 = -1, te = -1;
-            for (int c = b; c < B && off[c] / kTile == bucket; ++c) {
-                const int64_t nc = length(c);
-                if (nc == 0) continue;
-                if (nc > kTile) break;               // a long sequence ends the run
-                if (ts0 >= 0 && off[c] + nc - ts0 > kTile) {
-                    emit(k++, ts0, te, cs);
-                    ts0 = -1;
-                }
-                if (ts0 < 0) {
-                    ts0 = off[c];
-                    cs = c;
-                }
-                te = off[c] + nc;
+        if (!first) continue;
+        // the open unit: tokens [ts0, te), sequence-start mask m
+        int64_t ts0 = -1, te = -1;
+        uint32_t m0 = 0u, m1 = 0u, m2 = 0u, m3 = 0u;
+        auto close = [&]() {
+            const int slot = n_aligned + atomicAdd(&n_packed, 1);
+            if (slot < max_units) {
+                units[slot] = make_int4(static_cast<int>(ts0), static_cast<int>(te),
+                                        static_cast<int>(ts0), static_cast<int>(0x80000801u));
+                starts[slot] = make_uint4(m0, m1, m2, m3);
             }
-            if (ts0 >= 0) emit(k++, ts0, te, cs);
-            return k;
         };
-        const int mine = first ? pack([](int, int64_t, int64_t, int) {}) : 0;
-        int incl = mine;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += y;
+        for (int c = b; c < B && off[c] / kTile == bucket; ++c) {
+            const int64_t nc = length(c);
+            if (nc == 0) continue;
+            if (nc > kTile) break;                   // a long sequence ends the run
+            const int64_t oc = off[c];
+            if (ts0 >= 0 && oc + nc - ts0 > kTile) {
+                close();
+                ts0 = -1;
+            }
+            if (ts0 < 0) {
+                ts0 = oc;
+                m0 = m1 = m2 = m3 = 0u;
+            }
+            te = oc + nc;
+            const int r = static_cast<int>(oc - ts0);
+            const uint32_t bit = 1u << (r & 31);
+            m0 |= (r >> 5) == 0 ? bit : 0u;
+            m1 |= (r >> 5) == 1 ? bit : 0u;
+            m2 |= (r >> 5) == 2 ? bit : 0u;
+            m3 |= (r >> 5) == 3 ? bit : 0u;
         }
-        int wbase = 0;
-        if (lane == 31) wbase = atomicAdd(&n_packed, incl);
-        wbase = __shfl_sync(0xffffffffu, wbase, 31);
-        if (first) {
-            const int my0 = wbase + incl - mine;
-            pack([&](int k, int64_t ts0, int64_t te, int cs) {
-                const int slot = n_aligned + my0 + k;
-                if (slot < max_units) {
-                    units[slot] = make_int4(static_cast<int>(ts0), static_cast<int>(te),
-                                            static_cast<int>(ts0), static_cast<int>(0x80000801u));
-                    uint32_t m[4] = {0u, 0u, 0u, 0u};
-                    for (int c = cs; c < B && off[c] < te; ++c) {
-                        const int r = static_cast<int>(off[c] - ts0);
-                        m[r >> 5] |= 1u << (r & 31);
-                    }
-                    starts[slot] = make_uint4(m[0], m[1], m[2], m[3]);
-                }
-            });
-        }
+        if (ts0 >= 0) close();
     }
     __syncthreads();
     if (tid == 0) {
