@@ -513,6 +513,14 @@ def bench_layer(args, rank, world, local, peaks, peak_kind):
     max_ms, tot = reduce_timing(e0.elapsed_time(e1), float(fl) * args.steps, world, dev)
     _, toks = reduce_timing(0.0, float(li.T) * args.steps, world, dev)
     value = tot / (max_ms * 1e-3) / 1e12
+    # the step's six launches are timed together: the roofline is the step's
+    # FLOPs against the dense bf16 peak (the layer is tensor-bound throughout)
+    step_tf = fl / (max_ms / args.steps * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": round(step_tf, 2), "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": round(step_tf / peaks["bf16_tflops"], 4),
+                "peak_kind": "burst bf16 dense, %s" % peak_kind, "traffic": None,
+                "kernel": "whole layer step (f1, plan, bias tables, attention, LayerNorm gate, f2)"}
+    e2e = e2e_layer(args, li, dev, stream, fl, world, hstu, ws)
     return {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(max_ms / args.steps, 4),
@@ -523,9 +531,82 @@ def bench_layer(args, rank, world, local, peaks, peak_kind):
                    "l2": "layer working set > L2"},
         "tokens_per_s": round(toks / (max_ms * 1e-3), 1),
         "pct_of_bf16_peak": {"measured_burst": round(100 * value / peaks["bf16_tflops"], 2)},
-        "roofline": None, "cpu_baseline": None, "e2e": None,
-        "gpu_launches": 5 * args.steps, "clocks": sampler.summary(),
+        "roofline": roofline, "cpu_baseline": None, "e2e": e2e,
+        "gpu_launches": 6 * args.steps, "clocks": sampler.summary(),
     }
+
+
+def e2e_layer(args, li, dev, stream, flops, world, hstu, ws):
+    """End to end through hstu_layer_fwd: every step copies its activations x,
+    offsets and timestamps from pinned host memory and the output back; the
+    weights and bias tables are the model's parameters and stay on the device.
+    Pipelined like the attention's: step i's copies in overlap step i-1's
+    layer and step i-2's copy out."""
+    import torch
+    bf = torch.bfloat16
+
+    def pinned(a, dt=None):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        return (t.to(dt) if dt is not None else t).pin_memory()
+
+    to = lambda a, dt=None: (torch.from_numpy(np.ascontiguousarray(a)).to(dt)  # noqa: E731
+                             if dt else torch.from_numpy(np.ascontiguousarray(a))).to(dev)
+    W1, W2, pos, tb = to(li.W1, bf), to(li.W2, bf), to(li.pos_bias), to(li.time_bias)
+    host = dict(x=pinned(li.x, bf), off=pinned(li.seq_offsets), ts=pinned(li.timestamps))
+    devb = [{k: torch.empty_like(v, device=dev) for k, v in host.items()} for _ in range(2)]
+    out_dev = [torch.empty((li.T, li.D), dtype=bf, device=dev) for _ in range(2)]
+    out_host = [torch.empty((li.T, li.D), dtype=bf).pin_memory() for _ in range(2)]
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host[0].numel() * out_host[0].element_size()
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = {k: [torch.cuda.Event() for _ in range(2)] for k in ("in", "run", "out")}
+    used = [False, False]
+
+    def step(i):
+        b = i % 2
+        with torch.cuda.stream(s_in):
+            if used[b]:
+                s_in.wait_event(ev["run"][b])
+            for k in host:
+                devb[b][k].copy_(host[k], non_blocking=True)
+            ev["in"][b].record(s_in)
+        with torch.cuda.stream(stream):
+            stream.wait_event(ev["in"][b])
+            if used[b]:
+                stream.wait_event(ev["out"][b])
+            d = devb[b]
+            hstu.hstu_layer_fwd(d["x"], W1, W2, d["off"], d["ts"], pos, tb, li.H, li.d,
+                                li.max_seqlen, ln_eps=li.ln_eps, out=out_dev[b], workspace=ws,
+                                stream=stream)
+            ev["run"][b].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev["run"][b])
+            out_host[b].copy_(out_dev[b], non_blocking=True)
+            ev["out"][b].record(s_out)
+        used[b] = True
+
+    for i in range(max(2, min(args.warmup, 3))):
+        step(i)
+    n = max(1, min(args.steps, args.e2e_steps))
+    a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _barrier(world)
+    torch.cuda.synchronize(dev)
+    a.record(stream)
+    s_in.wait_stream(stream)
+    for i in range(n):
+        step(i)
+    for b in range(2):
+        stream.wait_event(ev["out"][b])
+        stream.wait_event(ev["in"][b])
+    e.record(stream)
+    torch.cuda.synchronize(dev)
+    _barrier(world)
+    ms, tot = reduce_timing(a.elapsed_time(e), float(flops) * n, world, dev)
+    return {"value": round(tot / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": n,
+            "ms_per_step": round(ms / n, 4),
+            "pipeline": "step i's host-to-device copies overlap step i-1's layer and step "
+                        "i-2's device-to-host copy (three streams, two buffer sets)"}
 
 
 def _barrier(world):
