@@ -60,6 +60,14 @@ def _bind(lib):
     lib.hstu_oracle_layer.restype = ctypes.c_int
     lib.hstu_oracle_layer.argtypes = [_i64, _i32, _p, _p, _p, _p, _p, _p, _p, _f64, _p, _i32,
                                       _i32, _i32, _p, _p, _i32, _p, _i32, _i32, _p, _i64, _p]
+    lib.hstu_oracle_e4m3_to_float.restype = ctypes.c_float
+    lib.hstu_oracle_e4m3_to_float.argtypes = [ctypes.c_uint8]
+    lib.hstu_oracle_e4m3_from_float.restype = ctypes.c_uint8
+    lib.hstu_oracle_e4m3_from_float.argtypes = [ctypes.c_float]
+    lib.hstu_oracle_quant_rows_e4m3.restype = None
+    lib.hstu_oracle_quant_rows_e4m3.argtypes = [_i64, _i32, _p, _p, _p]
+    lib.hstu_oracle_linear_fp8.restype = None
+    lib.hstu_oracle_linear_fp8.argtypes = [_i64, _i32, _i32, _p, _p, _p, _p, _p, _i32, _p, _p]
     lib.hstu_oracle_num_threads.restype = ctypes.c_int
     lib.hstu_oracle_num_threads.argtypes = []
     return lib
@@ -155,6 +163,51 @@ def linear(x, W, bias=None, act_silu: bool = False, residual=None, lib=None) -> 
     y = np.zeros((max(M, 1), N), dtype=np.float64)
     lib.hstu_oracle_linear(M, K, N, _ptr(x), _ptr(W), _ptr(bias), int(bool(act_silu)),
                            _ptr(residual), _ptr(y))
+    return y[:M]
+
+
+def e4m3_to_float(codes, lib=None) -> np.ndarray:
+    """Values of E4M3 codes (uint8 array) as float32."""
+    lib = lib or load()
+    table = np.array([lib.hstu_oracle_e4m3_to_float(c) for c in range(256)], dtype=np.float32)
+    return table[np.asarray(codes, dtype=np.uint8)]
+
+
+def e4m3_from_float(x, lib=None) -> np.ndarray:
+    """E4M3 codes of float32 values: nearest, ties to even, saturating at +-448."""
+    lib = lib or load()
+    x = np.asarray(x, dtype=np.float32)
+    return np.array([lib.hstu_oracle_e4m3_from_float(float(v)) for v in x.ravel()],
+                    dtype=np.uint8).reshape(x.shape)
+
+
+def quant_rows_e4m3(x, lib=None):
+    """Row-wise E4M3 quantization of x [M, K] (float32 values): (codes uint8
+    [M, K], scales float32 [M]) with x ~ value(codes) * scales[:, None]."""
+    lib = lib or load()
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    M, K = x.shape
+    codes = np.zeros((max(M, 1), K), dtype=np.uint8)
+    scales = np.zeros(max(M, 1), dtype=np.float32)
+    lib.hstu_oracle_quant_rows_e4m3(M, K, _ptr(x), _ptr(codes), _ptr(scales))
+    return codes[:M], scales[:M]
+
+
+def linear_fp8(xq, sx, wq, sw, bias=None, act_silu: bool = False, residual=None,
+               lib=None) -> np.ndarray:
+    """act(value(xq) value(wq)^T * sx[:, None] * sw[None, :] + bias) + residual,
+    fp64 from the E4M3 codes. xq [M, K], wq [N, K] uint8."""
+    lib = lib or load()
+    xq = np.ascontiguousarray(xq, dtype=np.uint8)
+    wq = np.ascontiguousarray(wq, dtype=np.uint8)
+    sx = np.ascontiguousarray(sx, dtype=np.float32)
+    sw = np.ascontiguousarray(sw, dtype=np.float32)
+    bias, residual = _f64a(bias), _f64a(residual)
+    M, K = xq.shape
+    N = wq.shape[0]
+    y = np.zeros((max(M, 1), N), dtype=np.float64)
+    lib.hstu_oracle_linear_fp8(M, K, N, _ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), _ptr(bias),
+                               int(bool(act_silu)), _ptr(residual), _ptr(y))
     return y[:M]
 
 

@@ -160,6 +160,104 @@ void hstu_oracle_linear(int64_t M, int32_t K, int32_t N, const double* x, const 
     }
 }
 
+/* ---------------------------------------------------------------- FP8 (E4M3)
+ * Row-wise E4M3 quantization and FP8 addmm for the layer's two projections
+ * (generative-recommenders README, section "FP8 linear reference and
+ * benchmark": row-wise E4M3 quantization of both operands, fp32
+ * accumulation, the row scales applied to the product).
+ *
+ * E4M3 (the OCP 8-bit float "E4M3FN" format): 1 sign bit, 4 exponent bits
+ * with bias 7, 3 mantissa bits. Exponent field 0 holds the subnormals
+ * m/8 * 2^-6; fields 1..15 hold (1 + m/8) * 2^(e - 7), except that field 15
+ * with mantissa 7 is NaN (no infinities), so the largest finite magnitude is
+ * 1.75 * 2^8 = 448. Conversion rounds to the nearest value, ties to an even
+ * mantissa, and saturates finite overflow (and infinity) to +-448. */
+
+float hstu_oracle_e4m3_to_float(uint8_t c) {
+    const int sign = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m / 8.0, -6);
+    else v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return (float)(sign ? -v : v);
+}
+
+/* nearest integer to q >= 0, ties to even */
+static double round_half_even(double q) {
+    const double f = floor(q), r = q - f;
+    if (r > 0.5) return f + 1.0;
+    if (r < 0.5) return f;
+    return fmod(f, 2.0) == 0.0 ? f : f + 1.0;
+}
+
+uint8_t hstu_oracle_e4m3_from_float(float x) {
+    if (isnan(x)) return 0x7F;
+    const uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    const double a = fabs((double)x);
+    if (a >= 448.0) return sign | 0x7E;                 /* saturate (448 itself included) */
+    if (a < ldexp(1.0, -6)) {                           /* subnormal range: steps of 2^-9 */
+        const double m = round_half_even(a / ldexp(1.0, -9));
+        return sign | (uint8_t)m;                       /* m == 8 is the smallest normal */
+    }
+    int ex;
+    const double f = frexp(a, &ex);                     /* a = f 2^ex, f in [0.5, 1) */
+    int e = ex - 1;                                     /* a = (2f) 2^e, 2f in [1, 2) */
+    double m = round_half_even((2.0 * f - 1.0) * 8.0);
+    if (m == 8.0) {
+        m = 0.0;
+        e += 1;
+    }
+    const int field = e + 7;
+    if (field > 15 || (field == 15 && m == 7.0)) return sign | 0x7E;
+    return sign | (uint8_t)((field << 3) | (int)m);
+}
+
+/* Row-wise quantization of x [M, K] (fp32 values): amax_r = max |x[r, :]|;
+ * inv_r = 448 / amax_r and scale_r = amax_r / 448 in fp32 (an all-zero row
+ * takes inv 0 and scale 1); code[r, c] = e4m3(x[r, c] * inv_r) with the product
+ * rounded to fp32 first. Then x[r, c] ~ e4m3_to_float(code) * scale_r. */
+void hstu_oracle_quant_rows_e4m3(int64_t M, int32_t K, const float* x, uint8_t* codes,
+                                 float* scales) {
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < M; ++r) {
+        float amax = 0.0f;
+        for (int32_t c = 0; c < K; ++c) {
+            const float v = fabsf(x[r * K + c]);
+            if (v > amax) amax = v;
+        }
+        volatile float inv = amax > 0.0f ? 448.0f / amax : 0.0f;
+        volatile float scale = amax > 0.0f ? amax / 448.0f : 1.0f;
+        for (int32_t c = 0; c < K; ++c) {
+            volatile float y = x[r * K + c] * inv;
+            codes[r * K + c] = hstu_oracle_e4m3_from_float(y);
+        }
+        scales[r] = scale;
+    }
+}
+
+/* y[m, n] = act(sum_c e4m3(xq[m, c]) e4m3(wq[n, c]) sx[m] sw[n] + bias[n])
+ *           + residual[m, n], in fp64 from the codes; xq [M, K], wq [N, K]. */
+void hstu_oracle_linear_fp8(int64_t M, int32_t K, int32_t N, const uint8_t* xq,
+                            const float* sx, const uint8_t* wq, const float* sw,
+                            const double* bias, int32_t act_silu, const double* residual,
+                            double* y) {
+    double lut[256];
+    for (int c = 0; c < 256; ++c) lut[c] = (double)hstu_oracle_e4m3_to_float((uint8_t)c);
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int32_t n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int32_t c = 0; c < K; ++c)
+                acc += lut[xq[m * K + c]] * lut[wq[(int64_t)n * K + c]];
+            acc *= (double)sx[m] * (double)sw[n];
+            if (bias) acc += bias[n];
+            if (act_silu) acc = hstu_oracle_silu(acc);
+            if (residual) acc += residual[m * N + n];
+            y[m * N + n] = acc;
+        }
+    }
+}
+
 /* y[m, :] = LayerNorm(a[m, :]) * u[m, :] over F features: biased variance,
  * eps inside the square root, then gamma / beta (NULL = 1 / 0).
  * a, u, y have row strides a_ld, u_ld, F. */

@@ -419,11 +419,116 @@ def check_layer_identities(lib):
     _close(out, x, 0.0, "U = 0 must give out = x")
 
 
+# --------------------------------------------------------------------------- FP8 (E4M3)
+
+def _e4m3_grid():
+    """Every finite non-negative E4M3 value from the format's definition:
+    subnormals m/8 * 2^-6, normals (1 + m/8) * 2^(e - 7), e = 1..15, without
+    the NaN pattern e = 15, m = 7."""
+    vals = [m / 8.0 * 2.0 ** -6 for m in range(8)]
+    vals += [(1 + m / 8.0) * 2.0 ** (e - 7) for e in range(1, 16) for m in range(8)
+             if not (e == 15 and m == 7)]
+    return np.array(vals)
+
+
+def check_e4m3_table(lib):
+    """Decoding every code gives the format's value grid (by construction here),
+    NaN for the two all-ones patterns, and encoding a decoded value gives the
+    code back."""
+    codes = np.arange(256, dtype=np.uint8)
+    vals = oracle.e4m3_to_float(codes, lib=lib).astype(np.float64)
+    assert np.isnan(vals[0x7F]) and np.isnan(vals[0xFF])
+    pos = np.delete(vals[:128], 0x7F)
+    assert np.array_equal(pos, _e4m3_grid()), "positive codes 0..126"
+    assert np.array_equal(np.delete(vals[128:], 0x7F), -_e4m3_grid()), "negative codes"
+    assert vals[0x7E] == 448.0 and vals[1] == 2.0 ** -9
+    finite = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    back = oracle.e4m3_from_float(oracle.e4m3_to_float(finite, lib=lib), lib=lib)
+    assert np.array_equal(back, finite), "round trip"
+
+
+def check_e4m3_rounding_against_torch(lib):
+    """Encoding agrees with torch's float8_e4m3fn cast (round to nearest, ties
+    to even) on every grid value, every midpoint between neighbours, points
+    just off the midpoints, and random values, of both signs, below the
+    saturation threshold."""
+    import torch
+    g = _e4m3_grid()
+    mids = (g[:-1] + g[1:]) / 2
+    off = np.concatenate([mids * (1 + 2.0 ** -20), mids * (1 - 2.0 ** -20)])
+    rng = np.random.default_rng(7)
+    rnd = np.exp(rng.uniform(np.log(2.0 ** -12), np.log(440.0), 4000))
+    x = np.concatenate([g, mids, off, rnd, [2.0 ** -11, 3 * 2.0 ** -11, 1e-30]]).astype(np.float32)
+    x = np.concatenate([x, -x])
+    got = oracle.e4m3_from_float(x, lib=lib)
+    want = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    bad = np.nonzero(got != want)[0]
+    assert bad.size == 0, "codes differ from torch at %s" % x[bad[:5]]
+
+
+def check_e4m3_saturation(lib):
+    """Finite overflow and infinity saturate to +-448 (code 0x7E / 0xFE); NaN
+    stays NaN."""
+    x = np.array([448.0, 449.0, 464.0, 480.0, 1e6, np.inf, -500.0, -np.inf], dtype=np.float32)
+    got = oracle.e4m3_from_float(x, lib=lib)
+    assert list(got) == [0x7E] * 6 + [0xFE] * 2
+    assert oracle.e4m3_from_float(np.array([np.nan], np.float32), lib=lib)[0] == 0x7F
+
+
+def check_quant_rows(lib):
+    """Row-wise quantization: the row's largest magnitude maps to 448 exactly;
+    scaling a row by a power of two leaves its codes alone and scales its
+    scale; an all-zero row gives zero codes and scale 1; the dequantized
+    values are within half a step of the E4M3 grid (relative 2^-4 in the
+    normal range, 2^-10 * scale below it)."""
+    rng = np.random.default_rng(3)
+    x = (rng.standard_normal((6, 40)) * np.array([1, 10, 1e-3, 300, 2.0 ** 20, 1])[:, None]).astype(np.float32)
+    x[5] = 0.0
+    codes, scales = oracle.quant_rows_e4m3(x, lib=lib)
+    amax = np.abs(x).max(axis=1)
+    for r in range(5):
+        i = int(np.argmax(np.abs(x[r])))
+        assert codes[r, i] & 0x7F == 0x7E, "row %d amax code" % r
+        assert scales[r] == np.float32(amax[r] / np.float32(448.0))
+    assert np.all(codes[5] & 0x7F == 0) and scales[5] == 1.0
+    c2, s2 = oracle.quant_rows_e4m3(x * np.float32(8.0), lib=lib)
+    assert np.array_equal(c2, codes) and np.array_equal(s2[:5], scales[:5] * 8)
+    deq = oracle.e4m3_to_float(codes, lib=lib).astype(np.float64) * scales[:, None]
+    err = np.abs(deq - x)
+    normal = np.abs(x) >= (2.0 ** -6) * scales[:, None] * 1.0001
+    assert np.all(err[normal] <= 2.0 ** -4 * np.abs(x[normal]) * (1 + 1e-6)), "normal range"
+    assert np.all(err[~normal] <= 2.0 ** -10 * np.broadcast_to(scales[:, None], x.shape)[~normal]
+                  * (1 + 1e-6)), "subnormal range"
+
+
+def check_linear_fp8(lib):
+    """FP8 addmm equals the fp64 product of the dequantized operands (numpy),
+    with bias, SiLU and residual as in the plain linear."""
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((9, 32)).astype(np.float32)
+    W = rng.standard_normal((5, 32)).astype(np.float32)
+    xq, sx = oracle.quant_rows_e4m3(x, lib=lib)
+    wq, sw = oracle.quant_rows_e4m3(W, lib=lib)
+    xd = oracle.e4m3_to_float(xq, lib=lib).astype(np.float64) * sx[:, None]
+    wd = oracle.e4m3_to_float(wq, lib=lib).astype(np.float64) * sw[:, None]
+    b = rng.standard_normal(5)
+    r = rng.standard_normal((9, 5))
+    _close(oracle.linear_fp8(xq, sx, wq, sw, lib=lib), xd @ wd.T, what="fp8 linear")
+    _close(oracle.linear_fp8(xq, sx, wq, sw, b, True, lib=lib), _silu_t(xd @ wd.T + b),
+           what="fp8 silu")
+    _close(oracle.linear_fp8(xq, sx, wq, sw, None, False, r, lib=lib), xd @ wd.T + r,
+           what="fp8 residual")
+    # and it approximates the unquantized product
+    assert np.linalg.norm(xd @ wd.T - x.astype(np.float64) @ W.T.astype(np.float64)) < \
+        0.1 * np.linalg.norm(x.astype(np.float64) @ W.T.astype(np.float64))
+
+
 ALL_CHECKS = [
     check_floor_log2, check_time_bucket, check_pos_index, check_bias_indices_array, check_silu,
     check_dense_bruteforce, check_padded_equals_jagged, check_causality,
     check_batch_independence, check_rows_subset, check_empty_and_length_one,
     check_closed_form_prefix_sum, check_time_only_closed_form, check_pos_only_toeplitz,
     check_scale_is_max_seqlen, check_qk_asymmetry, check_linear, check_layernorm_gate,
-    check_layer_composition, check_layer_identities,
+    check_layer_composition, check_layer_identities, check_e4m3_table,
+    check_e4m3_rounding_against_torch, check_e4m3_saturation, check_quant_rows, check_linear_fp8,
 ]

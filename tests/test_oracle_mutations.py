@@ -39,8 +39,27 @@ MUTANTS = [
     ("split_u_v_swapped", "memcpy(urow + r * F, uvqk + t * W,", "memcpy(urow + r * F, uvqk + t * W + F,"),
     ("residual_dropped", "hstu_oracle_linear(n, (int32_t)F, D, ygate, W2, b2, 0, xrow, out);",
      "hstu_oracle_linear(n, (int32_t)F, D, ygate, W2, b2, 0, NULL, out);"),
-    ("linear_bias_dropped", "if (bias) acc += bias[n];", ""),
-    ("silu_after_bias_missing", "if (act_silu) acc = hstu_oracle_silu(acc);", ""),
+    ("linear_bias_dropped",
+     "for (int32_t c = 0; c < K; ++c) acc += x[m * K + c] * W[(int64_t)n * K + c];\n"
+     "            if (bias) acc += bias[n];",
+     "for (int32_t c = 0; c < K; ++c) acc += x[m * K + c] * W[(int64_t)n * K + c];\n"),
+    ("silu_after_bias_missing",
+     "if (bias) acc += bias[n];\n            if (act_silu) acc = hstu_oracle_silu(acc);\n"
+     "            if (residual) acc += residual[m * N + n];\n            y[m * N + n] = acc;\n"
+     "        }\n    }\n}\n\n/* ------",
+     "if (bias) acc += bias[n];\n"
+     "            if (residual) acc += residual[m * N + n];\n            y[m * N + n] = acc;\n"
+     "        }\n    }\n}\n\n/* ------"),
+    ("e4m3_ties_away", "return fmod(f, 2.0) == 0.0 ? f : f + 1.0;", "return f + 1.0;"),
+    ("e4m3_exponent_bias_8", "else v = ldexp(1.0 + (double)m / 8.0, e - 7);",
+     "else v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
+    ("e4m3_no_subnormals", "if (e == 0) v = ldexp((double)m / 8.0, -6);",
+     "if (e == 0) v = 0.0;"),
+    ("e4m3_overflow_to_nan", "if (a >= 448.0) return sign | 0x7E;",
+     "if (a > 448.0) return sign | 0x7F;"),
+    ("quant_scale_not_amax", "if (v > amax) amax = v;", "if (v > amax) amax = v * 0.5f;"),
+    ("fp8_scale_inverted", "acc *= (double)sx[m] * (double)sw[n];",
+     "acc *= (double)sx[m] / (double)sw[n];"),
 ]
 
 
