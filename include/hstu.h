@@ -203,6 +203,34 @@ hstu_status_t hstu_debug_wait_timeout(int32_t wait_us, void* stream);
 
 /* ---------------------------------------------------------------- layer */
 
+/* ---------------------------------------------------------------- FP8 projections */
+
+/* Row-wise E4M3 quantization (generative-recommenders README, "FP8 linear
+ * reference and benchmark": row-wise E4M3 quantization of the projection
+ * operands). For each row r of x (device bf16 [M, K], row stride ldx):
+ *   amax = max |x[r, :]|, inv = 448 / amax, scales[r] = amax / 448 (fp32,
+ *   rounded to nearest; an all-zero row gets inv = 0, scales[r] = 1),
+ *   codes[r, c] = E4M3(fp32(x[r, c] * inv)), rounding to nearest (ties to an
+ *   even mantissa) and saturating finite overflow at +-448,
+ * so that x[r, c] ~ value(codes[r, c]) * scales[r]. codes: device uint8
+ * [M, K], row stride ldq (multiple of 16); scales: device fp32 [M]. K % 16
+ * == 0, ldx % 8 == 0, x and codes 16-byte aligned. One launch, one warp per
+ * row. */
+hstu_status_t hstu_quant_rows_e4m3(const void* x, int64_t ldx, int64_t M, int32_t K, void* codes,
+                                   int64_t ldq, float* scales, void* stream);
+
+/* FP8 addmm on tcgen05 (kind::f8f6f4): y[M, N] = epilogue(
+ *   (value(xq) value(wq)^T)[m, n] * x_scales[m] * w_scales[n] + bias[n])
+ * with xq [M, K] and wq [N, K] E4M3 codes from hstu_quant_rows_e4m3 (row
+ * strides ldx, ldw, multiples of 16), fp32 accumulation, and the epilogues,
+ * residual, bias and output of hstu_linear_fwd (y, residual bf16). K % 128 ==
+ * 0, N % 128 == 0. */
+hstu_status_t hstu_linear_fp8_fwd(const void* xq, int64_t ldx, const float* x_scales, int64_t M,
+                                  int32_t K, const void* wq, int64_t ldw, const float* w_scales,
+                                  int32_t N, const float* bias, hstu_epilogue_t epilogue,
+                                  const void* residual, int64_t ldr, void* y, int64_t ldy,
+                                  void* stream);
+
 /* y[M, N] = epilogue(x[M, K] W[N, K]^T + bias[N]) on tcgen05 tensor cores.
  * x, W, y, residual: device bf16, row strides ldx, ldw (=K typically), ldy, ldr.
  * bias: device fp32 [N] or NULL. residual: [M, N] bf16, required for

@@ -25,6 +25,7 @@ __all__ = [
     "hstu_attn_fwd", "hstu_attn_plan", "hstu_attn_run", "hstu_attn_workspace_bytes",
     "hstu_layer_fwd", "hstu_layer_workspace_bytes", "hstu_linear_fwd",
     "hstu_layernorm_gate_fwd", "hstu_debug_bias_indices", "hstu_debug_wait_timeout",
+    "hstu_quant_rows_e4m3", "hstu_linear_fp8_fwd",
     "hstu_device_status", "HstuError", "library_path",
 ]
 
@@ -194,6 +195,44 @@ def hstu_linear_fwd(x: torch.Tensor, W: torch.Tensor, bias: Optional[torch.Tenso
     _native.check("hstu_linear_fwd", _lib().hstu_linear_fwd(
         _ptr(x), x.stride(0), M, K, _ptr(W), W.stride(0), N, _ptr(bias), epi, _ptr(residual),
         0 if residual is None else residual.stride(0), _ptr(out), out.stride(0), _stream(stream)))
+    return out
+
+
+def hstu_quant_rows_e4m3(x: torch.Tensor, stream=None):
+    """Row-wise E4M3 quantization of a bf16 [M, K] matrix: (codes uint8 [M, K],
+    scales fp32 [M]) with x ~ value(codes) * scales[:, None]."""
+    _on_cuda(x)
+    if x.dtype != torch.bfloat16 or x.stride(1) != 1:
+        raise ValueError("x must be bf16 with unit column stride")
+    M, K = x.shape
+    codes = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+    scales = torch.empty(M, dtype=torch.float32, device=x.device)
+    _native.check("hstu_quant_rows_e4m3", _lib().hstu_quant_rows_e4m3(
+        _ptr(x), x.stride(0), M, K, _ptr(codes), codes.stride(0), _ptr(scales), _stream(stream)))
+    return codes, scales
+
+
+def hstu_linear_fp8_fwd(xq: torch.Tensor, x_scales: torch.Tensor, wq: torch.Tensor,
+                        w_scales: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                        epilogue: str = "none", residual: Optional[torch.Tensor] = None,
+                        out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """epilogue(value(xq) value(wq)^T * x_scales[:, None] * w_scales + bias) with
+    E4M3 codes from hstu_quant_rows_e4m3; bf16 out (and residual)."""
+    _on_cuda(xq, x_scales, wq, w_scales, bias, residual, out)
+    M, K = xq.shape
+    N = wq.shape[0]
+    epi = {"none": _native.HSTU_EPI_NONE, "silu": _native.HSTU_EPI_SILU,
+           "residual": _native.HSTU_EPI_RESIDUAL}[epilogue]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=xq.device)
+    if xq.dtype != torch.uint8 or wq.dtype != torch.uint8 or xq.stride(1) != 1 or wq.stride(1) != 1:
+        raise ValueError("xq, wq must be uint8 E4M3 codes with unit column stride")
+    if x_scales.dtype != torch.float32 or w_scales.dtype != torch.float32:
+        raise ValueError("scales must be fp32")
+    _native.check("hstu_linear_fp8_fwd", _lib().hstu_linear_fp8_fwd(
+        _ptr(xq), xq.stride(0), _ptr(x_scales), M, K, _ptr(wq), wq.stride(0), _ptr(w_scales), N,
+        _ptr(bias), epi, _ptr(residual), 0 if residual is None else residual.stride(0),
+        _ptr(out), out.stride(0), _stream(stream)))
     return out
 
 

@@ -1,11 +1,14 @@
 // gemm_tc.cuh -- y = epilogue(x W^T + b) on tcgen05 for the HSTU layer's two
-// projections (UVQK with SiLU, output projection with the residual add).
+// projections (UVQK with SiLU, output projection with the residual add), in
+// bf16 or with row-wise E4M3 operands (FP8: y = epilogue((xq wq^T) * sx[m] *
+// sw[n] + b), generative-recommenders README, "FP8 linear reference and
+// benchmark").
 //
 // Persistent: one CTA per SM walks output tiles of 128 x BN (BN = 256 when N
 // allows, else 128) in row-block-major order, so the CTAs running together
 // share each 128-row block of x in L2 while W (at most a few MB) stays there.
-// K streams in 64-element (128-byte swizzled) blocks through a 4-stage TMA
-// ring; the fp32 accumulator of a tile lives in TMEM, two buffers of BN
+// K streams in 128-byte swizzled blocks (64 bf16 or 128 E4M3 elements)
+// through a 4-stage TMA ring; the fp32 accumulator of a tile lives in TMEM, two buffers of BN
 // columns, so the epilogue of one tile overlaps the main loop of the next.
 // Warp roles: 0-7 epilogue (two per TMEM lane quarter, one row per thread,
 // BN/2 columns each), 8 TMA producer, 9 MMA issuer and TMEM owner. The
@@ -28,6 +31,8 @@ constexpr int kGemmThreads = (kGemmEpiWarps + 2) * 32;
 struct GemmArgs {
     int64_t M;
     int N, K;
+    const float* sx;                // FP8: [M] row scales of x
+    const float* sw;                // FP8: [N] row scales of W
     const float* bias;              // [N] or null
     const __nv_bfloat16* residual;  // [M, N] (ldr) or null
     int64_t ldr;
@@ -50,7 +55,7 @@ struct GemmSmem {
     static_assert(kAlloc <= 227 * 1024, "shared memory per block");
 };
 
-template <int EPI, int BN>   // EPI: hstu_epilogue_t (0 none, 1 silu, 2 residual)
+template <int EPI, int BN, bool FP8 = false>   // EPI: hstu_epilogue_t (0 none, 1 silu, 2 residual)
 __global__ void __launch_bounds__(kGemmThreads, 1)
 gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmR,
@@ -63,7 +68,8 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int nkb = g.K / 64;
+    constexpr int kKBlock = FP8 ? 128 : 64;   // elements per 128-byte k-block
+    const int nkb = g.K / kKBlock;
     const int tiles_n = g.N / BN;
     const int tiles = static_cast<int>((g.M + 127) / 128) * tiles_n;
 
@@ -117,8 +123,8 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                         break;
                     }
                     mbar_arrive_expect_tx(&full[s], L::kStageBytes);
-                    tma_load_2d(smem + L::kOffA + s * 16384, &tmA, &full[s], kb * 64, m0);
-                    tma_load_2d(smem + L::kOffB + s * L::kBBytes, &tmB, &full[s], kb * 64, n0);
+                    tma_load_2d(smem + L::kOffA + s * 16384, &tmA, &full[s], kb * kKBlock, m0);
+                    tma_load_2d(smem + L::kOffB + s * L::kBBytes, &tmB, &full[s], kb * kKBlock, n0);
                 }
             }
             // drain: stage s took ceil((it - s) / S) loads
@@ -131,7 +137,7 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     } else if (warp == kWarpMMA) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16_f32(128, BN, 0, 0);
+            constexpr uint32_t idesc = FP8 ? idesc_e4m3_f32(128, BN) : idesc_bf16_f32(128, BN, 0, 0);
             int it = 0, tl = 0;  // k-blocks consumed; tiles of this CTA
             bool ok = true;
             for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x, ++tl) {
@@ -149,11 +155,14 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                         break;
                     }
                     tc_fence_after();
+                    // four MMAs of 32 bytes of K each (K = 16 bf16 or 32 E4M3)
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_bf16_ss(acc, desc_kmajor_sw128(sA + s * 16384 + kk * 32),
-                                     desc_kmajor_sw128(sB + s * L::kBBytes + kk * 32), idesc,
-                                     (kb > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t da = desc_kmajor_sw128(sA + s * 16384 + kk * 32);
+                        const uint64_t db = desc_kmajor_sw128(sB + s * L::kBBytes + kk * 32);
+                        if (FP8) umma_f8_ss(acc, da, db, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+                        else umma_bf16_ss(acc, da, db, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+                    }
                     umma_commit(&empty[s]);
                 }
                 if (ok) umma_commit(&acc_full[buf]);
@@ -212,9 +221,13 @@ gemm_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 }
                 {
                     float f[32];
+                    const float rs = FP8 ? __ldg(g.sx + min(static_cast<int64_t>(m0) + q * 32 + lane,
+                                                            g.M - 1))
+                                         : 1.f;
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         f[e] = __uint_as_float(v[e]);
+                        if (FP8) f[e] = f[e] * rs * __ldg(g.sw + col0 + e);
                         if (g.bias) f[e] += __ldg(g.bias + col0 + e);
                         if (EPI == 1) f[e] = silu_tanh(f[e]);
                     }

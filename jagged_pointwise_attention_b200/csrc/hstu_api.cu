@@ -19,6 +19,7 @@
 #include "gemm_tc.cuh"
 #include "ln_gate.cuh"
 #include "plan.cuh"
+#include "quant_fp8.cuh"
 
 using namespace hstu;
 
@@ -61,6 +62,22 @@ bool make_tmap_bf16_box(CUtensorMap* tm, const void* base, uint64_t inner, uint6
     const CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// Boxes of 128 E4M3 codes (128 bytes, 128-byte swizzle) x box_rows.
+bool make_tmap_u8(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t rows,
+                  uint64_t row_stride_bytes, uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {row_stride_bytes};
+    cuuint32_t box[2] = {128, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -321,29 +338,34 @@ hstu_status_t plan_attn(const int64_t* off, int32_t B, int64_t T, int32_t max_se
     return launch_status();
 }
 
-template <int EPI, int BN>
+template <int EPI, int BN, bool FP8 = false>
 hstu_status_t launch_gemm(unsigned grid, cudaStream_t stream, const CUtensorMap& ta,
                           const CUtensorMap& tb, const CUtensorMap& ty, const CUtensorMap& tr,
                           const GemmArgs& g) {
     static int done[kMaxDevices] = {0};
-    if (!ensure_smem(gemm_bf16_kernel<EPI, BN>, GemmSmem<BN>::kAlloc, done)) return HSTU_ERR_CUDA;
-    gemm_bf16_kernel<EPI, BN>
+    if (!ensure_smem(gemm_bf16_kernel<EPI, BN, FP8>, GemmSmem<BN>::kAlloc, done))
+        return HSTU_ERR_CUDA;
+    gemm_bf16_kernel<EPI, BN, FP8>
         <<<grid, kGemmThreads, GemmSmem<BN>::kAlloc, stream>>>(ta, tb, ty, tr, g);
     return launch_status();
 }
 
-hstu_status_t run_linear(const void* x, int64_t ldx, int64_t M, int32_t K, const void* W,
-                         int64_t ldw, int32_t N, const float* bias, hstu_epilogue_t epi,
-                         const void* residual, int64_t ldr, void* y, int64_t ldy,
-                         cudaStream_t stream) {
+// y = epilogue(x W^T [* sx sw] + b): bf16 operands, or E4M3 codes with
+// row scales (fp8)
+hstu_status_t run_linear_any(bool fp8, const void* x, int64_t ldx, const float* sx, int64_t M,
+                             int32_t K, const void* W, int64_t ldw, const float* sw, int32_t N,
+                             const float* bias, hstu_epilogue_t epi, const void* residual,
+                             int64_t ldr, void* y, int64_t ldy, cudaStream_t stream) {
     if (M < 0 || K < 1 || N < 1) return HSTU_ERR_INVALID_ARG;
     if (epi != HSTU_EPI_NONE && epi != HSTU_EPI_SILU && epi != HSTU_EPI_RESIDUAL)
         return HSTU_ERR_INVALID_ARG;
-    if (K % 64 || N % 128) return HSTU_ERR_UNSUPPORTED;
+    if (K % (fp8 ? 128 : 64) || N % 128) return HSTU_ERR_UNSUPPORTED;
     if (M == 0) return HSTU_OK;
     if (M > (int64_t{1} << 31) - 256) return HSTU_ERR_UNSUPPORTED;
     if (!x || !W || !y) return HSTU_ERR_INVALID_ARG;
-    if (ldx < K || ldw < K || ldy < N || ldx % 8 || ldw % 8 || ldy % 8) return HSTU_ERR_INVALID_ARG;
+    if (fp8 && (!sx || !sw)) return HSTU_ERR_INVALID_ARG;
+    const int ab = fp8 ? 16 : 8;     // elements per 16 bytes of an operand row
+    if (ldx < K || ldw < K || ldy < N || ldx % ab || ldw % ab || ldy % 8) return HSTU_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(W) || !aligned16(y)) return HSTU_ERR_INVALID_ARG;
     if (epi == HSTU_EPI_RESIDUAL && (!residual || ldr < N || ldr % 8 || !aligned16(residual)))
         return HSTU_ERR_INVALID_ARG;
@@ -352,9 +374,12 @@ hstu_status_t run_linear(const void* x, int64_t ldx, int64_t M, int32_t K, const
     const int bn = N % 256 == 0 ? 256 : 128;
     // output and residual in 32 x 32 blocks (64-byte rows, 64-byte swizzle)
     CUtensorMap ta, tb, ty, tr;
-    if (!make_tmap_bf16(&ta, x, K, M, ldx * 2, 128) ||
-        !make_tmap_bf16(&tb, W, K, N, ldw * 2, static_cast<uint32_t>(bn)) ||
-        !make_tmap_bf16_box(&ty, y, N, M, ldy * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+    const bool maps_ok =
+        fp8 ? make_tmap_u8(&ta, x, K, M, ldx, 128) &&
+                  make_tmap_u8(&tb, W, K, N, ldw, static_cast<uint32_t>(bn))
+            : make_tmap_bf16(&ta, x, K, M, ldx * 2, 128) &&
+                  make_tmap_bf16(&tb, W, K, N, ldw * 2, static_cast<uint32_t>(bn));
+    if (!maps_ok || !make_tmap_bf16_box(&ty, y, N, M, ldy * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
         return HSTU_ERR_CUDA;
     if (epi == HSTU_EPI_RESIDUAL) {
         if (!make_tmap_bf16_box(&tr, residual, N, M, ldr * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
@@ -362,22 +387,36 @@ hstu_status_t run_linear(const void* x, int64_t ldx, int64_t M, int32_t K, const
     } else {
         tr = ty;    // not read
     }
-    GemmArgs g{M, N, K, bias, static_cast<const __nv_bfloat16*>(residual), ldr,
+    GemmArgs g{M, N, K, sx, sw, bias, static_cast<const __nv_bfloat16*>(residual), ldr,
                static_cast<__nv_bfloat16*>(y), ldy};
     const int64_t tiles = (M + 127) / 128 * (N / bn);
     const unsigned grid = static_cast<unsigned>(tiles < num_sms() ? tiles : num_sms());
-    if (bn == 256) {
-        switch (epi) {
-            case HSTU_EPI_NONE: return launch_gemm<0, 256>(grid, stream, ta, tb, ty, tr, g);
-            case HSTU_EPI_SILU: return launch_gemm<1, 256>(grid, stream, ta, tb, ty, tr, g);
-            default: return launch_gemm<2, 256>(grid, stream, ta, tb, ty, tr, g);
-        }
+#define HSTU_GEMM_CASES(F8)                                                                   \
+    if (bn == 256) {                                                                          \
+        switch (epi) {                                                                        \
+            case HSTU_EPI_NONE: return launch_gemm<0, 256, F8>(grid, stream, ta, tb, ty, tr, g); \
+            case HSTU_EPI_SILU: return launch_gemm<1, 256, F8>(grid, stream, ta, tb, ty, tr, g); \
+            default: return launch_gemm<2, 256, F8>(grid, stream, ta, tb, ty, tr, g);          \
+        }                                                                                     \
+    }                                                                                         \
+    switch (epi) {                                                                            \
+        case HSTU_EPI_NONE: return launch_gemm<0, 128, F8>(grid, stream, ta, tb, ty, tr, g);   \
+        case HSTU_EPI_SILU: return launch_gemm<1, 128, F8>(grid, stream, ta, tb, ty, tr, g);   \
+        default: return launch_gemm<2, 128, F8>(grid, stream, ta, tb, ty, tr, g);            \
     }
-    switch (epi) {
-        case HSTU_EPI_NONE: return launch_gemm<0, 128>(grid, stream, ta, tb, ty, tr, g);
-        case HSTU_EPI_SILU: return launch_gemm<1, 128>(grid, stream, ta, tb, ty, tr, g);
-        default: return launch_gemm<2, 128>(grid, stream, ta, tb, ty, tr, g);
+    if (fp8) {
+        HSTU_GEMM_CASES(true)
     }
+    HSTU_GEMM_CASES(false)
+#undef HSTU_GEMM_CASES
+}
+
+hstu_status_t run_linear(const void* x, int64_t ldx, int64_t M, int32_t K, const void* W,
+                         int64_t ldw, int32_t N, const float* bias, hstu_epilogue_t epi,
+                         const void* residual, int64_t ldr, void* y, int64_t ldy,
+                         cudaStream_t stream) {
+    return run_linear_any(false, x, ldx, nullptr, M, K, W, ldw, nullptr, N, bias, epi, residual,
+                          ldr, y, ldy, stream);
 }
 
 hstu_status_t run_ln_gate(const void* a, int64_t lda, const void* u, int64_t ldu, int64_t M,
@@ -534,6 +573,30 @@ hstu_status_t hstu_linear_fwd(const void* x, int64_t ldx, int64_t M, int32_t K, 
                               void* stream) {
     return run_linear(x, ldx, M, K, W, ldw, N, bias, epilogue, residual, ldr, y, ldy,
                       as_stream(stream));
+}
+
+hstu_status_t hstu_quant_rows_e4m3(const void* x, int64_t ldx, int64_t M, int32_t K, void* codes,
+                                   int64_t ldq, float* scales, void* stream) {
+    if (M < 0 || K < 1) return HSTU_ERR_INVALID_ARG;
+    if (K % 16) return HSTU_ERR_UNSUPPORTED;
+    if (M == 0) return HSTU_OK;
+    if (!x || !codes || !scales || ldx < K || ldq < K || ldx % 8 || ldq % 16 || !aligned16(x) ||
+        !aligned16(codes))
+        return HSTU_ERR_INVALID_ARG;
+    if ((M + 7) / 8 > 0x7fffffff) return HSTU_ERR_UNSUPPORTED;
+    QuantArgs a{static_cast<const __nv_bfloat16*>(x), ldx, M, K, static_cast<uint8_t*>(codes),
+                ldq, scales};
+    quant_rows_e4m3_kernel<<<static_cast<unsigned>((M + 7) / 8), 256, 0, as_stream(stream)>>>(a);
+    return launch_status();
+}
+
+hstu_status_t hstu_linear_fp8_fwd(const void* xq, int64_t ldx, const float* x_scales, int64_t M,
+                                  int32_t K, const void* wq, int64_t ldw, const float* w_scales,
+                                  int32_t N, const float* bias, hstu_epilogue_t epilogue,
+                                  const void* residual, int64_t ldr, void* y, int64_t ldy,
+                                  void* stream) {
+    return run_linear_any(true, xq, ldx, x_scales, M, K, wq, ldw, w_scales, N, bias, epilogue,
+                          residual, ldr, y, ldy, as_stream(stream));
 }
 
 hstu_status_t hstu_layernorm_gate_fwd(const void* a, int64_t lda, const void* u, int64_t ldu,

@@ -188,6 +188,18 @@ __device__ __forceinline__ void umma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, u
         : "memory");
 }
 
+// D(tmem) (+)= A(smem desc) * B(smem desc)^T, kind::f8f6f4 (K = 32 per
+// instruction); the operand formats come from the instruction descriptor.
+__device__ __forceinline__ void umma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Arrive once on `bar` when every tcgen05 operation issued so far by this
 // thread has completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
@@ -336,6 +348,16 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_maj
            | (1u << 10)                                   // B format: bf16
            | (static_cast<uint32_t>(a_mn_major) << 15)    // A major
            | (static_cast<uint32_t>(b_mn_major) << 16)    // B major
+           | (static_cast<uint32_t>(N >> 3) << 17)        // N / 8
+           | (static_cast<uint32_t>(M >> 4) << 24);       // M / 16
+}
+
+// E4M3 x E4M3 -> f32, both operands K-major (kind::f8f6f4: format code 0 is
+// E4M3 in the A and B format fields).
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+    return (1u << 4)                                      // D format: f32
+           | (0u << 7)                                    // A format: E4M3
+           | (0u << 10)                                   // B format: E4M3
            | (static_cast<uint32_t>(N >> 3) << 17)        // N / 8
            | (static_cast<uint32_t>(M >> 4) << 24);       // M / 16
 }
