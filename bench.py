@@ -609,6 +609,72 @@ def e2e_layer(args, li, dev, stream, flops, world, hstu, ws):
                         "i-2's device-to-host copy (three streams, two buffer sets)"}
 
 
+def bench_fp8_linear(args, rank, world, local, peaks, peak_kind):
+    """Row-wise E4M3 projections against bf16 ones on the layer's f1 shape
+    (79,913 x 512 -> 2048, SiLU) and the FP8 benchmark shape of the
+    generative-recommenders README (4096 x 512 -> 512). A step = quantize the
+    activations + FP8 GEMM (weights quantized once, as a model would cache
+    them); the GEMM alone is timed too. FP8 peak = measured bf16 burst x 2
+    (the nominal dense ratio)."""
+    import torch
+    import jagged_pointwise_attention_b200 as hstu
+    dev = torch.device("cuda", local)
+    g = torch.Generator(device="cpu").manual_seed(1234 + rank)
+    fp8_peak = 2 * peaks["bf16_tflops"]
+    shapes = [("f1_layer_T79913_K512_N2048_silu", 79913, 512, 2048, "silu"),
+              ("addmm_bench_m4096_k512_n512", 4096, 512, 512, "none")]
+    out = []
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / args.steps
+
+    for name, M, K, N, epi in shapes:
+        x = torch.randn((M, K), generator=g).to(torch.bfloat16).to(dev)
+        W = (torch.randn((N, K), generator=g) / K ** 0.5).to(torch.bfloat16).to(dev)
+        wq, sw = hstu.hstu_quant_rows_e4m3(W)
+        xq, sx = hstu.hstu_quant_rows_e4m3(x)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        flops = 2.0 * M * N * K
+
+        def fp8_step():
+            q, s_ = hstu.hstu_quant_rows_e4m3(x)
+            hstu.hstu_linear_fp8_fwd(q, s_, wq, sw, None, epi, out=y)
+
+        ms_step = timed(fp8_step)
+        ms_gemm = timed(lambda: hstu.hstu_linear_fp8_fwd(xq, sx, wq, sw, None, epi, out=y))
+        ms_bf16 = timed(lambda: hstu.hstu_linear_fwd(x, W, None, epi, out=y))
+        assert hstu.hstu_device_status() == 0
+        out.append({"shape": name, "M": M, "K": K, "N": N, "epilogue": epi,
+                    "fp8_step_ms": round(ms_step, 4), "fp8_gemm_ms": round(ms_gemm, 4),
+                    "bf16_gemm_ms": round(ms_bf16, 4),
+                    "fp8_gemm_tflops": round(flops / (ms_gemm * 1e-3) / 1e12, 1),
+                    "fp8_step_tflops": round(flops / (ms_step * 1e-3) / 1e12, 1),
+                    "bf16_gemm_tflops": round(flops / (ms_bf16 * 1e-3) / 1e12, 1),
+                    "fp8_gemm_frac_of_peak": round(flops / (ms_gemm * 1e-3) / 1e12 / fp8_peak, 4)})
+    main_ = out[0]
+    return {"metric": "row-wise E4M3 projection TFLOP/s (quantize + FP8 GEMM)",
+            "value": main_["fp8_step_tflops"], "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+            "dtype": "e4m3 x e4m3 -> f32 -> bf16", "data": "synthetic (seeded generator)",
+            "config": {"workload": main_["shape"], "parallelism": "dp%d" % world},
+            "roofline": {"bound": "tensor", "achieved": main_["fp8_gemm_tflops"],
+                         "peak": fp8_peak, "unit": "TFLOP/s",
+                         "frac": main_["fp8_gemm_frac_of_peak"],
+                         "peak_kind": "fp8 dense = 2 x measured bf16 burst (nominal ratio), %s"
+                                      % peak_kind, "traffic": None,
+                         "kernel": "gemm_bf16_kernel<EPI, BN, FP8=true>"},
+            "shapes": out}
+
+
 def _barrier(world):
     if world > 1:
         import torch.distributed as dist
@@ -671,6 +737,9 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--reference-budget-s", type=float, default=120.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fp8-linear", action="store_true",
+                    help="time the row-wise E4M3 projections (quantize + FP8 GEMM) against the "
+                         "bf16 ones on the projection shapes instead of the attention")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the timed steps one call at a time instead of replaying "
                          "CUDA graphs")
@@ -697,7 +766,9 @@ def main(argv=None):
                                 device_id=torch.device("cuda", local))
     peaks, kind = load_peaks()
     from gen import CONFIGS
-    if CONFIGS[args.config]["kind"] == "layer":
+    if args.fp8_linear:
+        line = bench_fp8_linear(args, rank, world, local, peaks, kind)
+    elif CONFIGS[args.config]["kind"] == "layer":
         line = bench_layer(args, rank, world, local, peaks, kind)
     else:
         line = bench_attention(args, rank, world, local, peaks, kind)
