@@ -490,9 +490,20 @@ def bench_layer(args, rank, world, local, peaks, peak_kind):
     lengths = np.diff(li.seq_offsets)
     fl = causal_flops(lengths, li.H, li.d, li.d) + layer_flops(li.T, li.D, li.H, li.d)
 
+    if args.fp8:
+        W1q, s1 = hstu.hstu_quant_rows_e4m3(W1)
+        W2q, s2 = hstu.hstu_quant_rows_e4m3(W2)
+        ws = torch.empty(hstu.hstu_layer_fp8_workspace_bytes(li.T, li.B, li.D, li.H, li.d,
+                                                              li.max_seqlen),
+                         dtype=torch.uint8, device=dev)
+
     def step():
-        hstu.hstu_layer_fwd(x, W1, W2, off, ts, pos, tb, li.H, li.d, li.max_seqlen,
-                            ln_eps=li.ln_eps, out=out, workspace=ws)
+        if args.fp8:
+            hstu.hstu_layer_fp8_fwd(x, W1q, s1, W2q, s2, off, ts, pos, tb, li.H, li.d,
+                                    li.max_seqlen, ln_eps=li.ln_eps, out=out, workspace=ws)
+        else:
+            hstu.hstu_layer_fwd(x, W1, W2, off, ts, pos, tb, li.H, li.d, li.max_seqlen,
+                                ln_eps=li.ln_eps, out=out, workspace=ws)
 
     for _ in range(args.warmup):
         step()
@@ -520,19 +531,20 @@ def bench_layer(args, rank, world, local, peaks, peak_kind):
                 "unit": "TFLOP/s", "frac": round(step_tf / peaks["bf16_tflops"], 4),
                 "peak_kind": "burst bf16 dense, %s" % peak_kind, "traffic": None,
                 "kernel": "whole layer step (f1, plan, bias tables, attention, LayerNorm gate, f2)"}
-    e2e = e2e_layer(args, li, dev, stream, fl, world, hstu, ws)
+    e2e = None if args.fp8 else e2e_layer(args, li, dev, stream, fl, world, hstu, ws)
     return {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(max_ms / args.steps, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 projections, bf16 attention" if args.fp8 else "bf16",
         "data": "synthetic (seeded generator; no dataset)",
-        "config": {"workload": cfg["name"], "B": li.B, "D": li.D, "H": li.H, "d": li.d,
+        "config": {"workload": cfg["name"] + ("_fp8_projections" if args.fp8 else ""),
+                   "B": li.B, "D": li.D, "H": li.H, "d": li.d,
                    "total_tokens": li.T, "parallelism": "dp%d" % world,
                    "l2": "layer working set > L2"},
         "tokens_per_s": round(toks / (max_ms * 1e-3), 1),
         "pct_of_bf16_peak": {"measured_burst": round(100 * value / peaks["bf16_tflops"], 2)},
         "roofline": roofline, "cpu_baseline": None, "e2e": e2e,
-        "gpu_launches": 6 * args.steps, "clocks": sampler.summary(),
+        "gpu_launches": (7 if args.fp8 else 6) * args.steps, "clocks": sampler.summary(),
     }
 
 
@@ -737,6 +749,9 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--reference-budget-s", type=float, default=120.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fp8", action="store_true",
+                    help="with --config 5: the layer with both projections in FP8 "
+                         "(hstu_layer_fp8_fwd, weights quantized once)")
     ap.add_argument("--fp8-linear", action="store_true",
                     help="time the row-wise E4M3 projections (quantize + FP8 GEMM) against the "
                          "bf16 ones on the projection shapes instead of the attention")

@@ -231,6 +231,15 @@ hstu_status_t hstu_linear_fp8_fwd(const void* xq, int64_t ldx, const float* x_sc
                                   const void* residual, int64_t ldr, void* y, int64_t ldy,
                                   void* stream);
 
+/* hstu_layernorm_gate_fwd with the bf16 result row quantized row-wise to E4M3
+ * in the same kernel (as hstu_quant_rows_e4m3 would quantize it) instead of
+ * stored: codes device uint8 [M, F] (row stride ldq, multiple of 16), scales
+ * device fp32 [M]. The fused output-normalization-to-FP8 step before f2. */
+hstu_status_t hstu_layernorm_gate_fp8_fwd(const void* a, int64_t lda, const void* u, int64_t ldu,
+                                          int64_t M, int32_t F, const float* gamma,
+                                          const float* beta, float eps, void* codes,
+                                          int64_t ldq, float* scales, void* stream);
+
 /* y[M, N] = epilogue(x[M, K] W[N, K]^T + bias[N]) on tcgen05 tensor cores.
  * x, W, y, residual: device bf16, row strides ldx, ldw (=K typically), ldy, ldr.
  * bias: device fp32 [N] or NULL. residual: [M, N] bf16, required for
@@ -274,6 +283,28 @@ hstu_status_t hstu_layer_fwd(const void* x, int64_t total_tokens, int32_t D,
                              const float* time_bias, int32_t num_time_buckets,
                              int32_t max_seqlen, void* out,
                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes of hstu_layer_fp8_fwd (D: the model width of x). */
+size_t hstu_layer_fp8_workspace_bytes(int64_t total_tokens, int32_t B, int32_t D, int32_t H,
+                                      int32_t d, int32_t max_seqlen);
+
+/* hstu_layer_fwd with both projections in FP8: x is quantized row-wise to
+ * E4M3, f1 runs on E4M3 codes (SiLU epilogue), the attention in bf16, the
+ * LayerNorm gate writes E4M3 codes of its bf16 result, and f2 runs on E4M3
+ * codes with the bf16 residual x. W1q [4*H*d, D] / w1_scales [4*H*d] and W2q
+ * [D, H*d] / w2_scales [D] are the weights quantized once by
+ * hstu_quant_rows_e4m3 (device uint8 / fp32). D % 128 == 0, H*d % 256 == 0
+ * (so both K are multiples of 128), d in {64, 128}; other arguments as
+ * hstu_layer_fwd. Seven launches: quantize, f1, plan, bias tables, attention,
+ * LayerNorm gate, f2. */
+hstu_status_t hstu_layer_fp8_fwd(const void* x, int64_t total_tokens, int32_t D, const void* W1q,
+                                 const float* w1_scales, const float* b1, const void* W2q,
+                                 const float* w2_scales, const float* b2, const float* ln_gamma,
+                                 const float* ln_beta, float ln_eps, const int64_t* seq_offsets,
+                                 int32_t B, int32_t H, int32_t d, const int64_t* timestamps,
+                                 const float* pos_bias, int32_t num_pos, const float* time_bias,
+                                 int32_t num_time_buckets, int32_t max_seqlen, void* out,
+                                 void* workspace, size_t workspace_bytes, void* stream);
 
 #ifdef __cplusplus
 }

@@ -25,7 +25,8 @@ __all__ = [
     "hstu_attn_fwd", "hstu_attn_plan", "hstu_attn_run", "hstu_attn_workspace_bytes",
     "hstu_layer_fwd", "hstu_layer_workspace_bytes", "hstu_linear_fwd",
     "hstu_layernorm_gate_fwd", "hstu_debug_bias_indices", "hstu_debug_wait_timeout",
-    "hstu_quant_rows_e4m3", "hstu_linear_fp8_fwd",
+    "hstu_quant_rows_e4m3", "hstu_linear_fp8_fwd", "hstu_layernorm_gate_fp8_fwd",
+    "hstu_layer_fp8_workspace_bytes", "hstu_layer_fp8_fwd",
     "hstu_device_status", "HstuError", "library_path",
 ]
 
@@ -278,4 +279,54 @@ def hstu_layer_fwd(x: torch.Tensor, W1: torch.Tensor, W2: torch.Tensor, seq_offs
         0 if pos_bias is None else pos_bias.shape[1], _ptr(time_bias),
         0 if time_bias is None else time_bias.shape[1], int(max_seqlen), _ptr(out),
         _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out
+
+
+def hstu_layernorm_gate_fp8_fwd(a: torch.Tensor, u: torch.Tensor, gamma=None, beta=None,
+                                eps: float = 1e-5, stream=None):
+    """LayerNorm(a) * u with the bf16 result rows quantized to E4M3 in the same
+    kernel: (codes uint8 [M, F], scales fp32 [M])."""
+    _on_cuda(a, u, gamma, beta)
+    M, F = a.shape
+    codes = torch.empty((M, F), dtype=torch.uint8, device=a.device)
+    scales = torch.empty(M, dtype=torch.float32, device=a.device)
+    _native.check("hstu_layernorm_gate_fp8_fwd", _lib().hstu_layernorm_gate_fp8_fwd(
+        _ptr(a), a.stride(0), _ptr(u), u.stride(0), M, F, _ptr(gamma), _ptr(beta), float(eps),
+        _ptr(codes), codes.stride(0), _ptr(scales), _stream(stream)))
+    return codes, scales
+
+
+def hstu_layer_fp8_workspace_bytes(total_tokens: int, B: int, D: int, H: int, d: int,
+                                   max_seqlen: int) -> int:
+    return int(_lib().hstu_layer_fp8_workspace_bytes(total_tokens, B, D, H, d, max_seqlen))
+
+
+def hstu_layer_fp8_fwd(x: torch.Tensor, W1q: torch.Tensor, w1_scales: torch.Tensor,
+                       W2q: torch.Tensor, w2_scales: torch.Tensor, seq_offsets: torch.Tensor,
+                       timestamps: Optional[torch.Tensor], pos_bias: Optional[torch.Tensor],
+                       time_bias: Optional[torch.Tensor], H: int, d: int, max_seqlen: int,
+                       b1=None, b2=None, ln_gamma=None, ln_beta=None, ln_eps: float = 1e-5,
+                       out: Optional[torch.Tensor] = None,
+                       workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """hstu_layer_fwd with both projections in FP8 (E4M3 weights from
+    hstu_quant_rows_e4m3, quantized once; activations quantized in the call)."""
+    _on_cuda(x, W1q, w1_scales, W2q, w2_scales, seq_offsets, timestamps, pos_bias, time_bias, b1,
+             b2, ln_gamma, ln_beta)
+    T, D = x.shape
+    B = seq_offsets.numel() - 1
+    if x.dtype != torch.bfloat16 or not x.is_contiguous():
+        raise ValueError("x must be contiguous bf16")
+    for t in (W1q, W2q):
+        if t.dtype != torch.uint8 or not t.is_contiguous():
+            raise ValueError("W1q, W2q must be contiguous uint8 E4M3 codes")
+    if out is None:
+        out = torch.empty_like(x)
+    if workspace is None:
+        workspace = _workspace(hstu_layer_fp8_workspace_bytes(T, B, D, H, d, max_seqlen), x.device)
+    _native.check("hstu_layer_fp8_fwd", _lib().hstu_layer_fp8_fwd(
+        _ptr(x), T, D, _ptr(W1q), _ptr(w1_scales), _ptr(b1), _ptr(W2q), _ptr(w2_scales), _ptr(b2),
+        _ptr(ln_gamma), _ptr(ln_beta), float(ln_eps), _ptr(seq_offsets), B, H, d,
+        _ptr(timestamps), _ptr(pos_bias), 0 if pos_bias is None else pos_bias.shape[1],
+        _ptr(time_bias), 0 if time_bias is None else time_bias.shape[1], int(max_seqlen),
+        _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream)))
     return out

@@ -419,29 +419,49 @@ hstu_status_t run_linear(const void* x, int64_t ldx, int64_t M, int32_t K, const
                           ldr, y, ldy, stream);
 }
 
-hstu_status_t run_ln_gate(const void* a, int64_t lda, const void* u, int64_t ldu, int64_t M,
-                          int32_t F, const float* gamma, const float* beta, float eps, void* y,
-                          int64_t ldy, cudaStream_t stream) {
+// Y = LayerNorm(A) * U as bf16 (quant == false) or as row-wise E4M3 codes of
+// that bf16 result with row scales (quant == true)
+hstu_status_t run_ln_gate_any(bool quant, const void* a, int64_t lda, const void* u, int64_t ldu,
+                              int64_t M, int32_t F, const float* gamma, const float* beta,
+                              float eps, void* y, int64_t ldy, void* yq, int64_t ldyq, float* ys,
+                              cudaStream_t stream) {
     if (M < 0 || F < 1 || !(eps >= 0.0f)) return HSTU_ERR_INVALID_ARG;
     if (F % 256 || F > 2048) return HSTU_ERR_UNSUPPORTED;
     if (M == 0) return HSTU_OK;
-    if (!a || !u || !y) return HSTU_ERR_INVALID_ARG;
-    if (lda < F || ldu < F || ldy < F || lda % 8 || ldu % 8 || ldy % 8) return HSTU_ERR_INVALID_ARG;
-    if (!aligned16(a) || !aligned16(u) || !aligned16(y)) return HSTU_ERR_INVALID_ARG;
+    if (!a || !u || lda < F || ldu < F || lda % 8 || ldu % 8 || !aligned16(a) || !aligned16(u))
+        return HSTU_ERR_INVALID_ARG;
+    if (quant ? (!yq || !ys || ldyq < F || ldyq % 16 || !aligned16(yq))
+              : (!y || ldy < F || ldy % 8 || !aligned16(y)))
+        return HSTU_ERR_INVALID_ARG;
     LnGateArgs args{static_cast<const __nv_bfloat16*>(a), lda, static_cast<const __nv_bfloat16*>(u),
-                    ldu, M, gamma, beta, eps, static_cast<__nv_bfloat16*>(y), ldy};
+                    ldu, M, gamma, beta, eps, static_cast<__nv_bfloat16*>(y), ldy,
+                    static_cast<uint8_t*>(yq), ldyq, ys};
     const unsigned grid = static_cast<unsigned>((M + 7) / 8);
-    switch (F / 256) {
-        case 1: ln_gate_kernel<1><<<grid, 256, 0, stream>>>(args); break;
-        case 2: ln_gate_kernel<2><<<grid, 256, 0, stream>>>(args); break;
-        case 3: ln_gate_kernel<3><<<grid, 256, 0, stream>>>(args); break;
-        case 4: ln_gate_kernel<4><<<grid, 256, 0, stream>>>(args); break;
-        case 5: ln_gate_kernel<5><<<grid, 256, 0, stream>>>(args); break;
-        case 6: ln_gate_kernel<6><<<grid, 256, 0, stream>>>(args); break;
-        case 7: ln_gate_kernel<7><<<grid, 256, 0, stream>>>(args); break;
-        default: ln_gate_kernel<8><<<grid, 256, 0, stream>>>(args); break;
+#define HSTU_LN_CASES(Q)                                                       \
+    switch (F / 256) {                                                         \
+        case 1: ln_gate_kernel<1, Q><<<grid, 256, 0, stream>>>(args); break;   \
+        case 2: ln_gate_kernel<2, Q><<<grid, 256, 0, stream>>>(args); break;   \
+        case 3: ln_gate_kernel<3, Q><<<grid, 256, 0, stream>>>(args); break;   \
+        case 4: ln_gate_kernel<4, Q><<<grid, 256, 0, stream>>>(args); break;   \
+        case 5: ln_gate_kernel<5, Q><<<grid, 256, 0, stream>>>(args); break;   \
+        case 6: ln_gate_kernel<6, Q><<<grid, 256, 0, stream>>>(args); break;   \
+        case 7: ln_gate_kernel<7, Q><<<grid, 256, 0, stream>>>(args); break;   \
+        default: ln_gate_kernel<8, Q><<<grid, 256, 0, stream>>>(args); break;  \
     }
+    if (quant) {
+        HSTU_LN_CASES(true)
+    } else {
+        HSTU_LN_CASES(false)
+    }
+#undef HSTU_LN_CASES
     return launch_status();
+}
+
+hstu_status_t run_ln_gate(const void* a, int64_t lda, const void* u, int64_t ldu, int64_t M,
+                          int32_t F, const float* gamma, const float* beta, float eps, void* y,
+                          int64_t ldy, cudaStream_t stream) {
+    return run_ln_gate_any(false, a, lda, u, ldu, M, F, gamma, beta, eps, y, ldy, nullptr, 0,
+                           nullptr, stream);
 }
 
 struct LayerWs {
@@ -456,6 +476,26 @@ LayerWs layer_ws(int64_t T, int32_t B, int32_t H, int32_t d, int32_t max_seqlen)
     w.y = round_up(w.attn + static_cast<size_t>(T) * F * 2, 256);
     w.plan = round_up(w.y + static_cast<size_t>(T) * F * 2, 256);
     // window tables for any num_pos: at most one per 128-token diagonal offset
+    w.total = w.plan + hstu_attn_workspace_bytes(B, T, max_seqlen, H, 128 * max_tiles_of(max_seqlen));
+    return w;
+}
+
+// FP8 layer workspace: [x codes T x D][x scales][UVQK bf16][A bf16]
+// [Y codes T x F][Y scales][attention workspace]
+struct LayerFp8Ws {
+    size_t xq, sx, uvqk, attn, yq, sy, plan, total;
+};
+
+LayerFp8Ws layer_fp8_ws(int64_t T, int32_t B, int32_t D, int32_t H, int32_t d, int32_t max_seqlen) {
+    LayerFp8Ws w{};
+    const size_t F = static_cast<size_t>(H) * d, t = static_cast<size_t>(T);
+    w.xq = 0;
+    w.sx = round_up(w.xq + t * D, 256);
+    w.uvqk = round_up(w.sx + t * 4, 256);
+    w.attn = round_up(w.uvqk + t * 4 * F * 2, 256);
+    w.yq = round_up(w.attn + t * F * 2, 256);
+    w.sy = round_up(w.yq + t * F, 256);
+    w.plan = round_up(w.sy + t * 4, 256);
     w.total = w.plan + hstu_attn_workspace_bytes(B, T, max_seqlen, H, 128 * max_tiles_of(max_seqlen));
     return w;
 }
@@ -649,6 +689,72 @@ hstu_status_t hstu_layer_fwd(const void* x, int64_t total_tokens, int32_t D, con
     st = run_ln_gate(attn, F, uvqk, 4 * F, T, F, ln_gamma, ln_beta, ln_eps, ygate, F, s);
     if (st != HSTU_OK) return st;
     return run_linear(ygate, F, T, F, W2, F, D, b2, HSTU_EPI_RESIDUAL, x, D, out, D, s);
+}
+
+hstu_status_t hstu_layernorm_gate_fp8_fwd(const void* a, int64_t lda, const void* u, int64_t ldu,
+                                          int64_t M, int32_t F, const float* gamma,
+                                          const float* beta, float eps, void* codes,
+                                          int64_t ldq, float* scales, void* stream) {
+    return run_ln_gate_any(true, a, lda, u, ldu, M, F, gamma, beta, eps, nullptr, 0, codes, ldq,
+                           scales, as_stream(stream));
+}
+
+size_t hstu_layer_fp8_workspace_bytes(int64_t total_tokens, int32_t B, int32_t D, int32_t H,
+                                      int32_t d, int32_t max_seqlen) {
+    if (total_tokens < 0 || D < 1 || H < 1 || d < 1 || !plan_sizes_ok(B, total_tokens, max_seqlen))
+        return 0;
+    return layer_fp8_ws(total_tokens, B, D, H, d, max_seqlen).total;
+}
+
+hstu_status_t hstu_layer_fp8_fwd(const void* x, int64_t total_tokens, int32_t D, const void* W1q,
+                                 const float* w1_scales, const float* b1, const void* W2q,
+                                 const float* w2_scales, const float* b2, const float* ln_gamma,
+                                 const float* ln_beta, float ln_eps, const int64_t* seq_offsets,
+                                 int32_t B, int32_t H, int32_t d, const int64_t* timestamps,
+                                 const float* pos_bias, int32_t num_pos, const float* time_bias,
+                                 int32_t num_time_buckets, int32_t max_seqlen, void* out,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+    const int64_t T = total_tokens;
+    if (T < 0 || D < 1 || H < 1 || d < 1 || !plan_sizes_ok(B, T, max_seqlen))
+        return HSTU_ERR_INVALID_ARG;
+    const int32_t F = H * d;
+    if (D % 128 || (d != 64 && d != 128) || F % 256 || F > 2048) return HSTU_ERR_UNSUPPORTED;
+    if (T == 0 || B == 0) return HSTU_OK;
+    if (!x || !W1q || !w1_scales || !W2q || !w2_scales || !out || !seq_offsets || !workspace)
+        return HSTU_ERR_INVALID_ARG;
+    const LayerFp8Ws w = layer_fp8_ws(T, B, D, H, d, max_seqlen);
+    if (workspace_bytes < w.total || !aligned16(workspace)) return HSTU_ERR_INVALID_ARG;
+    cudaStream_t s = as_stream(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    uint8_t* xq = ws + w.xq;
+    float* sx = reinterpret_cast<float*>(ws + w.sx);
+    __nv_bfloat16* uvqk = reinterpret_cast<__nv_bfloat16*>(ws + w.uvqk);
+    __nv_bfloat16* attn = reinterpret_cast<__nv_bfloat16*>(ws + w.attn);
+    uint8_t* yq = ws + w.yq;
+    float* sy = reinterpret_cast<float*>(ws + w.sy);
+    void* plan_ws = ws + w.plan;
+    const size_t plan_bytes = workspace_bytes - w.plan;
+    // 1. x -> E4M3 rows, f1 in FP8 with the SiLU epilogue
+    hstu_status_t st = hstu_quant_rows_e4m3(x, D, T, D, xq, D, sx, stream);
+    if (st != HSTU_OK) return st;
+    st = run_linear_any(true, xq, D, sx, T, D, W1q, D, w1_scales, 4 * F, b1, HSTU_EPI_SILU,
+                        nullptr, 0, uvqk, 4 * F, s);
+    if (st != HSTU_OK) return st;
+    // 2. attention (bf16)
+    st = plan_attn(seq_offsets, B, T, max_seqlen, plan_ws, plan_bytes, s);
+    if (st != HSTU_OK) return st;
+    AttnCall c{HSTU_DTYPE_BF16, uvqk + 2 * F, uvqk + 3 * F, uvqk + F, 4 * F, 4 * F, 4 * F,
+               seq_offsets, B, T, H, d, d, timestamps, pos_bias, num_pos, time_bias,
+               num_time_buckets, max_seqlen, attn, F, plan_ws, plan_bytes, s};
+    st = run_attn(c);
+    if (st != HSTU_OK) return st;
+    // 3. LayerNorm gate quantized to E4M3 rows in the same kernel
+    st = run_ln_gate_any(true, attn, F, uvqk, 4 * F, T, F, ln_gamma, ln_beta, ln_eps, nullptr, 0,
+                         yq, F, sy, s);
+    if (st != HSTU_OK) return st;
+    // 4. f2 in FP8 with the residual
+    return run_linear_any(true, yq, F, sy, T, F, W2q, F, w2_scales, D, b2, HSTU_EPI_RESIDUAL, x,
+                          D, out, D, s);
 }
 
 }  // extern "C"

@@ -3,11 +3,16 @@
 // Each lane holds 8 contiguous features per 256-feature block (16-byte
 // loads). Mean first, then the biased variance of the centred values (two
 // passes over registers, so no cancellation), rsqrt(var + eps), affine, gate.
+// With QUANT the bf16 result row is not stored but quantized row-wise to
+// E4M3 (exactly as quant_rows_e4m3_kernel would quantize it), the fused
+// output-normalization-to-FP8 step of the FP8 projections
+// (generative-recommenders README, "FP8 linear reference and benchmark").
 #pragma once
 
 #include <cuda_bf16.h>
 
 #include "common.cuh"
+#include "quant_fp8.cuh"
 
 namespace hstu {
 
@@ -22,6 +27,9 @@ struct LnGateArgs {
     float eps;
     __nv_bfloat16* y;
     int64_t ldy;
+    uint8_t* yq;        // QUANT: E4M3 codes [M, F] (row stride ldyq) and row scales
+    int64_t ldyq;
+    float* ys;
 };
 
 __device__ __forceinline__ void unpack8(const uint4 w, float (&f)[8]) {
@@ -33,7 +41,7 @@ __device__ __forceinline__ void unpack8(const uint4 w, float (&f)[8]) {
     }
 }
 
-template <int NV>   // F = 256 * NV features
+template <int NV, bool QUANT = false>   // F = 256 * NV features
 __global__ void __launch_bounds__(256) ln_gate_kernel(const LnGateArgs a) {
     constexpr int F = 256 * NV;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -62,6 +70,7 @@ __global__ void __launch_bounds__(256) ln_gate_kernel(const LnGateArgs a) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
     const float rstd = rsqrtf(sq * (1.0f / F) + a.eps);
+    uint4 yrow[QUANT ? NV : 1];     // QUANT: the row's bf16 results, for the row amax
 #pragma unroll
     for (int k = 0; k < NV; ++k) {
         const int col = k * 256 + lane * 8;
@@ -82,7 +91,21 @@ __global__ void __launch_bounds__(256) ln_gate_kernel(const LnGateArgs a) {
             __nv_bfloat162 v2 = __floats2bfloat162_rn(y0, y1);
             out[q] = *reinterpret_cast<uint32_t*>(&v2);
         }
-        *reinterpret_cast<uint4*>(a.y + m * a.ldy + col) = make_uint4(out[0], out[1], out[2], out[3]);
+        if (QUANT) yrow[QUANT ? k : 0] = make_uint4(out[0], out[1], out[2], out[3]);
+        else *reinterpret_cast<uint4*>(a.y + m * a.ldy + col) = make_uint4(out[0], out[1], out[2], out[3]);
+    }
+    if (QUANT) {
+        uint32_t amax_bits = 0u;
+#pragma unroll
+        for (int k = 0; k < NV; ++k) amax_bits = amax_bits8(yrow[QUANT ? k : 0], amax_bits);
+        amax_bits = __reduce_max_sync(0xffffffffu, amax_bits);
+        const float amax = __uint_as_float(amax_bits);
+        const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 0.f;
+#pragma unroll
+        for (int k = 0; k < NV; ++k)
+            *reinterpret_cast<uint2*>(a.yq + m * a.ldyq + k * 256 + lane * 8) =
+                e4m3_codes8(yrow[QUANT ? k : 0], inv);
+        if (lane == 0) a.ys[m] = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
     }
 }
 
