@@ -292,8 +292,10 @@ def bench_attention(args, rank, world, local, peaks, peak_kind):
     kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
     torch.cuda.synchronize(dev)
+    spin = getattr(torch.cuda, "_sleep", None)
     for i in range(args.steps):
-        torch.cuda._sleep(100000)
+        if spin is not None:
+            spin(100000)
         step(i, kev[i])
     torch.cuda.synchronize(dev)
     kernel_ms = [a.elapsed_time(b) for a, b in kev]
