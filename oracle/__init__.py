@@ -68,6 +68,11 @@ def _bind(lib):
     lib.hstu_oracle_quant_rows_e4m3.argtypes = [_i64, _i32, _p, _p, _p]
     lib.hstu_oracle_linear_fp8.restype = None
     lib.hstu_oracle_linear_fp8.argtypes = [_i64, _i32, _i32, _p, _p, _p, _p, _p, _i32, _p, _p]
+    lib.hstu_oracle_silu_grad.restype = _f64
+    lib.hstu_oracle_silu_grad.argtypes = [_f64]
+    lib.hstu_oracle_attn_bwd.restype = None
+    lib.hstu_oracle_attn_bwd.argtypes = [_p, _i32, _i32, _i32, _i32, _p, _p, _p, _p, _p, _i32,
+                                         _p, _i32, _i32, _p, _p, _p, _p, _p, _p]
     lib.hstu_oracle_num_threads.restype = ctypes.c_int
     lib.hstu_oracle_num_threads.argtypes = []
     return lib
@@ -164,6 +169,29 @@ def linear(x, W, bias=None, act_silu: bool = False, residual=None, lib=None) -> 
     lib.hstu_oracle_linear(M, K, N, _ptr(x), _ptr(W), _ptr(bias), int(bool(act_silu)),
                            _ptr(residual), _ptr(y))
     return y[:M]
+
+
+def attn_bwd(seq_offsets, q, k, v, timestamps, pos_bias, time_bias, max_seqlen: int, dout,
+             lib=None):
+    """Gradients of attn() for the upstream gradient dout, fp64:
+    (dq, dk, dv, dpos, dtime); dpos / dtime are None when the term is absent."""
+    lib = lib or load()
+    off = _i64a(seq_offsets)
+    q, k, v, dout = (np.ascontiguousarray(a, dtype=np.float64) for a in (q, k, v, dout))
+    T, H, dqk = q.shape
+    dv = v.shape[2]
+    pos, tb, ts = _f64a(pos_bias), _f64a(time_bias), _i64a(timestamps)
+    P = 0 if pos is None else pos.shape[1]
+    NB = 0 if tb is None else tb.shape[1]
+    dq = np.zeros((max(T, 1), H, dqk))
+    dk = np.zeros((max(T, 1), H, dqk))
+    dvv = np.zeros((max(T, 1), H, dv))
+    dpos = None if pos is None else np.zeros((H, P))
+    dtime = None if (tb is None or ts is None) else np.zeros((H, NB))
+    lib.hstu_oracle_attn_bwd(_ptr(off), len(off) - 1, H, dqk, dv, _ptr(q), _ptr(k), _ptr(v),
+                             _ptr(ts), _ptr(pos), P, _ptr(tb), NB, int(max_seqlen), _ptr(dout),
+                             _ptr(dq), _ptr(dk), _ptr(dvv), _ptr(dpos), _ptr(dtime))
+    return dq[:T], dk[:T], dvv[:T], dpos, dtime
 
 
 def e4m3_to_float(codes, lib=None) -> np.ndarray:

@@ -142,6 +142,77 @@ int hstu_oracle_attn(const int64_t* seq_offsets, int32_t B, int32_t H, int32_t d
     return bad ? -1 : 0;
 }
 
+/* ---------------------------------------------------------------- backward
+ * Gradients of the attention forward above for an upstream gradient dout
+ * [T,H,dv] (the chain rule through s = q.k + pos + time, p = silu(s) / N,
+ * out = sum p v; the pages' reference implementation has forward and
+ * backward attention kernels, generative-recommenders README, section "HSTU
+ * Ultra attention benchmark"):
+ *   dv[j]  = sum_{i>=j} p_ij dout[i]
+ *   ds_ij  = (dout[i] . v[j]) silu'(s_ij) / N,
+ *            silu'(s) = sig(s) (1 + s (1 - sig(s))), sig(s) = 1 / (1 + e^-s)
+ *   dq[i]  = sum_{j<=i} ds_ij k[j],   dk[j] = sum_{i>=j} ds_ij q[i]
+ *   dpos[h][r] = sum of ds_ij over pairs with min(i-j, P-1) = r
+ *   dtime[h][b] = sum of ds_ij over pairs with bucket(t_i - t_j) = b
+ * All arrays contiguous: q,k,dq,dk [T,H,dqk], v,dout,dv [T,H,dv], dpos [H,P],
+ * dtime [H,NB] (each may be NULL when its term is absent). Outputs are
+ * overwritten. Serial over pairs (the accumulation targets are shared). */
+double hstu_oracle_silu_grad(double s) {
+    const double sg = 1.0 / (1.0 + exp(-s));
+    return sg * (1.0 + s * (1.0 - sg));
+}
+
+void hstu_oracle_attn_bwd(const int64_t* seq_offsets, int32_t B, int32_t H, int32_t dqk,
+                          int32_t dv, const double* q, const double* k, const double* v,
+                          const int64_t* ts, const double* pos, int32_t num_pos,
+                          const double* tbias, int32_t num_buckets, int32_t max_seqlen,
+                          const double* dout, double* dq, double* dk, double* dvv,
+                          double* dpos, double* dtime) {
+    const int64_t T = seq_offsets[B];
+    for (int64_t e = 0; e < T * H * dqk; ++e) dq[e] = dk[e] = 0.0;
+    for (int64_t e = 0; e < T * H * dv; ++e) dvv[e] = 0.0;
+    if (dpos) for (int64_t e = 0; e < (int64_t)H * num_pos; ++e) dpos[e] = 0.0;
+    if (dtime) for (int64_t e = 0; e < (int64_t)H * num_buckets; ++e) dtime[e] = 0.0;
+    const double inv_n = 1.0 / (double)max_seqlen;
+    for (int32_t b = 0; b < B; ++b) {
+        const int64_t o = seq_offsets[b], n = seq_offsets[b + 1] - o;
+        for (int32_t h = 0; h < H; ++h) {
+            for (int64_t i = 0; i < n; ++i) {
+                const double* qi = q + ((o + i) * H + h) * dqk;
+                const double* gi = dout + ((o + i) * H + h) * dv;
+                for (int64_t j = 0; j <= i; ++j) {
+                    const double* kj = k + ((o + j) * H + h) * dqk;
+                    const double* vj = v + ((o + j) * H + h) * dv;
+                    double s = 0.0;
+                    for (int32_t c = 0; c < dqk; ++c) s += qi[c] * kj[c];
+                    int32_t pidx = -1, bkt = -1;
+                    if (pos) {
+                        pidx = hstu_oracle_pos_index(i, j, num_pos);
+                        s += pos[(int64_t)h * num_pos + pidx];
+                    }
+                    if (ts && tbias) {
+                        bkt = hstu_oracle_time_bucket(ts[o + i] - ts[o + j], num_buckets);
+                        s += tbias[(int64_t)h * num_buckets + bkt];
+                    }
+                    const double p = hstu_oracle_silu(s) * inv_n;
+                    double dp = 0.0;
+                    for (int32_t c = 0; c < dv; ++c) {
+                        dvv[((o + j) * H + h) * dv + c] += p * gi[c];
+                        dp += gi[c] * vj[c];
+                    }
+                    const double ds = dp * hstu_oracle_silu_grad(s) * inv_n;
+                    for (int32_t c = 0; c < dqk; ++c) {
+                        dq[((o + i) * H + h) * dqk + c] += ds * kj[c];
+                        dk[((o + j) * H + h) * dqk + c] += ds * qi[c];
+                    }
+                    if (dpos && pidx >= 0) dpos[(int64_t)h * num_pos + pidx] += ds;
+                    if (dtime && bkt >= 0) dtime[(int64_t)h * num_buckets + bkt] += ds;
+                }
+            }
+        }
+    }
+}
+
 /* y[m, :] = act(x[m, :] W^T + bias) + residual[m, :]; x [M,K], W [N,K].
  * act = 1 applies SiLU. bias / residual may be NULL. */
 void hstu_oracle_linear(int64_t M, int32_t K, int32_t N, const double* x, const double* W,

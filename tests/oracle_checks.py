@@ -419,6 +419,83 @@ def check_layer_identities(lib):
     _close(out, x, 0.0, "U = 0 must give out = x")
 
 
+# --------------------------------------------------------------------------- backward
+
+def check_silu_grad(lib):
+    """silu'(s) against torch autograd of torch's SiLU (a library routine)."""
+    xs = np.array([-30.0, -5.0, -1.3, -1e-3, 0.0, 2e-4, 0.7, 3.0, 12.0, 40.0])
+    t = torch.from_numpy(xs).requires_grad_(True)
+    torch.nn.functional.silu(t).sum().backward()
+    got = np.array([lib.hstu_oracle_silu_grad(float(x)) for x in xs])
+    _close(got, t.grad.numpy(), what="silu'")
+
+
+def _loss(lib, inp, dout, **kw):
+    return float(np.sum(_run(lib, inp, **kw) * dout))
+
+
+def check_attn_bwd_finite_differences(lib):
+    """Every gradient against central differences of <dout, attn(...)> in fp64
+    on a tiny ragged batch: sampled entries of q, k, v, every entry of the
+    position and time tables."""
+    inp = tiny_case(seed=3, lengths=(0, 1, 6, 11, 3), H=2, d=4, P=6, NB=9)
+    rng = np.random.default_rng(5)
+    dout = rng.standard_normal(inp.v.shape)
+    dq, dk, dv, dpos, dtime = oracle.attn_bwd(inp.seq_offsets, inp.q, inp.k, inp.v,
+                                              inp.timestamps, inp.pos_bias, inp.time_bias,
+                                              inp.max_seqlen, dout, lib=lib)
+    eps = 1e-6
+    base = dict(q=inp.q.astype(np.float64), k=inp.k.astype(np.float64),
+                v=inp.v.astype(np.float64), pos_bias=inp.pos_bias.astype(np.float64),
+                time_bias=inp.time_bias.astype(np.float64))
+    grads = dict(q=dq, k=dk, v=dv, pos_bias=dpos, time_bias=dtime)
+    for name, arr in base.items():
+        idx = [tuple(int(rng.integers(0, n)) for n in arr.shape) for _ in range(12)]
+        if name in ("pos_bias", "time_bias"):
+            idx = list(np.ndindex(*arr.shape))
+        for ix in idx:
+            plus, minus = arr.copy(), arr.copy()
+            plus[ix] += eps
+            minus[ix] -= eps
+            fd = (_loss(lib, inp, dout, **{name: plus}) - _loss(lib, inp, dout, **{name: minus})) \
+                / (2 * eps)
+            g = grads[name][ix]
+            assert abs(fd - g) <= 1e-6 * max(1.0, abs(fd)), "%s%s: fd %.9g grad %.9g" % (
+                name, ix, fd, g)
+
+
+def check_attn_bwd_closed_form(lib):
+    """q = k = 0 and constant biases c: every score is c, so dv[j] = silu(c)/N
+    times the suffix sum of dout over the rows i >= j of j's sequence, and the
+    position- and time-table gradients each sum to sum_{i>=j} (dout_i . v_j)
+    silu'(c) / N."""
+    inp = tiny_case(seed=4, lengths=(5, 0, 8, 1), H=1, d=3, P=4, NB=6)
+    c = 0.4
+    q0 = np.zeros_like(inp.q, dtype=np.float64)
+    pos = np.full_like(inp.pos_bias, c / 2, dtype=np.float64)
+    tb = np.full_like(inp.time_bias, c / 2, dtype=np.float64)
+    rng = np.random.default_rng(8)
+    dout = rng.standard_normal(inp.v.shape)
+    v = inp.v.astype(np.float64)
+    N = inp.max_seqlen
+    _, _, dv, dpos, dtime = oracle.attn_bwd(inp.seq_offsets, q0, q0, v, inp.timestamps, pos, tb,
+                                            N, dout, lib=lib)
+    sil = c / (1 + np.exp(-c))
+    sg = 1 / (1 + np.exp(-c))
+    dsil = sg * (1 + c * (1 - sg))
+    want_dv = np.zeros_like(v)
+    total = 0.0
+    off = inp.seq_offsets
+    for b in range(len(off) - 1):
+        for j in range(off[b], off[b + 1]):
+            want_dv[j] = sil / N * dout[j:off[b + 1]].sum(axis=0)
+            for i in range(j, off[b + 1]):
+                total += float(np.sum(dout[i] * v[j])) * dsil / N
+    _close(dv, want_dv, what="dv suffix sums")
+    _close(dpos.sum(), total, what="sum dpos")
+    _close(dtime.sum(), total, what="sum dtime")
+
+
 # --------------------------------------------------------------------------- FP8 (E4M3)
 
 def _e4m3_grid():
@@ -531,4 +608,5 @@ ALL_CHECKS = [
     check_scale_is_max_seqlen, check_qk_asymmetry, check_linear, check_layernorm_gate,
     check_layer_composition, check_layer_identities, check_e4m3_table,
     check_e4m3_rounding_against_torch, check_e4m3_saturation, check_quant_rows, check_linear_fp8,
+    check_silu_grad, check_attn_bwd_finite_differences, check_attn_bwd_closed_form,
 ]

@@ -60,6 +60,13 @@ MUTANTS = [
     ("quant_scale_not_amax", "if (v > amax) amax = v;", "if (v > amax) amax = v * 0.5f;"),
     ("fp8_scale_inverted", "acc *= (double)sx[m] * (double)sw[n];",
      "acc *= (double)sx[m] / (double)sw[n];"),
+    ("bwd_silu_grad_is_sigmoid", "return sg * (1.0 + s * (1.0 - sg));", "return sg;"),
+    ("bwd_dk_uses_k", "dk[((o + j) * H + h) * dqk + c] += ds * qi[c];",
+     "dk[((o + j) * H + h) * dqk + c] += ds * kj[c];"),
+    ("bwd_ds_missing_1_over_N", "const double ds = dp * hstu_oracle_silu_grad(s) * inv_n;",
+     "const double ds = dp * hstu_oracle_silu_grad(s);"),
+    ("bwd_dtime_dropped", "if (dtime && bkt >= 0) dtime[(int64_t)h * num_buckets + bkt] += ds;",
+     ""),
 ]
 
 
