@@ -623,6 +623,67 @@ def e2e_layer(args, li, dev, stream, flops, world, hstu, ws):
                         "i-2's device-to-host copy (three streams, two buffer sets)"}
 
 
+def bench_backward(args, rank, world, local, peaks, peak_kind):
+    """The fp32 attention backward on the --config workload (its lengths,
+    heads, head dimension and bias tables, inputs in fp32). Algorithmic FLOPs:
+    the four contractions dV = P^T dO, dP = dO V^T, dQ = dS K, dK = dS^T Q over
+    the causal pairs, twice the forward's. The kernels run on CUDA cores, so
+    the roofline is fp32 FMA: SMs x 128 lanes x 2 FLOP x the max SM clock."""
+    import torch
+    import jagged_pointwise_attention_b200 as hstu
+    from gen import CONFIGS, make_attn_inputs
+    cfg = CONFIGS[args.config]
+    if cfg["kind"] == "layer":
+        raise SystemExit("--backward takes an attention workload (--config 2, 3 or 4)")
+    inp = make_attn_inputs(args.config, seed=1000 + args.config + 7919 * rank)
+    dev = torch.device("cuda", local)
+    f32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(dev)  # noqa: E731
+    i64 = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)  # noqa: E731
+    q, k, v = f32(inp.q), f32(inp.k), f32(inp.v)
+    dout = torch.randn(v.shape, generator=torch.Generator().manual_seed(7), dtype=torch.float32).to(dev)
+    off, ts, pos, tb = i64(inp.seq_offsets), i64(inp.timestamps), f32(inp.pos_bias), f32(inp.time_bias)
+    lengths = np.diff(inp.seq_offsets)
+    flops = 2 * causal_flops(lengths, inp.H, inp.q.shape[2], inp.v.shape[2])
+
+    def step():
+        hstu.hstu_attn_bwd_f32(q, k, v, dout, off, ts, pos, tb, inp.max_seqlen)
+
+    for _ in range(args.warmup):
+        step()
+    assert hstu.hstu_device_status() == 0
+    sampler = ClockSampler(local)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _barrier(world)
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize(dev)
+    sampler.stop()
+    _barrier(world)
+    max_ms, tot = reduce_timing(e0.elapsed_time(e1), float(flops) * args.steps, world, dev)
+    value = tot / (max_ms * 1e-3) / 1e12
+    clocks = sampler.summary()
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    peak = sms * 128 * 2 * (clocks.get("sm_max_mhz") or 1965) * 1e6 / 1e12
+    return {"metric": "HSTU jagged attn bwd TFLOP/s (causal, fp32 CUDA cores)",
+            "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(max_ms / args.steps, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded generator; no dataset)",
+            "config": {"workload": cfg["name"] + "_backward_f32", "B": inp.B, "H": inp.H,
+                       "d": int(inp.q.shape[2]), "total_tokens": inp.T,
+                       "parallelism": "dp%d" % world},
+            "roofline": {"bound": "alu", "achieved": round(value, 3), "peak": round(peak, 1),
+                         "unit": "TFLOP/s", "frac": round(value / peak, 4),
+                         "peak_kind": "fp32 FMA: %d SMs x 128 lanes x 2 x max SM clock" % sms,
+                         "traffic": None,
+                         "kernel": "attn_bwd_q_kernel + attn_bwd_kv_kernel"},
+            "gpu_launches": 2 * args.steps, "clocks": clocks}
+
+
 def bench_fp8_linear(args, rank, world, local, peaks, peak_kind):
     """Row-wise E4M3 projections against bf16 ones on the layer's f1 shape
     (79,913 x 512 -> 2048, SiLU) and the FP8 benchmark shape of the
@@ -754,6 +815,9 @@ def parse_args(argv=None):
     ap.add_argument("--fp8", action="store_true",
                     help="with --config 5: the layer with both projections in FP8 "
                          "(hstu_layer_fp8_fwd, weights quantized once)")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the fp32 attention backward (hstu_attn_bwd_f32) on the "
+                         "--config workload's shapes instead of the forward")
     ap.add_argument("--fp8-linear", action="store_true",
                     help="time the row-wise E4M3 projections (quantize + FP8 GEMM) against the "
                          "bf16 ones on the projection shapes instead of the attention")
@@ -783,7 +847,9 @@ def main(argv=None):
                                 device_id=torch.device("cuda", local))
     peaks, kind = load_peaks()
     from gen import CONFIGS
-    if args.fp8_linear:
+    if args.backward:
+        line = bench_backward(args, rank, world, local, peaks, kind)
+    elif args.fp8_linear:
         line = bench_fp8_linear(args, rank, world, local, peaks, kind)
     elif CONFIGS[args.config]["kind"] == "layer":
         line = bench_layer(args, rank, world, local, peaks, kind)

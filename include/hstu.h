@@ -203,6 +203,29 @@ hstu_status_t hstu_debug_wait_timeout(int32_t wait_us, void* stream);
 
 /* ---------------------------------------------------------------- layer */
 
+/* ---------------------------------------------------------------- backward */
+
+/* Gradients of the attention (fp32 path, CUDA cores; the pages' reference
+ * implementation has forward and backward attention kernels,
+ * generative-recommenders README, "HSTU Ultra attention benchmark") for an
+ * upstream gradient dout of hstu_attn_fwd's output. With s_ij = q_i.k_j +
+ * pos + time, p_ij = silu(s_ij)/N:
+ *   dv_j = sum_{i>=j} p_ij dout_i;  ds_ij = (dout_i.v_j) silu'(s_ij) / N
+ *   dq_i = sum_{j<=i} ds_ij k_j;    dk_j = sum_{i>=j} ds_ij q_i
+ *   dpos[h][min(i-j, P-1)] and dtime[h][bucket] sum the ds_ij of their pairs.
+ * q, k, dq, dk: device fp32 [T, H, d_qk] contiguous; v, dout, dv: [T, H,
+ * d_v]; dpos [H, num_pos] required when pos_bias is given, dtime [H,
+ * num_time_buckets] when timestamps and time_bias are (both overwritten);
+ * d_qk, d_v <= 128; num_pos + num_time_buckets <= 12288. Other arguments as
+ * hstu_attn_run. Two kernel launches (a query pass and a key pass) plus the
+ * table clears. */
+hstu_status_t hstu_attn_bwd_f32(const float* q, const float* k, const float* v, const float* dout,
+                                const int64_t* seq_offsets, int32_t B, int64_t total_tokens,
+                                int32_t H, int32_t d_qk, int32_t d_v, const int64_t* timestamps,
+                                const float* pos_bias, int32_t num_pos, const float* time_bias,
+                                int32_t num_time_buckets, int32_t max_seqlen, float* dq, float* dk,
+                                float* dv, float* dpos, float* dtime, void* stream);
+
 /* ---------------------------------------------------------------- FP8 projections */
 
 /* Row-wise E4M3 quantization (generative-recommenders README, "FP8 linear

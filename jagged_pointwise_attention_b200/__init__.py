@@ -25,7 +25,8 @@ __all__ = [
     "hstu_attn_fwd", "hstu_attn_plan", "hstu_attn_run", "hstu_attn_workspace_bytes",
     "hstu_layer_fwd", "hstu_layer_workspace_bytes", "hstu_linear_fwd",
     "hstu_layernorm_gate_fwd", "hstu_debug_bias_indices", "hstu_debug_wait_timeout",
-    "hstu_quant_rows_e4m3", "hstu_linear_fp8_fwd", "hstu_layernorm_gate_fp8_fwd",
+    "hstu_attn_bwd_f32", "hstu_quant_rows_e4m3", "hstu_linear_fp8_fwd",
+    "hstu_layernorm_gate_fp8_fwd",
     "hstu_layer_fp8_workspace_bytes", "hstu_layer_fp8_fwd",
     "hstu_device_status", "HstuError", "library_path",
 ]
@@ -330,3 +331,28 @@ def hstu_layer_fp8_fwd(x: torch.Tensor, W1q: torch.Tensor, w1_scales: torch.Tens
         _ptr(time_bias), 0 if time_bias is None else time_bias.shape[1], int(max_seqlen),
         _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream)))
     return out
+
+
+def hstu_attn_bwd_f32(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dout: torch.Tensor,
+                      seq_offsets: torch.Tensor, timestamps: Optional[torch.Tensor],
+                      pos_bias: Optional[torch.Tensor], time_bias: Optional[torch.Tensor],
+                      max_seqlen: int, stream=None):
+    """Gradients of the attention for the upstream gradient dout (fp32):
+    (dq, dk, dv, dpos, dtime); dpos / dtime are None when the term is absent."""
+    _on_cuda(q, k, v, dout, seq_offsets, timestamps, pos_bias, time_bias)
+    for t in (q, k, v, dout):
+        if t.dtype != torch.float32 or not t.is_contiguous():
+            raise ValueError("q, k, v, dout must be contiguous fp32")
+    T, H, dqk = q.shape
+    dvd = v.shape[2]
+    B = seq_offsets.numel() - 1
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dpos = None if pos_bias is None else torch.empty_like(pos_bias)
+    use_time = timestamps is not None and time_bias is not None
+    dtime = torch.empty_like(time_bias) if use_time else None
+    _native.check("hstu_attn_bwd_f32", _lib().hstu_attn_bwd_f32(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(seq_offsets), B, T, H, dqk, dvd,
+        _ptr(timestamps), _ptr(pos_bias), 0 if pos_bias is None else pos_bias.shape[1],
+        _ptr(time_bias), 0 if time_bias is None else time_bias.shape[1], int(max_seqlen),
+        _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dpos), _ptr(dtime), _stream(stream)))
+    return dq, dk, dv, dpos, dtime

@@ -33,6 +33,9 @@ SIGNATURES = {
     "hstu_debug_wait_timeout": (ctypes.c_int, [c_i32, c_p]),
     "hstu_linear_fwd": (ctypes.c_int, [c_p, c_i64, c_i64, c_i32, c_p, c_i64, c_i32, c_p,
                                        ctypes.c_int, c_p, c_i64, c_p, c_i64, c_p]),
+    "hstu_attn_bwd_f32": (ctypes.c_int, [c_p, c_p, c_p, c_p, c_p, c_i32, c_i64, c_i32, c_i32,
+                                         c_i32, c_p, c_p, c_i32, c_p, c_i32, c_i32, c_p, c_p, c_p,
+                                         c_p, c_p, c_p]),
     "hstu_quant_rows_e4m3": (ctypes.c_int, [c_p, c_i64, c_i64, c_i32, c_p, c_i64, c_p, c_p]),
     "hstu_linear_fp8_fwd": (ctypes.c_int, [c_p, c_i64, c_p, c_i64, c_i32, c_p, c_i64, c_p, c_i32,
                                            c_p, ctypes.c_int, c_p, c_i64, c_p, c_i64, c_p]),

@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "hstu.h"
+#include "attn_bwd_simt.cuh"
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
 #include "bias_prep.cuh"
@@ -613,6 +614,50 @@ hstu_status_t hstu_linear_fwd(const void* x, int64_t ldx, int64_t M, int32_t K, 
                               void* stream) {
     return run_linear(x, ldx, M, K, W, ldw, N, bias, epilogue, residual, ldr, y, ldy,
                       as_stream(stream));
+}
+
+hstu_status_t hstu_attn_bwd_f32(const float* q, const float* k, const float* v, const float* dout,
+                                const int64_t* seq_offsets, int32_t B, int64_t total_tokens,
+                                int32_t H, int32_t d_qk, int32_t d_v, const int64_t* timestamps,
+                                const float* pos_bias, int32_t num_pos, const float* time_bias,
+                                int32_t num_time_buckets, int32_t max_seqlen, float* dq, float* dk,
+                                float* dv, float* dpos, float* dtime, void* stream) {
+    if (!plan_sizes_ok(B, total_tokens, max_seqlen) || H < 1 || d_qk < 1 || d_v < 1)
+        return HSTU_ERR_INVALID_ARG;
+    if (d_qk > 128 || d_v > 128 || H > 65535) return HSTU_ERR_UNSUPPORTED;
+    if (pos_bias && num_pos < 1) return HSTU_ERR_INVALID_ARG;
+    const bool use_time = timestamps && time_bias;
+    if (use_time && (num_time_buckets < 1 || num_time_buckets > kMaxTimeBuckets))
+        return HSTU_ERR_INVALID_ARG;
+    if ((pos_bias && !dpos) || (use_time && !dtime)) return HSTU_ERR_INVALID_ARG;
+    if (B == 0 || total_tokens == 0) return HSTU_OK;
+    if (!q || !k || !v || !dout || !seq_offsets || !dq || !dk || !dv) return HSTU_ERR_INVALID_ARG;
+    cudaStream_t s = as_stream(stream);
+    const int P = pos_bias ? num_pos : 0, NB = use_time ? num_time_buckets : 0;
+    const size_t tab_bytes = static_cast<size_t>(P + NB) * sizeof(float);
+    if (tab_bytes > 48 * 1024) return HSTU_ERR_UNSUPPORTED;     // shared-memory table partials
+    if (pos_bias && cudaMemsetAsync(dpos, 0, static_cast<size_t>(H) * P * sizeof(float), s) != cudaSuccess)
+        return HSTU_ERR_CUDA;
+    if (use_time &&
+        cudaMemsetAsync(dtime, 0, static_cast<size_t>(H) * NB * sizeof(float), s) != cudaSuccess)
+        return HSTU_ERR_CUDA;
+    AttnBwdArgs a{q, k, v, dout, seq_offsets, B, total_tokens, H, d_qk, d_v,
+                  use_time ? timestamps : nullptr, pos_bias, P, use_time ? time_bias : nullptr, NB,
+                  1.0f / static_cast<float>(max_seqlen), dq, dk, dv,
+                  pos_bias ? dpos : nullptr, use_time ? dtime : nullptr};
+    const dim3 grid(static_cast<unsigned>((total_tokens + 127) / 128), static_cast<unsigned>(H));
+    const int dmax = d_qk > d_v ? d_qk : d_v;
+    if (dmax <= 32) {
+        attn_bwd_q_kernel<32><<<grid, 128, tab_bytes, s>>>(a);
+        attn_bwd_kv_kernel<32><<<grid, 128, 0, s>>>(a);
+    } else if (dmax <= 64) {
+        attn_bwd_q_kernel<64><<<grid, 128, tab_bytes, s>>>(a);
+        attn_bwd_kv_kernel<64><<<grid, 128, 0, s>>>(a);
+    } else {
+        attn_bwd_q_kernel<128><<<grid, 128, tab_bytes, s>>>(a);
+        attn_bwd_kv_kernel<128><<<grid, 128, 0, s>>>(a);
+    }
+    return launch_status();
 }
 
 hstu_status_t hstu_quant_rows_e4m3(const void* x, int64_t ldx, int64_t M, int32_t K, void* codes,
