@@ -7,8 +7,9 @@
 //   dq_i = sum_{j<=i} ds_ij k_j                      (query pass)
 //   dk_j = sum_{i>=j} ds_ij q_i, dv_j = sum_{i>=j} p_ij dout_i   (key pass)
 //   dpos[h][min(i-j, P-1)] += ds_ij, dtime[h][bucket] += ds_ij   (query pass)
-// Two passes, one thread per (token, head) each, scores recomputed in both,
-// so no gradient of q, k or v needs an atomic; the table gradients collect in
+// Two passes, one warp per (token, head) each (lanes split the head
+// dimension, dot products reduced by shuffles), scores recomputed in both, so
+// no gradient of q, k or v needs an atomic; the table gradients collect in
 // shared memory per block and then in global memory with atomics. A first
 // correct version: the contractions belong on the tensor cores next.
 #pragma once
@@ -40,67 +41,98 @@ struct AttnBwdArgs {
     float* dtime;               // [H, NB] (zeroed before) or null
 };
 
-__device__ __forceinline__ float score_ij(const AttnBwdArgs& a, const float* qi, const float* kj,
-                                          int h, int64_t i, int64_t j, int64_t o, int* pidx,
-                                          int* bkt) {
-    float s = 0.f;
-    for (int c = 0; c < a.dqk; ++c) s = fmaf(qi[c], kj[c], s);
-    *pidx = -1;
-    *bkt = -1;
-    if (a.pos) {
-        *pidx = pos_index(i - o, j - o, a.P);
-        s += a.pos[static_cast<int64_t>(h) * a.P + *pidx];
-    }
-    if (a.ts && a.tb) {
-        *bkt = time_bucket64(a.ts[i] - a.ts[j], a.NB - 1);
-        s += a.tb[static_cast<int64_t>(h) * a.NB + *bkt];
-    }
-    return s;
-}
-
 __device__ __forceinline__ float silu_grad_f(float s) {
     const float sg = 1.0f / (1.0f + expf(-s));
     return sg * (1.0f + s * (1.0f - sg));
 }
 
-// Query pass: dq_i and the table gradients. Dynamic shared memory: P + NB
-// floats (the block's partial table gradients for head blockIdx.y).
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+// Bias of pair (i, j) (sequence start o): adds pos and time to s and returns
+// their table indices (-1 when the term is absent). Lane-uniform.
+__device__ __forceinline__ float pair_bias(const AttnBwdArgs& a, int h, int64_t i, int64_t j,
+                                           int* pidx, int* bkt) {
+    float bias = 0.f;
+    *pidx = -1;
+    *bkt = -1;
+    if (a.pos) {
+        *pidx = pos_index(i, j, a.P);
+        bias += __ldg(a.pos + static_cast<int64_t>(h) * a.P + *pidx);
+    }
+    if (a.ts && a.tb) {
+        *bkt = time_bucket64(__ldg(a.ts + i) - __ldg(a.ts + j), a.NB - 1);
+        bias += __ldg(a.tb + static_cast<int64_t>(h) * a.NB + *bkt);
+    }
+    return bias;
+}
+
+// Query pass: one warp per (query row i, head), lane l holding elements l,
+// l + 32, ... of q_i, dout_i and dq_i; dq_i and the table gradients.
+// Dynamic shared memory: P + NB floats, the block's partial table gradients
+// for head blockIdx.y. The time-table gradient of consecutive keys (which
+// mostly share a bucket) is summed in a register and added once per run.
 template <int DMAX>
 __global__ void __launch_bounds__(128) attn_bwd_q_kernel(const AttnBwdArgs a) {
+    constexpr int NE = DMAX / 32;
     extern __shared__ float tabs[];
     float* spos = tabs;
     float* stime = tabs + (a.pos ? a.P : 0);
-    const int h = blockIdx.y;
+    const int h = blockIdx.y, lane = threadIdx.x & 31;
     const int ntab = (a.pos ? a.P : 0) + ((a.ts && a.tb) ? a.NB : 0);
     for (int e = threadIdx.x; e < ntab; e += blockDim.x) tabs[e] = 0.f;
     __syncthreads();
-    const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t i = static_cast<int64_t>(blockIdx.x) * 4 + (threadIdx.x >> 5);
     if (i < a.T) {
         const int b = find_sequence(a.seq_offsets, a.B, i);
         const int64_t o = a.seq_offsets[b];
-        const float* qi = a.q + (i * a.H + h) * a.dqk;
-        const float* gi = a.dout + (i * a.H + h) * a.dv;
-        float dq[DMAX];
+        float qi[NE], gi[NE], dq[NE];
 #pragma unroll
-        for (int c = 0; c < DMAX; ++c) dq[c] = 0.f;
+        for (int t = 0; t < NE; ++t) {
+            const int c = lane + 32 * t;
+            qi[t] = c < a.dqk ? a.q[(i * a.H + h) * a.dqk + c] : 0.f;
+            gi[t] = c < a.dv ? a.dout[(i * a.H + h) * a.dv + c] : 0.f;
+            dq[t] = 0.f;
+        }
+        int run_bkt = -1;
+        float run = 0.f;
         for (int64_t j = o; j <= i; ++j) {
             const float* kj = a.k + (j * a.H + h) * a.dqk;
             const float* vj = a.v + (j * a.H + h) * a.dv;
+            float kk[NE], sp = 0.f, dpp = 0.f;
+#pragma unroll
+            for (int t = 0; t < NE; ++t) {
+                const int c = lane + 32 * t;
+                kk[t] = c < a.dqk ? kj[c] : 0.f;
+                sp = fmaf(qi[t], kk[t], sp);
+                if (c < a.dv) dpp = fmaf(gi[t], vj[c], dpp);
+            }
             int pidx, bkt;
-            const float s = score_ij(a, qi, kj, h, i, j, o, &pidx, &bkt);
-            float dp = 0.f;
-            for (int c = 0; c < a.dv; ++c) dp = fmaf(gi[c], vj[c], dp);
-            const float ds = dp * silu_grad_f(s) * a.inv_n;
+            const float s = warp_sum(sp) + pair_bias(a, h, i, j, &pidx, &bkt);
+            const float ds = warp_sum(dpp) * silu_grad_f(s) * a.inv_n;
 #pragma unroll
-            for (int c = 0; c < DMAX; ++c)
-                if (c < a.dqk) dq[c] = fmaf(ds, kj[c], dq[c]);
-            if (pidx >= 0) atomicAdd(&spos[pidx], ds);
-            if (bkt >= 0) atomicAdd(&stime[bkt], ds);
+            for (int t = 0; t < NE; ++t) dq[t] = fmaf(ds, kk[t], dq[t]);
+            if (lane == 0) {
+                if (pidx >= 0) atomicAdd(&spos[pidx], ds);
+                if (bkt >= 0) {
+                    if (bkt != run_bkt) {
+                        if (run_bkt >= 0) atomicAdd(&stime[run_bkt], run);
+                        run_bkt = bkt;
+                        run = 0.f;
+                    }
+                    run += ds;
+                }
+            }
         }
-        float* dqi = a.dq + (i * a.H + h) * a.dqk;
+        if (lane == 0 && run_bkt >= 0) atomicAdd(&stime[run_bkt], run);
 #pragma unroll
-        for (int c = 0; c < DMAX; ++c)
-            if (c < a.dqk) dqi[c] = dq[c];
+        for (int t = 0; t < NE; ++t) {
+            const int c = lane + 32 * t;
+            if (c < a.dqk) a.dq[(i * a.H + h) * a.dqk + c] = dq[t];
+        }
     }
     __syncthreads();
     if (a.dpos)
@@ -111,40 +143,51 @@ __global__ void __launch_bounds__(128) attn_bwd_q_kernel(const AttnBwdArgs a) {
             if (stime[e] != 0.f) atomicAdd(&a.dtime[static_cast<int64_t>(h) * a.NB + e], stime[e]);
 }
 
-// Key pass: dk_j and dv_j.
+// Key pass: one warp per (key row j, head), lanes over the elements as in the
+// query pass; dk_j and dv_j.
 template <int DMAX>
 __global__ void __launch_bounds__(128) attn_bwd_kv_kernel(const AttnBwdArgs a) {
-    const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    const int h = blockIdx.y;
+    constexpr int NE = DMAX / 32;
+    const int h = blockIdx.y, lane = threadIdx.x & 31;
+    const int64_t j = static_cast<int64_t>(blockIdx.x) * 4 + (threadIdx.x >> 5);
     if (j >= a.T) return;
     const int b = find_sequence(a.seq_offsets, a.B, j);
-    const int64_t o = a.seq_offsets[b], end = a.seq_offsets[b + 1];
-    const float* kj = a.k + (j * a.H + h) * a.dqk;
-    const float* vj = a.v + (j * a.H + h) * a.dv;
-    float dk[DMAX], dv[DMAX];
+    const int64_t end = a.seq_offsets[b + 1];
+    float kj[NE], vj[NE], dk[NE], dv[NE];
 #pragma unroll
-    for (int c = 0; c < DMAX; ++c) dk[c] = dv[c] = 0.f;
+    for (int t = 0; t < NE; ++t) {
+        const int c = lane + 32 * t;
+        kj[t] = c < a.dqk ? a.k[(j * a.H + h) * a.dqk + c] : 0.f;
+        vj[t] = c < a.dv ? a.v[(j * a.H + h) * a.dv + c] : 0.f;
+        dk[t] = dv[t] = 0.f;
+    }
     for (int64_t i = j; i < end; ++i) {
         const float* qi = a.q + (i * a.H + h) * a.dqk;
         const float* gi = a.dout + (i * a.H + h) * a.dv;
-        int pidx, bkt;
-        const float s = score_ij(a, qi, kj, h, i, j, o, &pidx, &bkt);
-        const float p = s / (1.0f + expf(-s)) * a.inv_n;
-        float dp = 0.f;
-        for (int c = 0; c < a.dv; ++c) dp = fmaf(gi[c], vj[c], dp);
-        const float ds = dp * silu_grad_f(s) * a.inv_n;
+        float qq[NE], gg[NE], sp = 0.f, dpp = 0.f;
 #pragma unroll
-        for (int c = 0; c < DMAX; ++c) {
-            if (c < a.dqk) dk[c] = fmaf(ds, qi[c], dk[c]);
-            if (c < a.dv) dv[c] = fmaf(p, gi[c], dv[c]);
+        for (int t = 0; t < NE; ++t) {
+            const int c = lane + 32 * t;
+            qq[t] = c < a.dqk ? qi[c] : 0.f;
+            gg[t] = c < a.dv ? gi[c] : 0.f;
+            sp = fmaf(qq[t], kj[t], sp);
+            dpp = fmaf(gg[t], vj[t], dpp);
+        }
+        int pidx, bkt;
+        const float s = warp_sum(sp) + pair_bias(a, h, i, j, &pidx, &bkt);
+        const float p = s / (1.0f + expf(-s)) * a.inv_n;
+        const float ds = warp_sum(dpp) * silu_grad_f(s) * a.inv_n;
+#pragma unroll
+        for (int t = 0; t < NE; ++t) {
+            dk[t] = fmaf(ds, qq[t], dk[t]);
+            dv[t] = fmaf(p, gg[t], dv[t]);
         }
     }
-    float* dkj = a.dk + (j * a.H + h) * a.dqk;
-    float* dvj = a.dvv + (j * a.H + h) * a.dv;
 #pragma unroll
-    for (int c = 0; c < DMAX; ++c) {
-        if (c < a.dqk) dkj[c] = dk[c];
-        if (c < a.dv) dvj[c] = dv[c];
+    for (int t = 0; t < NE; ++t) {
+        const int c = lane + 32 * t;
+        if (c < a.dqk) a.dk[(j * a.H + h) * a.dqk + c] = dk[t];
+        if (c < a.dv) a.dvv[(j * a.H + h) * a.dv + c] = dv[t];
     }
 }
 

@@ -645,7 +645,9 @@ hstu_status_t hstu_attn_bwd_f32(const float* q, const float* k, const float* v, 
                   use_time ? timestamps : nullptr, pos_bias, P, use_time ? time_bias : nullptr, NB,
                   1.0f / static_cast<float>(max_seqlen), dq, dk, dv,
                   pos_bias ? dpos : nullptr, use_time ? dtime : nullptr};
-    const dim3 grid(static_cast<unsigned>((total_tokens + 127) / 128), static_cast<unsigned>(H));
+    // four (token, head) warps per block
+    if ((total_tokens + 3) / 4 > 0x7fffffff) return HSTU_ERR_UNSUPPORTED;
+    const dim3 grid(static_cast<unsigned>((total_tokens + 3) / 4), static_cast<unsigned>(H));
     const int dmax = d_qk > d_v ? d_qk : d_v;
     if (dmax <= 32) {
         attn_bwd_q_kernel<32><<<grid, 128, tab_bytes, s>>>(a);
