@@ -122,6 +122,48 @@ def test_linear_and_ln_validation(lib):
     assert lib.hstu_debug_wait_timeout(0, None) == INV
 
 
+def test_fp8_validation(lib):
+    INV, UNS = _native.HSTU_ERR_INVALID_ARG, _native.HSTU_ERR_UNSUPPORTED
+    # quantization: K % 16, code row stride % 16, null scales, empty
+    assert lib.hstu_quant_rows_e4m3(16, 104, 4, 100, 16, 112, 16, None) == UNS
+    assert lib.hstu_quant_rows_e4m3(16, 128, 4, 128, 16, 136, 16, None) == INV
+    assert lib.hstu_quant_rows_e4m3(16, 128, 4, 128, 16, 128, None, None) == INV
+    assert lib.hstu_quant_rows_e4m3(16, 128, 0, 128, 16, 128, 16, None) == 0
+    # FP8 linear: K % 128, missing scales, code strides % 16
+    assert lib.hstu_linear_fp8_fwd(16, 64, 16, 10, 64, 16, 64, 16, 128, None, 0, None, 0, 16, 128,
+                                   None) == UNS
+    assert lib.hstu_linear_fp8_fwd(16, 128, None, 10, 128, 16, 128, 16, 128, None, 0, None, 0, 16,
+                                   128, None) == INV
+    assert lib.hstu_linear_fp8_fwd(16, 136, 16, 10, 128, 16, 128, 16, 128, None, 0, None, 0, 16,
+                                   128, None) == INV
+    # fused LayerNorm gate quantization: code stride % 16
+    assert lib.hstu_layernorm_gate_fp8_fwd(16, 512, 16, 512, 4, 512, None, None,
+                                           ctypes.c_float(1e-5), 16, 520, 16, None) == INV
+    assert lib.hstu_layer_fp8_workspace_bytes(1000, 4, 512, 4, 128, 512) > \
+        lib.hstu_layer_workspace_bytes(1000, 4, 4, 128, 512) - 1
+
+
+def test_backward_validation(lib):
+    INV, UNS = _native.HSTU_ERR_INVALID_ARG, _native.HSTU_ERR_UNSUPPORTED
+
+    def bwd(**kw):
+        a = dict(q=16, k=16, v=16, dout=16, off=16, B=2, T=10, H=2, dqk=32, dv=32, ts=None,
+                 pos=None, P=0, tb=None, NB=0, N=8, dq=16, dk=16, dvv=16, dpos=None, dtime=None)
+        a.update(kw)
+        return lib.hstu_attn_bwd_f32(a["q"], a["k"], a["v"], a["dout"], a["off"], a["B"], a["T"],
+                                     a["H"], a["dqk"], a["dv"], a["ts"], a["pos"], a["P"],
+                                     a["tb"], a["NB"], a["N"], a["dq"], a["dk"], a["dvv"],
+                                     a["dpos"], a["dtime"], None)
+    assert bwd(dqk=129) == UNS
+    assert bwd(H=0) == INV
+    assert bwd(pos=16, P=8) == INV                       # dpos missing
+    assert bwd(ts=16, tb=16, NB=8) == INV                # dtime missing
+    assert bwd(ts=16, tb=16, NB=2000, dtime=16) == INV   # bucket count
+    assert bwd(pos=16, P=13000, dpos=16) == UNS          # table partials exceed shared memory
+    assert bwd(q=None) == INV
+    assert bwd(B=0, T=0) == 0
+
+
 def test_binding_fails_loudly_without_library(tmp_path):
     with pytest.raises(ImportError):
         _native.load(str(tmp_path / "missing.so"))
