@@ -99,31 +99,48 @@ __global__ void __launch_bounds__(128) attn_bwd_q_kernel(const AttnBwdArgs a) {
         }
         int run_bkt = -1;
         float run = 0.f;
-        for (int64_t j = o; j <= i; ++j) {
-            const float* kj = a.k + (j * a.H + h) * a.dqk;
-            const float* vj = a.v + (j * a.H + h) * a.dv;
-            float kk[NE], sp = 0.f, dpp = 0.f;
+        // U keys per step: their shuffle reductions are independent
+        constexpr int U = 4;
+        for (int64_t j0 = o; j0 <= i; j0 += U) {
+            const int nu = static_cast<int>(i - j0 + 1 < U ? i - j0 + 1 : U);
+            float kk[U][NE], sp[U], dpp[U];
 #pragma unroll
-            for (int t = 0; t < NE; ++t) {
-                const int c = lane + 32 * t;
-                kk[t] = c < a.dqk ? kj[c] : 0.f;
-                sp = fmaf(qi[t], kk[t], sp);
-                if (c < a.dv) dpp = fmaf(gi[t], vj[c], dpp);
+            for (int u = 0; u < U; ++u) {
+                sp[u] = dpp[u] = 0.f;
+                const int64_t j = j0 + (u < nu ? u : 0);
+                const float* kj = a.k + (j * a.H + h) * a.dqk;
+                const float* vj = a.v + (j * a.H + h) * a.dv;
+#pragma unroll
+                for (int t = 0; t < NE; ++t) {
+                    const int c = lane + 32 * t;
+                    kk[u][t] = c < a.dqk ? kj[c] : 0.f;
+                    sp[u] = fmaf(qi[t], kk[u][t], sp[u]);
+                    if (c < a.dv) dpp[u] = fmaf(gi[t], vj[c], dpp[u]);
+                }
             }
-            int pidx, bkt;
-            const float s = warp_sum(sp) + pair_bias(a, h, i, j, &pidx, &bkt);
-            const float ds = warp_sum(dpp) * silu_grad_f(s) * a.inv_n;
 #pragma unroll
-            for (int t = 0; t < NE; ++t) dq[t] = fmaf(ds, kk[t], dq[t]);
-            if (lane == 0) {
-                if (pidx >= 0) atomicAdd(&spos[pidx], ds);
-                if (bkt >= 0) {
-                    if (bkt != run_bkt) {
-                        if (run_bkt >= 0) atomicAdd(&stime[run_bkt], run);
-                        run_bkt = bkt;
-                        run = 0.f;
+            for (int u = 0; u < U; ++u) {
+                sp[u] = warp_sum(sp[u]);
+                dpp[u] = warp_sum(dpp[u]);
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (u >= nu) break;
+                int pidx, bkt;
+                const float s = sp[u] + pair_bias(a, h, i, j0 + u, &pidx, &bkt);
+                const float ds = dpp[u] * silu_grad_f(s) * a.inv_n;
+#pragma unroll
+                for (int t = 0; t < NE; ++t) dq[t] = fmaf(ds, kk[u][t], dq[t]);
+                if (lane == 0) {
+                    if (pidx >= 0) atomicAdd(&spos[pidx], ds);
+                    if (bkt >= 0) {
+                        if (bkt != run_bkt) {
+                            if (run_bkt >= 0) atomicAdd(&stime[run_bkt], run);
+                            run_bkt = bkt;
+                            run = 0.f;
+                        }
+                        run += ds;
                     }
-                    run += ds;
                 }
             }
         }
@@ -161,26 +178,43 @@ __global__ void __launch_bounds__(128) attn_bwd_kv_kernel(const AttnBwdArgs a) {
         vj[t] = c < a.dv ? a.v[(j * a.H + h) * a.dv + c] : 0.f;
         dk[t] = dv[t] = 0.f;
     }
-    for (int64_t i = j; i < end; ++i) {
-        const float* qi = a.q + (i * a.H + h) * a.dqk;
-        const float* gi = a.dout + (i * a.H + h) * a.dv;
-        float qq[NE], gg[NE], sp = 0.f, dpp = 0.f;
+    // U queries per step: their shuffle reductions are independent
+    constexpr int U = 4;
+    for (int64_t i0 = j; i0 < end; i0 += U) {
+        const int nu = static_cast<int>(end - i0 < U ? end - i0 : U);
+        float qq[U][NE], gg[U][NE], sp[U], dpp[U];
 #pragma unroll
-        for (int t = 0; t < NE; ++t) {
-            const int c = lane + 32 * t;
-            qq[t] = c < a.dqk ? qi[c] : 0.f;
-            gg[t] = c < a.dv ? gi[c] : 0.f;
-            sp = fmaf(qq[t], kj[t], sp);
-            dpp = fmaf(gg[t], vj[t], dpp);
+        for (int u = 0; u < U; ++u) {
+            sp[u] = dpp[u] = 0.f;
+            const int64_t i = i0 + (u < nu ? u : 0);
+            const float* qi = a.q + (i * a.H + h) * a.dqk;
+            const float* gi = a.dout + (i * a.H + h) * a.dv;
+#pragma unroll
+            for (int t = 0; t < NE; ++t) {
+                const int c = lane + 32 * t;
+                qq[u][t] = c < a.dqk ? qi[c] : 0.f;
+                gg[u][t] = c < a.dv ? gi[c] : 0.f;
+                sp[u] = fmaf(qq[u][t], kj[t], sp[u]);
+                dpp[u] = fmaf(gg[u][t], vj[t], dpp[u]);
+            }
         }
-        int pidx, bkt;
-        const float s = warp_sum(sp) + pair_bias(a, h, i, j, &pidx, &bkt);
-        const float p = s / (1.0f + expf(-s)) * a.inv_n;
-        const float ds = warp_sum(dpp) * silu_grad_f(s) * a.inv_n;
 #pragma unroll
-        for (int t = 0; t < NE; ++t) {
-            dk[t] = fmaf(ds, qq[t], dk[t]);
-            dv[t] = fmaf(p, gg[t], dv[t]);
+        for (int u = 0; u < U; ++u) {
+            sp[u] = warp_sum(sp[u]);
+            dpp[u] = warp_sum(dpp[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (u >= nu) break;
+            int pidx, bkt;
+            const float s = sp[u] + pair_bias(a, h, i0 + u, j, &pidx, &bkt);
+            const float p = s / (1.0f + expf(-s)) * a.inv_n;
+            const float ds = dpp[u] * silu_grad_f(s) * a.inv_n;
+#pragma unroll
+            for (int t = 0; t < NE; ++t) {
+                dk[t] = fmaf(ds, qq[u][t], dk[t]);
+                dv[t] = fmaf(p, gg[u][t], dv[t]);
+            }
         }
     }
 #pragma unroll
