@@ -464,6 +464,42 @@ def check_attn_bwd_finite_differences(lib):
                 name, ix, fd, g)
 
 
+def check_attn_bwd_against_torch_autograd(lib):
+    """The oracle's gradients against torch autograd of a dense, per-sequence
+    torch formulation of the forward (matmul scores, gathered bias matrices,
+    lower-triangular mask, torch SiLU), written independently of the oracle."""
+    inp = tiny_case(seed=6, lengths=(4, 0, 9, 1, 12), H=2, d=3, P=5, NB=7)
+    rng = np.random.default_rng(13)
+    dout = rng.standard_normal(inp.v.shape)
+    tq = torch.tensor(inp.q, dtype=torch.float64, requires_grad=True)
+    tk = torch.tensor(inp.k, dtype=torch.float64, requires_grad=True)
+    tv = torch.tensor(inp.v, dtype=torch.float64, requires_grad=True)
+    tpos = torch.tensor(inp.pos_bias, dtype=torch.float64, requires_grad=True)
+    ttb = torch.tensor(inp.time_bias, dtype=torch.float64, requires_grad=True)
+    off, ts, N = inp.seq_offsets, inp.timestamps, inp.max_seqlen
+    P, NB = inp.pos_bias.shape[1], inp.time_bias.shape[1]
+    loss = torch.zeros((), dtype=torch.float64)
+    for b in range(len(off) - 1):
+        o, n = int(off[b]), int(off[b + 1] - off[b])
+        if n == 0:
+            continue
+        I, J = np.meshgrid(np.arange(n), np.arange(n), indexing="ij")
+        pidx = torch.from_numpy(np.clip(I - J, 0, P - 1))
+        dt = ts[o + I] - ts[o + J]
+        bidx = torch.from_numpy(np.clip(_floor_log2_frexp(np.maximum(dt, 1)), 0, NB - 1))
+        mask = torch.tril(torch.ones((n, n), dtype=torch.float64))
+        for h in range(inp.H):
+            S = tq[o:o + n, h] @ tk[o:o + n, h].T + tpos[h][pidx] + ttb[h][bidx]
+            out = (torch.nn.functional.silu(S) * mask) @ tv[o:o + n, h] / N
+            loss = loss + (out * torch.from_numpy(dout[o:o + n, h])).sum()
+    loss.backward()
+    got = oracle.attn_bwd(off, inp.q, inp.k, inp.v, ts, inp.pos_bias, inp.time_bias, N, dout,
+                          lib=lib)
+    for name, g, t in zip(("dq", "dk", "dv", "dpos", "dtime"), got,
+                          (tq, tk, tv, tpos, ttb)):
+        _close(g, t.grad.numpy(), what="autograd " + name)
+
+
 def check_attn_bwd_closed_form(lib):
     """q = k = 0 and constant biases c: every score is c, so dv[j] = silu(c)/N
     times the suffix sum of dout over the rows i >= j of j's sequence, and the
@@ -609,4 +645,5 @@ ALL_CHECKS = [
     check_layer_composition, check_layer_identities, check_e4m3_table,
     check_e4m3_rounding_against_torch, check_e4m3_saturation, check_quant_rows, check_linear_fp8,
     check_silu_grad, check_attn_bwd_finite_differences, check_attn_bwd_closed_form,
+    check_attn_bwd_against_torch_autograd,
 ]
