@@ -16,6 +16,8 @@
  *   out[o+i,h,:] = (1/max_seqlen) * sum_{j<=i} silu(s_ij) * v[o+j,h,:]
  *
  * with silu(x) = x * sigmoid(x). No softmax, no 1/sqrt(d) score scale.
+ * Besides the bf16 forward path: row-wise E4M3 (FP8) projections and the
+ * attention backward (fp32), in their own sections below.
  *
  * Conventions for every entry point:
  *  - Pointers marked "device" must be device memory of the current CUDA device
