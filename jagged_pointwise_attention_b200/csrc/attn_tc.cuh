@@ -74,6 +74,7 @@ struct KeySummary;
 struct AttnArgs {
     const int4* units;          // plan: (q0, q_end, k0, nk | nt << 11 | packed << 31)
     const int* unit_count;
+    int max_units;              // capacity of the work list (the count is clamped to it)
     int* item_counter;          // plan: zeroed; next work item to hand out
     const uint4* starts;        // plan: per packed unit, rows where a sequence begins
     const uint4* ptab;          // bias prep: [H][DD][248] window tables (see BiasStage)
@@ -454,7 +455,7 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const int n_items = *args.unit_count * args.H;
+    const int n_items = min(*args.unit_count, args.max_units) * args.H;
 
     const uint32_t sQ = smem_u32(smem + L::kOffQ);
     const uint32_t sK = smem_u32(smem + L::kOffK);

@@ -55,6 +55,12 @@ __device__ __forceinline__ uint32_t window_word(const float* prow, int P, int re
     return wd;
 }
 
+// Programmatic launch chain plan -> bias prep -> attention. The attention
+// waits (griddepcontrol.wait) only for this grid, its direct prerequisite, so
+// this grid must not complete before the plan has: every block of it executes
+// griddepcontrol.wait before it exits, including the blocks that never read
+// the plan's output. The table blocks wait after writing their entries, so
+// that work still overlaps the plan.
 __global__ void __launch_bounds__(128) bias_prep_kernel(const BiasPrepArgs a) {
     // let the attention that follows start its set-up (it waits for this grid)
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -62,23 +68,25 @@ __global__ void __launch_bounds__(128) bias_prep_kernel(const BiasPrepArgs a) {
     if (static_cast<int>(blockIdx.x) < a.table_blocks) {
         // entry s of table (h, dd) holds R[s..s+7]: words (R[s+2i], R[s+2i+1])
         const int64_t e = static_cast<int64_t>(blockIdx.x) * 128 + tid;
-        if (e >= static_cast<int64_t>(a.H) * a.DD * kWinEntries) return;
-        const int s = static_cast<int>(e % kWinEntries);
-        const int hd = static_cast<int>(e / kWinEntries);
-        const int h = hd / a.DD, dd = hd % a.DD;
-        const float* prow = a.pos ? a.pos + static_cast<int64_t>(h) * a.P : nullptr;
-        const int rel0 = 128 * dd + 127;                 // window offset of R[0]
-        const uint32_t sel = (s & 1) ? 0x5432u : 0x3210u;
-        uint32_t x[5];
+        if (e < static_cast<int64_t>(a.H) * a.DD * kWinEntries) {
+            const int s = static_cast<int>(e % kWinEntries);
+            const int hd = static_cast<int>(e / kWinEntries);
+            const int h = hd / a.DD, dd = hd % a.DD;
+            const float* prow = a.pos ? a.pos + static_cast<int64_t>(h) * a.P : nullptr;
+            const int rel0 = 128 * dd + 127;                 // window offset of R[0]
+            const uint32_t sel = (s & 1) ? 0x5432u : 0x3210u;
+            uint32_t x[5];
 #pragma unroll
-        for (int k = 0; k < 5; ++k) x[k] = window_word(prow, a.P, rel0, (s >> 1) + k);
-        a.ptab[e] = make_uint4(__byte_perm(x[0], x[1], sel), __byte_perm(x[1], x[2], sel),
-                               __byte_perm(x[2], x[3], sel), __byte_perm(x[3], x[4], sel));
+            for (int k = 0; k < 5; ++k) x[k] = window_word(prow, a.P, rel0, (s >> 1) + k);
+            a.ptab[e] = make_uint4(__byte_perm(x[0], x[1], sel), __byte_perm(x[1], x[2], sel),
+                                   __byte_perm(x[2], x[3], sel), __byte_perm(x[3], x[4], sel));
+        }
+        asm volatile("griddepcontrol.wait;" ::: "memory");   // complete only after the plan
         return;
     }
     // key summary of unit u: its 128 rows as keys
-    if (a.ts == nullptr) return;
     asm volatile("griddepcontrol.wait;" ::: "memory");   // the plan's units
+    if (a.ts == nullptr) return;
     const int u = static_cast<int>(blockIdx.x) - a.table_blocks;
     const int n_units = min(*a.unit_count, a.max_units);
     if (u >= n_units) return;

@@ -284,6 +284,7 @@ hstu_status_t run_attn(const AttnCall& c) {
     }
     AttnArgs a{reinterpret_cast<const int4*>(ws + kAttnWsHeader),
                reinterpret_cast<const int*>(ws),
+               static_cast<int>(max_units),
                reinterpret_cast<int*>(ws + 16),
                reinterpret_cast<const uint4*>(ws + kAttnWsHeader +
                                               attn_units_bytes(c.B, c.T, c.max_seqlen)),

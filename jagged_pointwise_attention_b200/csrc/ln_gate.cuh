@@ -100,12 +100,13 @@ __global__ void __launch_bounds__(256) ln_gate_kernel(const LnGateArgs a) {
         for (int k = 0; k < NV; ++k) amax_bits = amax_bits8(yrow[QUANT ? k : 0], amax_bits);
         amax_bits = __reduce_max_sync(0xffffffffu, amax_bits);
         const float amax = __uint_as_float(amax_bits);
-        const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 0.f;
+        const float2 f = e4m3_row_factors(amax);
+        const float inv = f.x;
 #pragma unroll
         for (int k = 0; k < NV; ++k)
             *reinterpret_cast<uint2*>(a.yq + m * a.ldyq + k * 256 + lane * 8) =
                 e4m3_codes8(yrow[QUANT ? k : 0], inv);
-        if (lane == 0) a.ys[m] = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+        if (lane == 0) a.ys[m] = f.y;
     }
 }
 

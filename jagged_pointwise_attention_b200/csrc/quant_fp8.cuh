@@ -3,10 +3,12 @@
 // reference and benchmark").
 //
 // Per row r: amax = max |x[r, :]|, inv = 448 / amax and scale = amax / 448
-// (fp32, rounded to nearest; an all-zero row takes inv 0, scale 1), and
-// code = E4M3(x * inv) with the product rounded to fp32 and the conversion
-// rounding to nearest, ties to even, saturating at +-448. One warp per row;
-// each lane reads 8 bf16 (16 bytes) per step and writes 8 codes.
+// (fp32, rounded to nearest), and code = E4M3(x * inv) with the product
+// rounded to fp32 and the conversion rounding to nearest, ties to even,
+// saturating at +-448. A row whose inv is not a finite fp32 number (all
+// zeros, or amax below 448 / FLT_MAX) takes inv 0 and scale 1: zero codes.
+// One warp per row; each lane reads 8 bf16 (16 bytes) per step and writes 8
+// codes.
 #pragma once
 
 #include <cuda_fp8.h>
@@ -55,6 +57,13 @@ __device__ __forceinline__ uint32_t amax_bits8(const uint4 v, uint32_t m) {
     return m;
 }
 
+// The row's (inv, scale) from its amax, as described above.
+__device__ __forceinline__ float2 e4m3_row_factors(float amax) {
+    const float q = amax > 0.f ? __fdiv_rn(448.f, amax) : 0.f;
+    const bool finite = amax > 0.f && q <= 3.402823466e38f;
+    return make_float2(finite ? q : 0.f, finite ? __fdiv_rn(amax, 448.f) : 1.f);
+}
+
 // Rows of up to kQuantCached * 256 values are read once, into registers (all loads
 // of a lane in flight together); longer rows are read twice.
 constexpr int kQuantCached = 4;
@@ -82,8 +91,8 @@ __global__ void __launch_bounds__(256) quant_rows_e4m3_kernel(const QuantArgs a)
     }
     amax_bits = __reduce_max_sync(0xffffffffu, amax_bits);
     const float amax = __uint_as_float(amax_bits);
-    const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 0.f;
-    const float scale = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+    const float2 f = e4m3_row_factors(amax);
+    const float inv = f.x, scale = f.y;
     if (cached) {
 #pragma unroll
         for (int i = 0; i < kQuantCached; ++i) {

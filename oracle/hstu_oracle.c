@@ -25,6 +25,7 @@
  * Everything is evaluated in double precision, one output row at a time, in
  * the order of the definition. No blocking, no fusion, no reordering.
  */
+#include <float.h>
 #include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
@@ -284,9 +285,11 @@ uint8_t hstu_oracle_e4m3_from_float(float x) {
 }
 
 /* Row-wise quantization of x [M, K] (fp32 values): amax_r = max |x[r, :]|;
- * inv_r = 448 / amax_r and scale_r = amax_r / 448 in fp32 (an all-zero row
- * takes inv 0 and scale 1); code[r, c] = e4m3(x[r, c] * inv_r) with the product
- * rounded to fp32 first. Then x[r, c] ~ e4m3_to_float(code) * scale_r. */
+ * inv_r = 448 / amax_r and scale_r = amax_r / 448 in fp32; code[r, c] =
+ * e4m3(x[r, c] * inv_r) with the product rounded to fp32 first. Then
+ * x[r, c] ~ e4m3_to_float(code) * scale_r. A row whose inv_r is not a finite
+ * fp32 number -- all zeros, or amax_r below 448 / FLT_MAX (about 1.3e-36) --
+ * takes inv 0 and scale 1, so its codes are (signed) zeros. */
 void hstu_oracle_quant_rows_e4m3(int64_t M, int32_t K, const float* x, uint8_t* codes,
                                  float* scales) {
 #pragma omp parallel for schedule(static)
@@ -296,8 +299,10 @@ void hstu_oracle_quant_rows_e4m3(int64_t M, int32_t K, const float* x, uint8_t* 
             const float v = fabsf(x[r * K + c]);
             if (v > amax) amax = v;
         }
-        volatile float inv = amax > 0.0f ? 448.0f / amax : 0.0f;
-        volatile float scale = amax > 0.0f ? amax / 448.0f : 1.0f;
+        volatile float q = amax > 0.0f ? 448.0f / amax : 0.0f;
+        const int finite = amax > 0.0f && q <= FLT_MAX;
+        volatile float inv = finite ? q : 0.0f;
+        volatile float scale = finite ? amax / 448.0f : 1.0f;
         for (int32_t c = 0; c < K; ++c) {
             volatile float y = x[r * K + c] * inv;
             codes[r * K + c] = hstu_oracle_e4m3_from_float(y);

@@ -612,6 +612,14 @@ def check_quant_rows(lib):
     assert np.all(err[normal] <= 2.0 ** -4 * np.abs(x[normal]) * (1 + 1e-6)), "normal range"
     assert np.all(err[~normal] <= 2.0 ** -10 * np.broadcast_to(scales[:, None], x.shape)[~normal]
                   * (1 + 1e-6)), "subnormal range"
+    # rows too small for a finite 448 / amax in fp32 (amax < 448 / FLT_MAX):
+    # never NaN codes, and the dequantized row is within that bound of x
+    fmax = float(np.finfo(np.float32).max)
+    tiny = np.array([[1e-37, -3e-38, 0.0, 2e-37], [1.2e-38, 0.0, -1.2e-38, 5e-37]], np.float32)
+    tc, ts_ = oracle.quant_rows_e4m3(tiny, lib=lib)
+    assert not np.any((tc & 0x7F) == 0x7F), "NaN codes for a tiny row"
+    tdeq = oracle.e4m3_to_float(tc, lib=lib).astype(np.float64) * ts_[:, None]
+    assert np.all(np.isfinite(tdeq)) and np.all(np.abs(tdeq - tiny) <= 448.0 / fmax), "tiny rows"
 
 
 def check_linear_fp8(lib):

@@ -40,18 +40,21 @@ def test_quant_codes_bit_exact(M, K):
 def test_quant_edge_rows():
     """All-zero rows (signed zeros kept), a row whose amax is a power of two,
     one tiny value among large ones (underflow to a subnormal or zero code),
-    a row of equal magnitudes."""
+    a row of equal magnitudes, and a row too small for a finite 448 / amax
+    (quantized like a zero row, never to NaN codes)."""
     K = 64
-    x = np.zeros((6, K), dtype=np.float32)
+    x = np.zeros((7, K), dtype=np.float32)
     x[1, ::2] = -0.0
     x[2] = np.linspace(-4, 4, K)
     x[3, 0], x[3, 1:] = 3e-6, 1000.0
     x[4] = -7.5
     x[5] = round_to_bf16(np.random.default_rng(0).standard_normal(K).astype(np.float32)) * 1e-30
+    x[6] = np.random.default_rng(1).standard_normal(K).astype(np.float32) * 1e-37
     x = round_to_bf16(x)
     got_c, got_s, want_c, want_s = _quant_both(x)
     assert np.array_equal(got_s, want_s)
     assert np.array_equal(got_c, want_c)
+    assert not np.any((got_c & 0x7F) == 0x7F), "NaN codes"
 
 
 @pytest.mark.parametrize("M,K,N,epi", [(300, 512, 384, "silu"), (1000, 512, 2048, "silu"),

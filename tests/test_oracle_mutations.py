@@ -58,6 +58,8 @@ MUTANTS = [
     ("e4m3_overflow_to_nan", "if (a >= 448.0) return sign | 0x7E;",
      "if (a > 448.0) return sign | 0x7F;"),
     ("quant_scale_not_amax", "if (v > amax) amax = v;", "if (v > amax) amax = v * 0.5f;"),
+    ("quant_inv_overflow_unchecked", "const int finite = amax > 0.0f && q <= FLT_MAX;",
+     "const int finite = amax > 0.0f;"),
     ("fp8_scale_inverted", "acc *= (double)sx[m] * (double)sw[n];",
      "acc *= (double)sx[m] / (double)sw[n];"),
     ("bwd_silu_grad_is_sigmoid", "return sg * (1.0 + s * (1.0 - sg));", "return sg;"),
