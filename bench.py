@@ -233,14 +233,62 @@ def oracle_sample_rate(inp, budget_s: float, seed: int = 0):
 
 # ----------------------------------------------------------------------------- GPU arm
 
-def bench_attention(args, rank, world, local, peaks, peak_kind):
+def l2_note(in_bytes, ncopies):
+    """How the timing keeps HBM honest: inputs larger than L2, or rotating
+    input copies whose total is more than twice L2."""
+    if ncopies == 1:
+        return "inputs %.0f MB > L2" % (in_bytes / 2 ** 20)
+    return "rotating %d input copies (%.0f MB) > 2x L2" % (ncopies, ncopies * in_bytes / 2 ** 20)
+
+
+def attn_copies(in_bytes):
+    return max(1, int(np.ceil(2 * L2_BYTES / max(in_bytes, 1))))
+
+
+def workload_config(cfg_id, B, T, max_seqlen, seed, world, extra):
+    """The ``config`` dict of a line; both arms print the same one."""
+    from gen import CONFIGS
+    cfg = CONFIGS[cfg_id]
+    c = {"workload": cfg["name"], "B": B, "total_tokens": T, "max_seqlen": max_seqlen,
+         "num_pos": cfg["num_pos"], "num_time_buckets": cfg["num_buckets"], "seed": seed,
+         "parallelism": "dp%d" % world}
+    c.update(extra)
+    return c
+
+
+def launch_floor_ms(dev, steps):
+    """Per-launch time of a graph of ``steps`` launches of a one-element torch
+    kernel: the floor a graph-replayed step of one launch cannot go below."""
+    import torch
+    x = torch.zeros(1, device=dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(steps):
+            x.add_(1.0)
+    g.replay()
+    torch.cuda.synchronize(dev)
+    best = None
+    for _ in range(3):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize(dev)
+        t = a.elapsed_time(b) / steps
+        best = t if best is None else min(best, t)
+    del g
+    return best
+
+
+def bench_attention(args, rank, world, local, peaks, peak_kind, cfg_id=None, cpu_budget_s=None):
     import torch
     import jagged_pointwise_attention_b200 as hstu
     from gen import CONFIGS, make_attn_inputs
 
-    cfg = CONFIGS[args.config]
-    seed = 1000 + args.config + 7919 * rank
-    inp = make_attn_inputs(args.config, seed=seed)
+    cfg_id = args.config if cfg_id is None else cfg_id
+    cfg = CONFIGS[cfg_id]
+    seed = 1000 + cfg_id + 7919 * rank
+    inp = make_attn_inputs(cfg_id, seed=seed)
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
     bf = torch.bfloat16 if inp.dtype == "bf16" else torch.float32
@@ -250,7 +298,7 @@ def bench_attention(args, rank, world, local, peaks, peak_kind):
     nbytes = attn_bytes(inp.T, inp.B, H, d, d, inp.pos_bias.shape[1], inp.time_bias.shape[1],
                         2 if inp.dtype == "bf16" else 4)
     in_bytes = inp.T * H * 3 * d * (2 if bf == torch.bfloat16 else 4)
-    ncopies = max(1, int(np.ceil(2 * L2_BYTES / max(in_bytes, 1))))
+    ncopies = attn_copies(in_bytes)
 
     def to_dev(a, dt=None):
         t = torch.from_numpy(np.ascontiguousarray(a))
@@ -345,7 +393,7 @@ def bench_attention(args, rank, world, local, peaks, peak_kind):
     gbs = nbytes / (k_avg_ms * 1e-3) / 1e9
     tag = "attn_fwd_bf16_" + cfg["name"]
     traffic = profiled_traffic(tag)
-    if args.config == 4:
+    if cfg_id == 4:
         roofline = {"bound": "tensor", "achieved": round(tflops, 2),
                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                     "frac": round(tflops / peaks["bf16_tflops"], 4),
@@ -363,9 +411,18 @@ def bench_attention(args, rank, world, local, peaks, peak_kind):
     # end to end: pinned host inputs -> device, public API call, result -> pinned host
     e2e = e2e_attention(args, inp, dev, stream, flops, world)
 
+    if cfg_id != 4:
+        # the short batches are latency-bound: report the launch floor of a
+        # graph-replayed step and the HBM-bar time next to the step
+        floor = launch_floor_ms(dev, max(args.steps, 10))
+        roofline.update({"launch_floor_ms": round(floor, 4),
+                         "hbm_bar_ms": round(nbytes / (0.6 * peaks["hbm_gbs"] * 1e9) * 1e3, 4),
+                         "step_over_kernel": round(ms_per_step / k_avg_ms, 3)})
+
     cpu = None
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
-        v, nrows, secs, thr = oracle_sample_rate(inp, args.cpu_budget_s)
+        v, nrows, secs, thr = oracle_sample_rate(
+            inp, args.cpu_budget_s if cpu_budget_s is None else cpu_budget_s)
         cpu = {"value": round(v, 6), "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
                "sample": "%d random query rows (all heads) of the same batch, fp64, %.1f s"
                          % (nrows, secs)}
@@ -376,15 +433,9 @@ def bench_attention(args, rank, world, local, peaks, peak_kind):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": inp.dtype,
         "data": "synthetic (seeded generator; no dataset)",
-        "config": {"workload": cfg["name"], "B": inp.B, "H": H, "d": d,
-                   "total_tokens": inp.T, "max_seqlen": inp.max_seqlen,
-                   "num_pos": int(inp.pos_bias.shape[1]), "num_time_buckets":
-                   int(inp.time_bias.shape[1]), "seed": seed, "parallelism": "dp%d" % world,
-                   "l2": ("inputs %.0f MB > L2" % (in_bytes / 2 ** 20)) if ncopies == 1 else
-                         ("rotating %d input copies (%.0f MB) > 2x L2" %
-                          (ncopies, ncopies * in_bytes / 2 ** 20)),
-                   "launch": "eager" if args.no_graph else
-                             "one CUDA graph of the K steps (plan + run each)"},
+        "config": workload_config(cfg_id, inp.B, inp.T, inp.max_seqlen, seed, world,
+                                  {"H": H, "d": d, "l2": l2_note(in_bytes, ncopies)}),
+        "launch": "eager" if args.no_graph else "one CUDA graph of the K steps (plan + run each)",
         "pct_of_bf16_peak": {"measured_burst": round(100 * value / peaks["bf16_tflops"], 2),
                              "nominal_2250": round(100 * value / NOMINAL_BF16_TFLOPS, 2)},
         "tokens_per_s": round(total_tokens / (max_ms * 1e-3), 1),
@@ -471,14 +522,47 @@ def e2e_attention(args, inp, dev, stream, flops, world):
                         "step i-2's device-to-host copy (three streams, two buffer sets)"}
 
 
-def bench_layer(args, rank, world, local, peaks, peak_kind):
+def oracle_layer_rate(li, budget_s: float, seed: int = 0):
+    """Time the fp64 oracle's whole layer on a random subset of whole
+    sequences of ``li`` sized to about ``budget_s`` seconds. Returns
+    (TFLOP/s, sequences, tokens, seconds, threads)."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    off = li.seq_offsets
+    order = rng.permutation(li.B)
+
+    def run(seqs):
+        seqs = np.sort(seqs)
+        idx = np.concatenate([np.arange(off[b], off[b + 1]) for b in seqs])
+        lens = np.diff(off)[seqs]
+        o = np.zeros(len(seqs) + 1, np.int64)
+        np.cumsum(lens, out=o[1:])
+        t0 = time.perf_counter()
+        oracle.layer(o, li.x[idx], li.W1, li.W2, li.H, li.d, li.timestamps[idx], li.pos_bias,
+                     li.time_bias, li.max_seqlen, ln_eps=li.ln_eps)
+        dt = time.perf_counter() - t0
+        fl = causal_flops(lens, li.H, li.d, li.d) + layer_flops(int(lens.sum()), li.D, li.H, li.d)
+        return fl, dt, int(lens.sum())
+
+    k = 1
+    while True:
+        fl, dt, ntok = run(order[:k])
+        if dt >= budget_s / 4 or k >= li.B:
+            break
+        k = min(li.B, max(k + 1, int(k * budget_s / 4 / max(dt, 1e-3))))
+    rate = fl / dt
+    return rate / 1e12, k, ntok, dt, oracle.num_threads()
+
+
+def bench_layer(args, rank, world, local, peaks, peak_kind, cfg_id=None, cpu_budget_s=None):
     import torch
     import jagged_pointwise_attention_b200 as hstu
     from gen import CONFIGS, make_layer_inputs
 
-    cfg = CONFIGS[args.config]
-    seed = 1000 + args.config + 7919 * rank
-    li = make_layer_inputs(args.config, seed=seed)
+    cfg_id = args.config if cfg_id is None else cfg_id
+    cfg = CONFIGS[cfg_id]
+    seed = 1000 + cfg_id + 7919 * rank
+    li = make_layer_inputs(cfg_id, seed=seed)
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
     bf = torch.bfloat16
@@ -534,18 +618,27 @@ def bench_layer(args, rank, world, local, peaks, peak_kind):
                 "peak_kind": "burst bf16 dense, %s" % peak_kind, "traffic": None,
                 "kernel": "whole layer step (f1, plan, bias tables, attention, LayerNorm gate, f2)"}
     e2e = None if args.fp8 else e2e_layer(args, li, dev, stream, fl, world, hstu, ws)
+    cpu = None
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        v, nseq, ntok, secs, thr = oracle_layer_rate(
+            li, args.cpu_budget_s if cpu_budget_s is None else cpu_budget_s)
+        cpu = {"value": round(v, 6), "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+               "sample": "%d random whole sequences (%d tokens) of the same batch, the whole "
+                         "layer in fp64, %.1f s" % (nseq, ntok, secs)}
     return {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(max_ms / args.steps, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 projections, bf16 attention" if args.fp8 else "bf16",
         "data": "synthetic (seeded generator; no dataset)",
-        "config": {"workload": cfg["name"] + ("_fp8_projections" if args.fp8 else ""),
-                   "B": li.B, "D": li.D, "H": li.H, "d": li.d,
-                   "total_tokens": li.T, "parallelism": "dp%d" % world,
-                   "l2": "layer working set > L2"},
+        "config": workload_config(cfg_id, li.B, li.T, li.max_seqlen, seed, world,
+                                  {"D": li.D, "H": li.H, "d": li.d,
+                                   "projections": "e4m3" if args.fp8 else "bf16",
+                                   "l2": "layer working set %.0f MB > L2" % (
+                                       (ws.numel() + 2 * x.numel() * 2) / 2 ** 20)}),
+        "launch": "eager, one call per step",
         "tokens_per_s": round(toks / (max_ms * 1e-3), 1),
         "pct_of_bf16_peak": {"measured_burst": round(100 * value / peaks["bf16_tflops"], 2)},
-        "roofline": roofline, "cpu_baseline": None, "e2e": e2e,
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": (7 if args.fp8 else 6) * args.steps, "clocks": sampler.summary(),
     }
 
@@ -759,40 +852,66 @@ def _barrier(world):
 # ----------------------------------------------------------------------------- reference arm
 
 def bench_reference(args, rank, world):
-    """The fp64 CPU oracle on the host cores: each step a bounded row sample of
-    the same workload, sized so the whole run ends within a few minutes."""
+    """The fp64 CPU oracle on the host cores: each step a bounded sample of the
+    same workload (random query rows of the attention batch, or random whole
+    sequences of the layer batch), sized so the whole run ends within a few
+    minutes. ``ms_per_step`` is the measured wall time of one sampled step;
+    the time the oracle would take for the whole batch is extrapolated from
+    the rate and labelled as such."""
     if rank != 0:
         return None
-    from gen import CONFIGS, make_attn_inputs
+    from gen import CONFIGS, make_attn_inputs, make_layer_inputs
     import oracle
-    cfg = CONFIGS[args.config]
-    if cfg["kind"] != "attn":
-        return {"impl": "reference", "unavailable": "reference arm covers the attention "
-                "workloads only"}
-    inp = make_attn_inputs(args.config, seed=1000 + args.config)
+    cfg_id = 4 if args.config is None else args.config
+    cfg = CONFIGS[cfg_id]
+    seed = 1000 + cfg_id
     n_steps = args.steps + args.warmup
     per_step = max(0.5, min(20.0, args.reference_budget_s / max(n_steps, 1)))
-    rates, secs, rows = [], 0.0, 0
+    rates, walls, secs, units = [], [], 0.0, 0
+    if cfg["kind"] == "layer":
+        li = make_layer_inputs(cfg_id, seed=seed)
+        fl_batch = causal_flops(np.diff(li.seq_offsets), li.H, li.d, li.d) + \
+            layer_flops(li.T, li.D, li.H, li.d)
+        ws_bytes = 2 * li.T * (4 + 1 + 1) * li.H * li.d
+        conf = workload_config(cfg_id, li.B, li.T, li.max_seqlen, seed, world,
+                               {"D": li.D, "H": li.H, "d": li.d, "projections": "bf16",
+                                "l2": "layer working set %.0f MB > L2" % (
+                                    (ws_bytes + 2 * li.T * li.D * 2) / 2 ** 20)})
+        what = "random whole sequences"
+    else:
+        inp = make_attn_inputs(cfg_id, seed=seed)
+        fl_batch = causal_flops(inp.lengths, inp.H, inp.d, inp.d)
+        in_bytes = inp.T * inp.H * 3 * inp.d * (2 if inp.dtype == "bf16" else 4)
+        conf = workload_config(cfg_id, inp.B, inp.T, inp.max_seqlen, seed, world,
+                               {"H": inp.H, "d": inp.d,
+                                "l2": l2_note(in_bytes, attn_copies(in_bytes))})
+        what = "random query rows (all heads)"
     for s in range(n_steps):
-        v, nr, dt, thr = oracle_sample_rate(inp, per_step, seed=s)
+        t0 = time.perf_counter()
+        if cfg["kind"] == "layer":
+            v, nu, _, dt, thr = oracle_layer_rate(li, per_step, seed=s)
+        else:
+            v, nu, dt, thr = oracle_sample_rate(inp, per_step, seed=s)
+        wall = time.perf_counter() - t0
         if s >= args.warmup:
             rates.append(v)
+            walls.append(wall)
             secs += dt
-            rows += nr
+            units += nu
     value = float(np.mean(rates))
-    fl_step = causal_flops(inp.lengths, inp.H, inp.d, inp.d)
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(fl_step / (value * 1e12) * 1e3, 3) if value > 0 else None,
+        "ms_per_step": round(1e3 * float(np.mean(walls)), 3),
+        "ms_per_full_batch_extrapolated": round(fl_batch / (value * 1e12) * 1e3, 3)
+        if value > 0 else None,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded generator; no dataset)",
-        "config": {"workload": cfg["name"], "B": inp.B, "H": inp.H, "d": inp.d,
-                   "total_tokens": inp.T, "parallelism": "host cores"},
+        "config": conf, "launch": "host cores (OpenMP), no GPU",
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
                          "kind": "oracle",
-                         "sample": "%d random query rows over %d steps (%.1f s of fp64 CPU work)"
-                                   % (rows, args.steps, secs)},
+                         "sample": "%d %s over %d steps (%.1f s of fp64 CPU work); each step a "
+                                   "bounded sample of the batch" % (units, what, args.steps, secs)},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
@@ -806,7 +925,9 @@ def parse_args(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", type=int, default=4, choices=[2, 3, 4, 5])
+    ap.add_argument("--config", type=int, default=None, choices=[2, 3, 4, 5],
+                    help="time one workload only (default: the 8192-length workload as the "
+                         "headline line, with the other workloads' lines under 'configs')")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
@@ -847,14 +968,27 @@ def main(argv=None):
                                 device_id=torch.device("cuda", local))
     peaks, kind = load_peaks()
     from gen import CONFIGS
-    if args.backward:
-        line = bench_backward(args, rank, world, local, peaks, kind)
-    elif args.fp8_linear:
-        line = bench_fp8_linear(args, rank, world, local, peaks, kind)
-    elif CONFIGS[args.config]["kind"] == "layer":
-        line = bench_layer(args, rank, world, local, peaks, kind)
+    if args.backward or args.fp8_linear:
+        if args.config is None:
+            args.config = 2 if args.backward else 4
+        fn = bench_backward if args.backward else bench_fp8_linear
+        line = fn(args, rank, world, local, peaks, kind)
+    elif args.config is not None:
+        fn = bench_layer if CONFIGS[args.config]["kind"] == "layer" else bench_attention
+        line = fn(args, rank, world, local, peaks, kind)
     else:
-        line = bench_attention(args, rank, world, local, peaks, kind)
+        # headline: the 8192-length workload; the other workloads' lines,
+        # each timed the same way, under "configs"
+        line = bench_attention(args, rank, world, local, peaks, kind, cfg_id=4)
+        subs = {}
+        for c in (2, 3, 5):
+            fn = bench_layer if CONFIGS[c]["kind"] == "layer" else bench_attention
+            sub = fn(args, rank, world, local, peaks, kind, cfg_id=c,
+                     cpu_budget_s=min(args.cpu_budget_s, 8.0))
+            subs[sub["config"]["workload"]] = sub
+        line["configs"] = subs
+        line["gpu_launches_all_lines"] = line["gpu_launches"] + sum(
+            v["gpu_launches"] for v in subs.values())
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
