@@ -121,7 +121,8 @@ hstu_status_t hstu_attn_plan(const int64_t* seq_offsets, int32_t B, int64_t tota
  *          max_seqlen, H, num_pos or 1) bytes; the run reads the plan's part
  *          and rewrites the bias tables behind it (two launches: the tables,
  *          then the attention)
- * Supported: bf16 with d_qk == d_v in {64, 128}; fp32 with d_qk, d_v <= 128. */
+ * Supported: bf16 with d_qk == d_v in {32, 64, 128} (d = 32 is staged as
+ * 64-column tiles); fp32 with d_qk, d_v <= 128. */
 hstu_status_t hstu_attn_run(hstu_dtype_t dtype,
                             const void* q, int64_t q_tok_stride,
                             const void* k, int64_t k_tok_stride,

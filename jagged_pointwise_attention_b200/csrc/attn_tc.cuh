@@ -59,6 +59,12 @@
 //   the smallest and the largest key timestamp of a 32-key chunk, the bucket
 //   is constant over the chunk and the per-score bucket work is skipped.
 //
+// Head dimension d = 32 is staged as 64-column tiles (the next head's columns,
+// or zeros past the last head): S uses only the first 32 columns of Q and K,
+// and PV computes 64 output columns of which the first 32 are stored.
+//
+// Batches of short sequences take attn_short.cuh instead: one launch, no plan.
+//
 // Every wait is bounded; a wait that runs out raises kErrTimeout, the other
 // roles notice through a shared abort flag, and the CTA drains its own copies
 // and MMAs before it frees TMEM and exits.
@@ -98,12 +104,13 @@ constexpr uint32_t kTmemCols = 512;
 
 template <int D, int G>
 struct AttnCfg {
+    static constexpr int DT = D < 64 ? 64 : D;                         // staged tile width
     static constexpr int kPointwiseWarps = 4 * G;
     static constexpr int kWarpK = 4 * G, kWarpV = 4 * G + 1, kWarpMMA = 4 * G + 2,
                          kWarpPV = 4 * G + 3;
     static constexpr int kThreads = (4 * G + 4) * 32;
-    static constexpr int kStages = D == 64 ? 3 : 2;                     // Q, K and V rings
-    static constexpr int kOBufs = 128 * G + 2 * D <= static_cast<int>(kTmemCols) ? 2 : 1;
+    static constexpr int kStages = DT == 64 ? 3 : 2;                    // Q, K and V rings
+    static constexpr int kOBufs = 128 * G + 2 * DT <= static_cast<int>(kTmemCols) ? 2 : 1;
     static constexpr uint32_t kTmemO = 128 * G;
 };
 
@@ -116,7 +123,8 @@ struct AttnCfg {
 // 16-byte bank slot s mod 8, so the eight consecutive k0 of a quarter warp
 // never conflict. The window depends only on the head and on the tile's
 // diagonal offset (q0 - kt0) / 128, so the tables are built once per launch
-// (bias_prep_kernel) and copied in per tile.
+// (bias_prep_kernel, or per CTA in shared memory by the short-batch kernel)
+// and copied in per tile.
 // Key timestamps are kept relative to `base` (the tile's first key) in 32
 // bits, exact whenever every timestamp involved lies within 2^30 of base:
 // ok[c] says so for the keys of chunk c, and cmin/cmax are the chunk's
@@ -140,10 +148,48 @@ struct alignas(16) BiasStage {
 };
 static_assert(sizeof(BiasStage) == kWinBytes + sizeof(KeySummary), "stage layout");
 
+// R[k] pair as the attention stages it: word m = (R[2m], R[2m+1]) with
+// R[k] = bf16(pos[clamp(base - k)]) / 2 for k <= 254 and R[255] = 0. `row(a)`
+// returns pos[clamp(a, 0, P - 1)] of the head's table.
+template <typename Row>
+__device__ __forceinline__ uint32_t window_word(Row row, int rel0, int m) {
+    const int a = rel0 - 2 * m;
+    const float v0 = row(a);
+    const float v1 = m < 127 ? row(a - 1) : 0.f;
+    uint32_t wd;
+    // bf16(v) / 2 is exactly bf16(v / 2) (a power-of-two scale)
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(wd) : "r"(pack_bf16x2(v0, v1)), "r"(0x3f003f00u));
+    return wd;
+}
+
+// Entry s of the window table of diagonal offset dd: R[s..s+7] as words
+// (R[s+2i], R[s+2i+1]).
+template <typename Row>
+__device__ __forceinline__ uint4 window_entry_of(Row row, int dd, int s) {
+    const int rel0 = 128 * dd + 127;                 // window offset of R[0]
+    const uint32_t sel = (s & 1) ? 0x5432u : 0x3210u;
+    uint32_t x[5];
+#pragma unroll
+    for (int k = 0; k < 5; ++k) x[k] = window_word(row, rel0, (s >> 1) + k);
+    return make_uint4(__byte_perm(x[0], x[1], sel), __byte_perm(x[1], x[2], sel),
+                      __byte_perm(x[2], x[3], sel), __byte_perm(x[3], x[4], sel));
+}
+
+// Entry e of the window tables [H][DD][248], read from the position table in
+// global memory (pos null: the position term is absent, all zeros).
+__device__ __forceinline__ uint4 window_entry(const float* pos, int P, int DD, int64_t e) {
+    const int s = static_cast<int>(e % kWinEntries);
+    const int hd = static_cast<int>(e / kWinEntries);
+    const int h = hd / DD, dd = hd % DD;
+    if (pos == nullptr) return make_uint4(0u, 0u, 0u, 0u);
+    const float* prow = pos + static_cast<int64_t>(h) * P;
+    return window_entry_of([&](int a) { return __ldg(prow + min(max(a, 0), P - 1)); }, dd, s);
+}
+
 template <int D, int G>
 struct AttnSmem {
     using C = AttnCfg<D, G>;
-    static constexpr int kTileBytes = kTile * D * 2;                    // one Q, K or V tile
+    static constexpr int kTileBytes = kTile * C::DT * 2;                // one Q, K or V tile
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + C::kStages * kTileBytes;
     static constexpr int kOffV = kOffK + C::kStages * kTileBytes;
@@ -389,13 +435,14 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                      const __grid_constant__ CUtensorMap tmV, const AttnArgs args) {
     using C = AttnCfg<D, G>;
     using L = AttnSmem<D, G>;
+    constexpr int DT = C::DT;
     constexpr int S = C::kStages;
     constexpr int OB = C::kOBufs;
-    constexpr int kKB = D / 64;   // 64-element (128-byte) column blocks per row
+    constexpr int kKB = DT / 64;   // 64-element (128-byte) column blocks per row
     constexpr int kTileBytes = L::kTileBytes;
-    static_assert(D == 64 || D == 128, "head dim");
+    static_assert(D == 32 || D == 64 || D == 128, "head dim");
     static_assert(G >= 1 && G <= 3 && S <= 3 && OB <= 2, "barrier map");
-    static_assert(128 * G + OB * D <= static_cast<int>(kTmemCols), "TMEM budget");
+    static_assert(128 * G + OB * DT <= static_cast<int>(kTmemCols), "TMEM budget");
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -640,7 +687,7 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                 if (!mbar_wait(&bars[kBarDrain], 0, nullptr)) raise_error(kErrTimeout);
             } else {
                 // ---- PV_n: O += P V, A operand (P) from TMEM
-                constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+                constexpr uint32_t idesc_pv = idesc_bf16_f32(128, DT, 0, 1);
                 const uint64_t dv0 = desc_mnmajor_sw128(sV, 16384);
                 for (int it = 0; ok; ++it) {
                     Item I;
@@ -665,7 +712,7 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                         tc_fence_after();
                         const uint64_t dv = dv0 + static_cast<uint64_t>(vs * kStageDesc);
                         const uint32_t pb = tmem + b * 128;
-                        const uint32_t dst = tmem + C::kTmemO + ob * D;
+                        const uint32_t dst = tmem + C::kTmemO + ob * DT;
 #pragma unroll
                         for (int kk = 0; kk < kTile / 16; ++kk) {
                             // keys 16kk..16kk+15: columns 32*(kk/2) + 8*(kk%2) of the P buffer
@@ -824,7 +871,7 @@ attn_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ,
                         for (int ch = 0; ch < D / 32; ++ch) {
                             uint32_t ov[32];
                             __syncwarp();
-                            tmem_ld32(tmem + lane_base + C::kTmemO + ob * D + ch * 32, ov);
+                            tmem_ld32(tmem + lane_base + C::kTmemO + ob * DT + ch * 32, ov);
                             if (row_valid) {
                                 uint32_t wv[16];
 #pragma unroll

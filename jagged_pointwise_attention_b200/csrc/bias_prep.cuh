@@ -42,19 +42,6 @@ struct BiasPrepArgs {
     int table_blocks;           // blocks [0, table_blocks) build tables, the rest one unit each
 };
 
-// R[k] pair as the attention stages it: word m = (R[2m], R[2m+1]) with
-// R[k] = bf16(pos[clamp(base - k)]) / 2 for k <= 254 and R[255] = 0.
-__device__ __forceinline__ uint32_t window_word(const float* prow, int P, int rel0, int m) {
-    if (prow == nullptr) return 0u;
-    const int a = rel0 - 2 * m;
-    const float v0 = __ldg(prow + min(max(a, 0), P - 1));
-    const float v1 = m < 127 ? __ldg(prow + min(max(a - 1, 0), P - 1)) : 0.f;
-    uint32_t wd;
-    // bf16(v) / 2 is exactly bf16(v / 2) (a power-of-two scale)
-    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(wd) : "r"(pack_bf16x2(v0, v1)), "r"(0x3f003f00u));
-    return wd;
-}
-
 // Programmatic launch chain plan -> bias prep -> attention. The attention
 // waits (griddepcontrol.wait) only for this grid, its direct prerequisite, so
 // this grid must not complete before the plan has: every block of it executes
@@ -68,19 +55,8 @@ __global__ void __launch_bounds__(128) bias_prep_kernel(const BiasPrepArgs a) {
     if (static_cast<int>(blockIdx.x) < a.table_blocks) {
         // entry s of table (h, dd) holds R[s..s+7]: words (R[s+2i], R[s+2i+1])
         const int64_t e = static_cast<int64_t>(blockIdx.x) * 128 + tid;
-        if (e < static_cast<int64_t>(a.H) * a.DD * kWinEntries) {
-            const int s = static_cast<int>(e % kWinEntries);
-            const int hd = static_cast<int>(e / kWinEntries);
-            const int h = hd / a.DD, dd = hd % a.DD;
-            const float* prow = a.pos ? a.pos + static_cast<int64_t>(h) * a.P : nullptr;
-            const int rel0 = 128 * dd + 127;                 // window offset of R[0]
-            const uint32_t sel = (s & 1) ? 0x5432u : 0x3210u;
-            uint32_t x[5];
-#pragma unroll
-            for (int k = 0; k < 5; ++k) x[k] = window_word(prow, a.P, rel0, (s >> 1) + k);
-            a.ptab[e] = make_uint4(__byte_perm(x[0], x[1], sel), __byte_perm(x[1], x[2], sel),
-                                   __byte_perm(x[2], x[3], sel), __byte_perm(x[3], x[4], sel));
-        }
+        if (e < static_cast<int64_t>(a.H) * a.DD * kWinEntries)
+            a.ptab[e] = window_entry(a.pos, a.P, a.DD, e);
         asm volatile("griddepcontrol.wait;" ::: "memory");   // complete only after the plan
         return;
     }

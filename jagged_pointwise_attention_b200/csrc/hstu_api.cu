@@ -195,7 +195,8 @@ hstu_status_t validate_attn(const AttnCall& c) {
     if (c.pos && c.P < 1) return HSTU_ERR_INVALID_ARG;
     if (c.tb && (c.NB < 1 || c.NB > kMaxTimeBuckets)) return HSTU_ERR_INVALID_ARG;
     if (c.dtype == HSTU_DTYPE_BF16) {
-        if (c.dqk != c.dv || (c.dqk != 64 && c.dqk != 128)) return HSTU_ERR_UNSUPPORTED;
+        if (c.dqk != c.dv || (c.dqk != 32 && c.dqk != 64 && c.dqk != 128))
+            return HSTU_ERR_UNSUPPORTED;
         if (!aligned16(c.q) || !aligned16(c.k) || !aligned16(c.v) || !aligned16(c.out))
             return HSTU_ERR_INVALID_ARG;
         if (c.qs % 8 || c.ks % 8 || c.vs % 8 || c.os % 8) return HSTU_ERR_INVALID_ARG;
@@ -232,6 +233,22 @@ hstu_status_t launch_attn_pdl(Kernel kernel, unsigned grid, int threads, size_t 
     return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
 }
 
+// The plan kernel: the longest-first work list into the workspace's plan part.
+hstu_status_t launch_plan(const int64_t* off, int32_t B, int64_t T, int32_t max_seqlen, void* ws,
+                          cudaStream_t stream) {
+    const int max_tiles = max_tiles_of(max_seqlen);
+    const int64_t max_units = max_units_of(B, T, max_seqlen);
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    size_t smem = static_cast<size_t>((3 * (max_tiles + 1) + 1) & ~1) * sizeof(int);
+    if (B < kPlanSmemOffsets) smem += static_cast<size_t>(B + 1) * sizeof(int64_t);
+    plan_kernel<<<1, 1024, smem, stream>>>(
+        off, B, T, max_seqlen, max_tiles, static_cast<int>(max_units),
+        reinterpret_cast<int4*>(w + kAttnWsHeader),
+        reinterpret_cast<uint4*>(w + kAttnWsHeader + attn_units_bytes(B, T, max_seqlen)),
+        reinterpret_cast<int*>(w), reinterpret_cast<int*>(w + 16));
+    return launch_status();
+}
+
 hstu_status_t run_attn(const AttnCall& c) {
     const hstu_status_t st = validate_attn(c);
     if (st != HSTU_OK || c.B == 0 || c.T == 0) return st;
@@ -255,10 +272,11 @@ hstu_status_t run_attn(const AttnCall& c) {
         !make_tmap_bf16(&tk, c.k, inner, c.T, c.ks * 2, 128) ||
         !make_tmap_bf16(&tv, c.v, inner, c.T, c.vs * 2, 128))
         return HSTU_ERR_CUDA;
-    const int64_t max_units = max_units_of(c.B, c.T, c.max_seqlen);
     uint8_t* ws = static_cast<uint8_t*>(c.ws);
     const int P = c.pos ? c.P : 1;
     const int DD = attn_window_tables(P, c.max_seqlen);
+    constexpr int G = kAttnGroups;
+    const int64_t max_units = max_units_of(c.B, c.T, c.max_seqlen);
     uint4* ptab = reinterpret_cast<uint4*>(ws + attn_plan_bytes(c.B, c.T, c.max_seqlen));
     KeySummary* ksum = reinterpret_cast<KeySummary*>(
         ws + attn_plan_bytes(c.B, c.T, c.max_seqlen) + attn_tables_bytes(c.H, P, c.max_seqlen));
@@ -295,7 +313,7 @@ hstu_status_t run_attn(const AttnCall& c) {
                c.T,
                use_time ? c.ts : nullptr,
                c.pos,
-               c.pos ? c.P : 1,
+               P,
                use_time ? c.tb : nullptr,
                use_time ? c.NB : 0,
                inv_n,
@@ -305,20 +323,30 @@ hstu_status_t run_attn(const AttnCall& c) {
     if (items > 0x7fffffff) return HSTU_ERR_UNSUPPORTED;
     // persistent: one CTA per SM, work items dealt round-robin
     const unsigned grid = static_cast<unsigned>(items < num_sms() ? items : num_sms());
-    constexpr int G = kAttnGroups;
-    static int smem_done64[kMaxDevices] = {0}, smem_done128[kMaxDevices] = {0};
-    if (c.dqk == 64) {
-        if (!ensure_smem(attn_fwd_bf16_kernel<64, G>, AttnSmem<64, G>::kAlloc, smem_done64))
+    static int smem_done32[kMaxDevices] = {0}, smem_done64[kMaxDevices] = {0},
+               smem_done128[kMaxDevices] = {0};
+    if (c.dqk == 32) {
+        if (!ensure_smem(attn_fwd_bf16_kernel<32, G>, AttnSmem<32, G>::kAlloc,
+                         smem_done32))
             return HSTU_ERR_CUDA;
-        return launch_attn_pdl(attn_fwd_bf16_kernel<64, G>, grid, AttnCfg<64, G>::kThreads,
-                               AttnSmem<64, G>::kAlloc, c.stream, tq, tk, tv, a);
-    } else {
-        if (!ensure_smem(attn_fwd_bf16_kernel<128, G>, AttnSmem<128, G>::kAlloc, smem_done128))
-            return HSTU_ERR_CUDA;
-        return launch_attn_pdl(attn_fwd_bf16_kernel<128, G>, grid, AttnCfg<128, G>::kThreads,
-                                AttnSmem<128, G>::kAlloc, c.stream, tq, tk, tv, a);
+        return launch_attn_pdl(attn_fwd_bf16_kernel<32, G>, grid,
+                               AttnCfg<32, G>::kThreads, AttnSmem<32, G>::kAlloc,
+                               c.stream, tq, tk, tv, a);
     }
-    return launch_status();
+    if (c.dqk == 64) {
+        if (!ensure_smem(attn_fwd_bf16_kernel<64, G>, AttnSmem<64, G>::kAlloc,
+                         smem_done64))
+            return HSTU_ERR_CUDA;
+        return launch_attn_pdl(attn_fwd_bf16_kernel<64, G>, grid,
+                               AttnCfg<64, G>::kThreads, AttnSmem<64, G>::kAlloc,
+                               c.stream, tq, tk, tv, a);
+    }
+    if (!ensure_smem(attn_fwd_bf16_kernel<128, G>, AttnSmem<128, G>::kAlloc,
+                     smem_done128))
+        return HSTU_ERR_CUDA;
+    return launch_attn_pdl(attn_fwd_bf16_kernel<128, G>, grid,
+                           AttnCfg<128, G>::kThreads, AttnSmem<128, G>::kAlloc,
+                           c.stream, tq, tk, tv, a);
 }
 
 hstu_status_t plan_attn(const int64_t* off, int32_t B, int64_t T, int32_t max_seqlen, void* ws,
@@ -327,17 +355,7 @@ hstu_status_t plan_attn(const int64_t* off, int32_t B, int64_t T, int32_t max_se
     if (B == 0 || T == 0) return HSTU_OK;
     if (!off || !ws || !aligned16(ws) || ws_bytes < attn_plan_bytes(B, T, max_seqlen))
         return HSTU_ERR_INVALID_ARG;
-    const int max_tiles = max_tiles_of(max_seqlen);
-    const int64_t max_units = max_units_of(B, T, max_seqlen);
-    uint8_t* w = static_cast<uint8_t*>(ws);
-    size_t smem = static_cast<size_t>((3 * (max_tiles + 1) + 1) & ~1) * sizeof(int);
-    if (B < kPlanSmemOffsets) smem += static_cast<size_t>(B + 1) * sizeof(int64_t);
-    plan_kernel<<<1, 1024, smem, stream>>>(
-        off, B, T, max_seqlen, max_tiles, static_cast<int>(max_units),
-        reinterpret_cast<int4*>(w + kAttnWsHeader),
-        reinterpret_cast<uint4*>(w + kAttnWsHeader + attn_units_bytes(B, T, max_seqlen)),
-        reinterpret_cast<int*>(w), reinterpret_cast<int*>(w + 16));
-    return launch_status();
+    return launch_plan(off, B, T, max_seqlen, ws, stream);
 }
 
 template <int EPI, int BN, bool FP8 = false>

@@ -96,6 +96,11 @@ def test_attention_argument_validation(lib):
     assert _attn(lib, q=24) == INV                        # misaligned base
     assert _attn(lib, dqk=96, dv=96, qs=384, ks=384, vs=384, os=384) == UNS
     assert _attn(lib, dv=64, vs=256, os=256) == UNS       # d_qk != d_v on bf16
+    # bf16 takes d in {32, 64, 128}: d = 32 gets past the head-dimension check
+    # (and fails later, on the workspace), d = 48 does not
+    d32 = dict(dqk=32, dv=32, qs=128, ks=128, vs=128, os=128)
+    assert _attn(lib, wsb=64, **d32) == INV
+    assert _attn(lib, dqk=48, dv=48, qs=192, ks=192, vs=192, os=192, wsb=64) == UNS
     assert _attn(lib, ws=None) == INV
     assert _attn(lib, wsb=64) == INV                      # workspace too small
     assert _attn(lib, tb=16, NB=0) == INV

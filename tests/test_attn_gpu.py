@@ -257,3 +257,147 @@ def test_time_bucket_of_every_pair(d):
         bad = np.argwhere(err > bound)
         assert bad.size == 0, "key tile %d: %d outputs off, first (token, head, col) %s: %g vs %g" % (
             kt, len(bad), bad[0].tolist(), got[tuple(bad[0])], want[tuple(bad[0])])
+
+
+# ----------------------------------------------------------------- short sequences, d = 32
+#
+# Batches of sequences of at most 256 tokens: packed tiles of several short
+# sequences next to the one- and two-tile units of sequences of 129..256
+# tokens, empty and one-token sequences, many sequences starting in one
+# 128-token stretch of the batch, and head dimension 32 (staged as 64-column
+# tiles).
+
+
+@pytest.mark.parametrize("d", [32, 64])
+def test_short_batch_ragged(d):
+    lens = [0, 1, 5, 128, 0, 129, 7, 127, 2, 256, 64, 64, 1, 0, 200, 33, 95, 1]
+    inp = custom_attn_inputs(lens, H=3, d=d, num_pos=300, num_buckets=64, seed=30 + d,
+                             bias_std=0.5)
+    assert inp.max_seqlen <= 256
+    assert_bf16_close(run_gpu(inp), run_oracle(inp), "short ragged d=%d" % d)
+
+
+def test_short_batch_many_tiny_sequences():
+    # more than 32 sequences start in some 128-token buckets
+    rng = np.random.default_rng(31)
+    lens = rng.integers(0, 4, size=3000)
+    inp = custom_attn_inputs(lens, H=2, d=64, num_pos=8, num_buckets=16, seed=31, bias_std=0.5)
+    assert_bf16_close(run_gpu(inp), run_oracle(inp), "tiny sequences")
+
+
+def test_short_batch_d128():
+    lens = [3, 200, 0, 90, 129]
+    inp = custom_attn_inputs(lens, H=2, d=128, num_pos=256, num_buckets=32, seed=32)
+    assert_bf16_close(run_gpu(inp), run_oracle(inp), "short batch d=128")
+
+
+def test_short_batch_huge_timestamps_clip_and_clamp():
+    lens = [200, 50, 1, 129]
+    inp = custom_attn_inputs(lens, H=2, d=64, num_pos=17, num_buckets=6, seed=33, bias_std=0.5)
+    rng = np.random.default_rng(33)
+    inp.timestamps = rng.integers(-(2 ** 40), 2 ** 40, size=inp.T).astype(np.int64)
+    assert_bf16_close(run_gpu(inp), run_oracle(inp), "short: huge timestamps, clip, clamp")
+
+
+@pytest.mark.parametrize("d", [32, 64])
+def test_short_batch_terms_dropped(d):
+    inp = custom_attn_inputs([17, 200, 3, 128, 90], H=2, d=d, num_pos=256, num_buckets=32,
+                             seed=34, bias_std=0.5)
+    got = run_gpu(inp, timestamps=None)
+    assert_bf16_close(got, run_oracle(inp, timestamps=None, time_bias=None), "no time")
+    got = run_gpu(inp, pos_bias=None, time_bias=None)
+    assert_bf16_close(got, run_oracle(inp, pos_bias=None, time_bias=None), "no bias")
+
+
+def test_short_batch_plan_reuse_and_sequence_independence():
+    """One plan serves several runs (the run re-arms its item counter), and a
+    sequence gives the same rows (within rounding of the packing) alone and in
+    the batch."""
+    inp = make_attn_inputs(3, max_batch=300)
+    t = attn_tensors(inp)
+    ws = torch.empty(hstu.hstu_attn_workspace_bytes(inp.B, inp.T, inp.max_seqlen, inp.H,
+                                                    inp.pos_bias.shape[1]),
+                     dtype=torch.uint8, device="cuda")
+    hstu.hstu_attn_plan(t["seq_offsets"], inp.max_seqlen, inp.T, ws)
+    outs = []
+    for _ in range(3):
+        out = torch.full_like(t["q"], float("nan"))
+        hstu.hstu_attn_run(t["q"], t["k"], t["v"], t["seq_offsets"], t["timestamps"],
+                           t["pos_bias"], t["time_bias"], inp.max_seqlen, out, ws)
+        outs.append(out.float().cpu().numpy())
+    assert hstu.hstu_device_status() == 0
+    assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[0], outs[2])
+    assert_bf16_close(outs[0], run_oracle(inp), "short batch, planned once")
+    off = inp.seq_offsets
+    for s in (0, 7, 151):
+        sl = slice(int(off[s]), int(off[s + 1]))
+        alone = hstu.hstu_attn_fwd(t["q"][sl], t["k"][sl], t["v"][sl],
+                                   dev(np.array([0, int(off[s + 1] - off[s])], np.int64)),
+                                   t["timestamps"][sl], t["pos_bias"], t["time_bias"],
+                                   inp.max_seqlen)
+        assert_bf16_close(alone.float().cpu().numpy(), outs[0][sl], "sequence %d alone" % s)
+
+
+def test_time_bucket_of_every_pair_short_batch():
+    """As test_time_bucket_of_every_pair, on a batch of short sequences (packed
+    tiles and the aligned tiles of sequences of 129..256 tokens)."""
+    lens = [256, 90, 33, 1, 129, 70, 200]
+    H, NB, d = 2, 32, 64
+    inp = custom_attn_inputs(lens, H=H, d=d, num_pos=8, num_buckets=NB, seed=35)
+    off = inp.seq_offsets
+    last = slice(int(off[-2]), int(off[-1]))
+    inp.timestamps[last] = np.cumsum(np.full(lens[-1], 1 << 26, np.int64)) + (1 << 40)
+    inp.q[:] = 0
+    inp.k[:] = 0
+    inp.pos_bias[:] = 0
+    b = np.arange(NB, dtype=np.float32)
+    inp.time_bias[0] = 1.0 + 0.75 * b
+    inp.time_bias[1] = 2.0 + 0.5 * b
+    T = inp.T
+    pos_in_seq = np.arange(T) - np.repeat(off[:-1], np.diff(off))
+    for kt in range(2):
+        v = np.zeros((T, H, d), np.float32)
+        sel = (pos_in_seq >= 128 * kt) & (pos_in_seq < 128 * kt + 128)
+        v[np.nonzero(sel)[0], :, (pos_in_seq[sel] - 128 * kt) % d] = 1.0
+        inp.v = v
+        got = run_gpu(inp, v=dev(v, torch.bfloat16))
+        want = run_oracle(inp)
+        err = np.abs(got - want)
+        bad = np.argwhere(err > 0.015 * np.abs(want) + 1e-6)
+        assert bad.size == 0, "key tile %d: %d outputs off, first %s" % (kt, len(bad), bad[0].tolist())
+
+
+@pytest.mark.parametrize("d", [32])
+def test_planned_d32_multi_tile(d):
+    lens = [1, 127, 128, 129, 300, 0, 513, 64, 255, 256, 2]
+    inp = custom_attn_inputs(lens, H=3, d=d, num_pos=400, num_buckets=128, dtype="bf16", seed=36)
+    assert_bf16_close(run_gpu(inp), run_oracle(inp), "ragged d=32 (planned)")
+
+
+# ----------------------------------------------------------------- the bias terms are seen
+
+
+@pytest.mark.parametrize("cfg", [2, 4])
+def test_workload_output_sees_the_bias_terms(cfg):
+    """With the workloads' N(0, 0.02^2) tables each bias term moves the output
+    by about as much as the bf16 rounding of the pointwise stage does (both
+    near 3e-3 relative), so a kernel that dropped a term could still pass the
+    rel-Frobenius bar. Here the GPU output must be measurably closer to the
+    oracle with both terms than to the oracle without them: its error must be
+    at most 0.90 times its distance to the oracle without either term, and at
+    most 0.95 times its distance to the oracle without the position term and
+    to the one without the time term. A kernel that dropped a term would sit
+    above 1.0 against the oracle without that term (its error is the rounding
+    noise plus the term's effect, its distance the noise alone)."""
+    inp = make_attn_inputs(cfg)
+    got = run_gpu(inp)
+    rows = np.arange(inp.T) if cfg == 2 else sampled_rows(inp.seq_offsets, n_random=256, seed=4)
+    g = got[rows].astype(np.float64)
+    want = run_oracle(inp, rows=rows)
+    err = np.linalg.norm(g - want)
+    for name, over, bar in [("without either term", dict(pos_bias=None, time_bias=None), 0.90),
+                            ("without the position term", dict(pos_bias=None), 0.95),
+                            ("without the time term", dict(time_bias=None), 0.95)]:
+        dist = np.linalg.norm(g - run_oracle(inp, rows=rows, **over))
+        assert err <= bar * dist, "config %d: error %.4g, distance %.4g to the oracle %s" % (
+            cfg, err, dist, name)
