@@ -58,8 +58,11 @@ def _bind(lib):
     lib.hstu_oracle_layernorm_gate.restype = None
     lib.hstu_oracle_layernorm_gate.argtypes = [_i64, _i32, _p, _i64, _p, _i64, _p, _p, _f64, _p]
     lib.hstu_oracle_layer.restype = ctypes.c_int
-    lib.hstu_oracle_layer.argtypes = [_i64, _i32, _p, _p, _p, _p, _p, _p, _p, _f64, _p, _i32,
-                                      _i32, _i32, _p, _p, _i32, _p, _i32, _i32, _p, _i64, _p]
+    lib.hstu_oracle_layer.argtypes = [_i64, _i32, _p, _p, _p, _p, _p, _p, _p, _f64, _p, _p,
+                                      _i32, _p, _i32, _i32, _i32, _p, _p, _i32, _p, _i32, _i32,
+                                      _p, _i64, _p]
+    lib.hstu_oracle_layernorm.restype = None
+    lib.hstu_oracle_layernorm.argtypes = [_i64, _i32, _p, _i64, _p, _p, _f64, _p]
     lib.hstu_oracle_e4m3_to_float.restype = ctypes.c_float
     lib.hstu_oracle_e4m3_to_float.argtypes = [ctypes.c_uint8]
     lib.hstu_oracle_e4m3_from_float.restype = ctypes.c_uint8
@@ -250,11 +253,24 @@ def layernorm_gate(a, u, gamma=None, beta=None, eps: float = 1e-5, lib=None) -> 
     return y[:M]
 
 
+def layernorm(a, gamma=None, beta=None, eps: float = 1e-5, lib=None) -> np.ndarray:
+    """LayerNorm over the last axis in fp64 (biased variance, eps inside the
+    square root, affine gamma / beta or identity). a: [M, F]."""
+    lib = lib or load()
+    a, gamma, beta = _f64a(a), _f64a(gamma), _f64a(beta)
+    M, F = a.shape
+    y = np.zeros((max(M, 1), F), dtype=np.float64)
+    lib.hstu_oracle_layernorm(M, F, _ptr(a), F, _ptr(gamma), _ptr(beta), float(eps), _ptr(y))
+    return y[:M]
+
+
 def layer(seq_offsets, x, W1, W2, H: int, d: int, timestamps, pos_bias, time_bias,
           max_seqlen: int, b1=None, b2=None, ln_gamma=None, ln_beta=None,
-          ln_eps: float = 1e-5, rows: Optional[Sequence[int]] = None, lib=None) -> np.ndarray:
+          ln_eps: float = 1e-5, rows: Optional[Sequence[int]] = None, lib=None,
+          input_norm: bool = False, in_gamma=None, in_beta=None) -> np.ndarray:
     """HSTU layer forward in fp64: x + (LayerNorm(attn(Q,K,V)) * U) W2^T + b2 with
-    U|V|Q|K = silu(x W1^T + b1). Returns [T,D] or [len(rows),D]."""
+    U|V|Q|K = silu(x' W1^T + b1), x' = x or, with input_norm, LayerNorm(x)
+    (affine in_gamma / in_beta, the same eps). Returns [T,D] or [len(rows),D]."""
     lib = lib or load()
     off = _i64a(seq_offsets)
     x, W1, W2 = _f64a(x), _f64a(W1), _f64a(W2)
@@ -266,8 +282,10 @@ def layer(seq_offsets, x, W1, W2, H: int, d: int, timestamps, pos_bias, time_bia
     r = None if rows is None else _i64a(rows)
     n = T if r is None else r.shape[0]
     out = np.zeros((max(n, 1), D), dtype=np.float64)
+    ig, ib = _f64a(in_gamma), _f64a(in_beta)
     rc = lib.hstu_oracle_layer(T, D, _ptr(x), _ptr(W1), _ptr(b1), _ptr(W2), _ptr(b2), _ptr(g),
-                               _ptr(bt), float(ln_eps), _ptr(off), len(off) - 1, H, d, _ptr(ts),
+                               _ptr(bt), float(ln_eps), _ptr(ig), _ptr(ib), 1 if input_norm else 0,
+                               _ptr(off), len(off) - 1, H, d, _ptr(ts),
                                _ptr(pos), P, _ptr(tb), NB, int(max_seqlen), _ptr(r),
                                0 if r is None else n, _ptr(out))
     if rc != 0:

@@ -334,38 +334,55 @@ void hstu_oracle_linear_fp8(int64_t M, int32_t K, int32_t N, const uint8_t* xq,
     }
 }
 
-/* y[m, :] = LayerNorm(a[m, :]) * u[m, :] over F features: biased variance,
- * eps inside the square root, then gamma / beta (NULL = 1 / 0).
- * a, u, y have row strides a_ld, u_ld, F. */
+/* One row of LayerNorm over F features: biased variance, eps inside the
+ * square root, then gamma / beta (NULL = 1 / 0). */
+static void ln_row(const double* ar, int32_t F, const double* gamma, const double* beta,
+                   double eps, double* yr) {
+    double mean = 0.0;
+    for (int32_t c = 0; c < F; ++c) mean += ar[c];
+    mean /= (double)F;
+    double var = 0.0;
+    for (int32_t c = 0; c < F; ++c) var += (ar[c] - mean) * (ar[c] - mean);
+    var /= (double)F;
+    double rstd = 1.0 / sqrt(var + eps);
+    for (int32_t c = 0; c < F; ++c)
+        yr[c] = (ar[c] - mean) * rstd * (gamma ? gamma[c] : 1.0) + (beta ? beta[c] : 0.0);
+}
+
+/* y[m, :] = LayerNorm(a[m, :]) * u[m, :] over F features (ln_row), a, u, y
+ * with row strides a_ld, u_ld, F. */
 void hstu_oracle_layernorm_gate(int64_t M, int32_t F, const double* a, int64_t a_ld,
                                 const double* u, int64_t u_ld, const double* gamma,
                                 const double* beta, double eps, double* y) {
 #pragma omp parallel for schedule(static)
     for (int64_t m = 0; m < M; ++m) {
-        const double* ar = a + m * a_ld;
-        double mean = 0.0;
-        for (int32_t c = 0; c < F; ++c) mean += ar[c];
-        mean /= (double)F;
-        double var = 0.0;
-        for (int32_t c = 0; c < F; ++c) var += (ar[c] - mean) * (ar[c] - mean);
-        var /= (double)F;
-        double rstd = 1.0 / sqrt(var + eps);
-        for (int32_t c = 0; c < F; ++c) {
-            double g = gamma ? gamma[c] : 1.0;
-            double bt = beta ? beta[c] : 0.0;
-            y[m * F + c] = ((ar[c] - mean) * rstd * g + bt) * u[m * u_ld + c];
-        }
+        ln_row(a + m * a_ld, F, gamma, beta, eps, y + m * F);
+        for (int32_t c = 0; c < F; ++c) y[m * F + c] *= u[m * u_ld + c];
     }
+}
+
+/* y[m, :] = LayerNorm(a[m, :]) over F features (ln_row); a has row stride
+ * a_ld, y row stride F. The layer's input normalization (generative-
+ * recommenders README, "HSTU Ultra attention benchmark": input norm before
+ * the UVQK projection). */
+void hstu_oracle_layernorm(int64_t M, int32_t F, const double* a, int64_t a_ld,
+                           const double* gamma, const double* beta, double eps, double* y) {
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) ln_row(a + m * a_ld, F, gamma, beta, eps, y + m * F);
 }
 
 /* Full layer forward for the requested rows (rows == NULL: every token).
  * x [T,D], W1 [4Hd,D] (output columns U|V|Q|K), W2 [D,Hd]; out [n,D].
+ * With input_norm, the projection reads LayerNorm(x) (over D features, the
+ * output norm's eps, affine in_gamma / in_beta, NULL = identity); the
+ * residual adds x itself.
  * Only the prefix of each touched sequence up to its last requested row is
  * projected, since later tokens cannot reach a requested row.
  * Returns 0, -1 for a bad row, -2 on allocation failure. */
 int hstu_oracle_layer(int64_t T, int32_t D, const double* x, const double* W1,
                       const double* b1, const double* W2, const double* b2,
                       const double* gamma, const double* beta, double eps,
+                      const double* in_gamma, const double* in_beta, int32_t input_norm,
                       const int64_t* seq_offsets, int32_t B, int32_t H, int32_t d,
                       const int64_t* ts, const double* pos, int32_t num_pos,
                       const double* tbias, int32_t num_buckets, int32_t max_seqlen,
@@ -378,8 +395,18 @@ int hstu_oracle_layer(int64_t T, int32_t D, const double* x, const double* W1,
     double* ygate = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1) * (size_t)F);
     double* urow = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1) * (size_t)F);
     double* xrow = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1) * (size_t)D);
+    double* xn = input_norm ? (double*)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1) * (size_t)D)
+                            : NULL;
+    const double* xin = x;
     int rc = 0;
-    if (!upto || !uvqk || !attn || !ygate || !urow || !xrow) { rc = -2; goto done; }
+    if (!upto || !uvqk || !attn || !ygate || !urow || !xrow || (input_norm && !xn)) {
+        rc = -2;
+        goto done;
+    }
+    if (input_norm) {
+        hstu_oracle_layernorm(T, D, x, D, in_gamma, in_beta, eps, xn);
+        xin = xn;
+    }
     for (int32_t b = 0; b < B; ++b) upto[b] = seq_offsets[b];  /* exclusive end */
     for (int64_t r = 0; r < n; ++r) {
         int64_t t = rows ? rows[r] : r;
@@ -387,11 +414,11 @@ int hstu_oracle_layer(int64_t T, int32_t D, const double* x, const double* W1,
         if (b < 0) { rc = -1; goto done; }
         if (t + 1 > upto[b]) upto[b] = t + 1;
     }
-    /* 1. UVQK = silu(x W1^T + b1) for each needed prefix */
+    /* 1. UVQK = silu(x W1^T + b1), x normalized or not, for each needed prefix */
     for (int32_t b = 0; b < B; ++b) {
         int64_t o = seq_offsets[b], m = upto[b] - o;
         if (m > 0)
-            hstu_oracle_linear(m, D, (int32_t)W, x + o * D, W1, b1, 1, NULL, uvqk + o * W);
+            hstu_oracle_linear(m, D, (int32_t)W, xin + o * D, W1, b1, 1, NULL, uvqk + o * W);
     }
     /* 2. attention with U|V|Q|K views of the projection (token stride 4Hd) */
     rc = hstu_oracle_attn(seq_offsets, B, H, d, d, uvqk + 2 * F, W, uvqk + 3 * F, W,
@@ -411,7 +438,7 @@ int hstu_oracle_layer(int64_t T, int32_t D, const double* x, const double* W1,
     }
     hstu_oracle_linear(n, (int32_t)F, D, ygate, W2, b2, 0, xrow, out);
 done:
-    free(upto); free(uvqk); free(attn); free(ygate); free(urow); free(xrow);
+    free(upto); free(uvqk); free(attn); free(ygate); free(urow); free(xrow); free(xn);
     return rc;
 }
 

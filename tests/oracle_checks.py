@@ -408,6 +408,44 @@ def check_layer_composition(lib):
                         ln_beta=bt, rows=rows, lib=lib), got[rows], 0, "layer rows")
 
 
+def check_layernorm(lib):
+    """The input LayerNorm against torch.layer_norm (a library routine), with
+    and without the affine parameters."""
+    rng = np.random.default_rng(11)
+    a = rng.standard_normal((7, 24)) * 2.5 - 0.7
+    g = 1 + rng.standard_normal(24) * 0.2
+    bt = rng.standard_normal(24) * 0.2
+    t = torch.from_numpy(a)
+    _close(oracle.layernorm(a, g, bt, 1e-5, lib=lib),
+           torch.nn.functional.layer_norm(t, (24,), torch.from_numpy(g), torch.from_numpy(bt),
+                                          eps=1e-5).numpy(), what="layernorm affine")
+    _close(oracle.layernorm(a, eps=1e-3, lib=lib),
+           torch.nn.functional.layer_norm(t, (24,), eps=1e-3).numpy(), what="layernorm")
+
+
+def check_layer_input_norm(lib):
+    """The layer with an input LayerNorm: the projection reads LayerNorm(x),
+    the residual adds x itself (torch composition with the dense reference)."""
+    off, x, W1, W2, H, d, ts, pos, tb, N = _tiny_layer(seed=4)
+    T, D = x.shape
+    F = H * d
+    rng = np.random.default_rng(6)
+    ig, ib = 1 + rng.standard_normal(D) * 0.2, rng.standard_normal(D) * 0.2
+    got = oracle.layer(off, x, W1, W2, H, d, ts, pos, tb, N, ln_eps=1e-5, lib=lib,
+                       input_norm=True, in_gamma=ig, in_beta=ib)
+    xn = torch.nn.functional.layer_norm(torch.from_numpy(x), (D,), torch.from_numpy(ig),
+                                        torch.from_numpy(ib), eps=1e-5).numpy()
+    uvqk = _silu_t(xn @ W1.T)
+    U, V, Q, K = (uvqk[:, i * F:(i + 1) * F].reshape(T, H, d) for i in range(4))
+    A = dense_reference(off, Q, K, V, ts, pos, tb, N).reshape(T, F)
+    Y = torch.nn.functional.layer_norm(torch.from_numpy(A), (F,), eps=1e-5).numpy() * U.reshape(T, F)
+    _close(got, x + Y @ W2.T, what="layer with input norm")
+    rows = [T - 1, 0, 6]
+    _close(oracle.layer(off, x, W1, W2, H, d, ts, pos, tb, N, ln_eps=1e-5, rows=rows, lib=lib,
+                        input_norm=True, in_gamma=ig, in_beta=ib), got[rows], 0,
+           "layer with input norm, rows")
+
+
 def check_layer_identities(lib):
     off, x, W1, W2, H, d, ts, pos, tb, N = _tiny_layer(seed=3)
     F = H * d
@@ -650,7 +688,8 @@ ALL_CHECKS = [
     check_batch_independence, check_rows_subset, check_empty_and_length_one,
     check_closed_form_prefix_sum, check_time_only_closed_form, check_pos_only_toeplitz,
     check_scale_is_max_seqlen, check_qk_asymmetry, check_linear, check_layernorm_gate,
-    check_layer_composition, check_layer_identities, check_e4m3_table,
+    check_layer_composition, check_layer_identities, check_layernorm, check_layer_input_norm,
+    check_e4m3_table,
     check_e4m3_rounding_against_torch, check_e4m3_saturation, check_quant_rows, check_linear_fp8,
     check_silu_grad, check_attn_bwd_finite_differences, check_attn_bwd_closed_form,
     check_attn_bwd_against_torch_autograd,

@@ -34,7 +34,7 @@ MUTANTS = [
      "if (bkt > num_buckets - 1) bkt = num_buckets - 2;"),
     ("unbiased_variance", "var /= (double)F;", "var /= (double)(F - 1);"),
     ("eps_outside_sqrt", "double rstd = 1.0 / sqrt(var + eps);", "double rstd = 1.0 / (sqrt(var) + eps);"),
-    ("gate_dropped", "* u[m * u_ld + c];", ";"),
+    ("gate_dropped", "*= u[m * u_ld + c];", "*= 1.0;"),
     ("split_q_k_swapped", "uvqk + 2 * F, W, uvqk + 3 * F, W,", "uvqk + 3 * F, W, uvqk + 2 * F, W,"),
     ("split_u_v_swapped", "memcpy(urow + r * F, uvqk + t * W,", "memcpy(urow + r * F, uvqk + t * W + F,"),
     ("residual_dropped", "hstu_oracle_linear(n, (int32_t)F, D, ygate, W2, b2, 0, xrow, out);",
@@ -50,6 +50,10 @@ MUTANTS = [
      "if (bias) acc += bias[n];\n"
      "            if (residual) acc += residual[m * N + n];\n            y[m * N + n] = acc;\n"
      "        }\n    }\n}\n\n/* ------"),
+    ("input_norm_not_applied", "        xin = xn;\n", "        xin = x;\n"),
+    ("input_norm_residual_normalized", "memcpy(xrow + r * D, x + t * D,", "memcpy(xrow + r * D, xin + t * D,"),
+    ("layernorm_no_affine", "yr[c] = (ar[c] - mean) * rstd * (gamma ? gamma[c] : 1.0) + (beta ? beta[c] : 0.0);",
+     "yr[c] = (ar[c] - mean) * rstd;"),
     ("e4m3_ties_away", "return fmod(f, 2.0) == 0.0 ? f : f + 1.0;", "return f + 1.0;"),
     ("e4m3_exponent_bias_8", "else v = ldexp(1.0 + (double)m / 8.0, e - 7);",
      "else v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
