@@ -554,12 +554,15 @@ def oracle_layer_rate(li, budget_s: float, seed: int = 0):
     return rate / 1e12, k, ntok, dt, oracle.num_threads()
 
 
-def bench_layer(args, rank, world, local, peaks, peak_kind, cfg_id=None, cpu_budget_s=None):
+def bench_layer(args, rank, world, local, peaks, peak_kind, cfg_id=None, cpu_budget_s=None,
+                fp8=None, input_norm=None):
     import torch
     import jagged_pointwise_attention_b200 as hstu
     from gen import CONFIGS, make_layer_inputs
 
     cfg_id = args.config if cfg_id is None else cfg_id
+    fp8 = args.fp8 if fp8 is None else fp8
+    input_norm = args.input_norm if input_norm is None else input_norm
     cfg = CONFIGS[cfg_id]
     seed = 1000 + cfg_id + 7919 * rank
     li = make_layer_inputs(cfg_id, seed=seed)
@@ -571,25 +574,35 @@ def bench_layer(args, rank, world, local, peaks, peak_kind, cfg_id=None, cpu_bud
     x, W1, W2 = to(li.x, bf), to(li.W1, bf), to(li.W2, bf)
     off, ts, pos, tb = to(li.seq_offsets), to(li.timestamps), to(li.pos_bias), to(li.time_bias)
     out = torch.empty_like(x)
-    ws = torch.empty(hstu.hstu_layer_workspace_bytes(li.T, li.B, li.H, li.d, li.max_seqlen),
+    ws = torch.empty(hstu.hstu_layer_workspace_bytes(li.T, li.B, li.D, li.H, li.d, li.max_seqlen),
                      dtype=torch.uint8, device=dev)
     lengths = np.diff(li.seq_offsets)
     fl = causal_flops(lengths, li.H, li.d, li.d) + layer_flops(li.T, li.D, li.H, li.d)
 
-    if args.fp8:
+    # the input LayerNorm's affine terms (the model's parameters)
+    rng = np.random.default_rng(seed + 1)
+    in_g = to((1 + 0.1 * rng.standard_normal(li.D)).astype(np.float32)) if input_norm else None
+    in_b = to((0.1 * rng.standard_normal(li.D)).astype(np.float32)) if input_norm else None
+    if fp8:
         W1q, s1 = hstu.hstu_quant_rows_e4m3(W1)
         W2q, s2 = hstu.hstu_quant_rows_e4m3(W2)
         ws = torch.empty(hstu.hstu_layer_fp8_workspace_bytes(li.T, li.B, li.D, li.H, li.d,
                                                               li.max_seqlen),
                          dtype=torch.uint8, device=dev)
 
-    def step():
-        if args.fp8:
-            hstu.hstu_layer_fp8_fwd(x, W1q, s1, W2q, s2, off, ts, pos, tb, li.H, li.d,
-                                    li.max_seqlen, ln_eps=li.ln_eps, out=out, workspace=ws)
+    def layer_call(xx, oo, o, sq, strm=None):   # x, out, seq_offsets, timestamps
+        if fp8:
+            hstu.hstu_layer_fp8_fwd(xx, W1q, s1, W2q, s2, o, sq, pos, tb, li.H, li.d,
+                                    li.max_seqlen, ln_eps=li.ln_eps, out=oo, workspace=ws,
+                                    stream=strm, input_norm=input_norm, in_gamma=in_g,
+                                    in_beta=in_b)
         else:
-            hstu.hstu_layer_fwd(x, W1, W2, off, ts, pos, tb, li.H, li.d, li.max_seqlen,
-                                ln_eps=li.ln_eps, out=out, workspace=ws)
+            hstu.hstu_layer_fwd(xx, W1, W2, o, sq, pos, tb, li.H, li.d, li.max_seqlen,
+                                ln_eps=li.ln_eps, out=oo, workspace=ws, stream=strm,
+                                input_norm=input_norm, in_gamma=in_g, in_beta=in_b)
+
+    def step():
+        layer_call(x, out, off, ts)
 
     for _ in range(args.warmup):
         step()
@@ -616,10 +629,11 @@ def bench_layer(args, rank, world, local, peaks, peak_kind, cfg_id=None, cpu_bud
     roofline = {"bound": "tensor", "achieved": round(step_tf, 2), "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": round(step_tf / peaks["bf16_tflops"], 4),
                 "peak_kind": "burst bf16 dense, %s" % peak_kind, "traffic": None,
-                "kernel": "whole layer step (f1, plan, bias tables, attention, LayerNorm gate, f2)"}
-    e2e = None if args.fp8 else e2e_layer(args, li, dev, stream, fl, world, hstu, ws)
+                "kernel": "whole layer step (%sf1, plan, bias tables, attention, LayerNorm "
+                          "gate, f2)" % ("input LayerNorm, " if input_norm else "")}
+    e2e = e2e_layer(args, li, dev, stream, fl, world, layer_call)
     cpu = None
-    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+    if world == 1 and rank == 0 and not args.no_cpu_baseline and cpu_budget_s != 0:
         v, nseq, ntok, secs, thr = oracle_layer_rate(
             li, args.cpu_budget_s if cpu_budget_s is None else cpu_budget_s)
         cpu = {"value": round(v, 6), "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
@@ -628,23 +642,27 @@ def bench_layer(args, rank, world, local, peaks, peak_kind, cfg_id=None, cpu_bud
     return {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(max_ms / args.steps, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 projections, bf16 attention" if args.fp8 else "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3 projections, bf16 attention" if fp8 else "bf16",
         "data": "synthetic (seeded generator; no dataset)",
         "config": workload_config(cfg_id, li.B, li.T, li.max_seqlen, seed, world,
                                   {"D": li.D, "H": li.H, "d": li.d,
-                                   "projections": "e4m3" if args.fp8 else "bf16",
+                                   "projections": "e4m3" if fp8 else "bf16",
+                                   "input_layernorm": bool(input_norm),
                                    "l2": "layer working set %.0f MB > L2" % (
                                        (ws.numel() + 2 * x.numel() * 2) / 2 ** 20)}),
         "launch": "eager, one call per step",
         "tokens_per_s": round(toks / (max_ms * 1e-3), 1),
         "pct_of_bf16_peak": {"measured_burst": round(100 * value / peaks["bf16_tflops"], 2)},
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": (7 if args.fp8 else 6) * args.steps, "clocks": sampler.summary(),
+        "gpu_launches": (7 if fp8 or input_norm else 6) * args.steps,
+        "clocks": sampler.summary(),
     }
 
 
-def e2e_layer(args, li, dev, stream, flops, world, hstu, ws):
-    """End to end through hstu_layer_fwd: every step copies its activations x,
+def e2e_layer(args, li, dev, stream, flops, world, layer_call):
+    """End to end through the layer entry point that `layer_call` makes
+    (hstu_layer_fwd or hstu_layer_fp8_fwd): every step copies its activations x,
     offsets and timestamps from pinned host memory and the output back; the
     weights and bias tables are the model's parameters and stay on the device.
     Pipelined like the attention's: step i's copies in overlap step i-1's
@@ -656,9 +674,6 @@ def e2e_layer(args, li, dev, stream, flops, world, hstu, ws):
         t = torch.from_numpy(np.ascontiguousarray(a))
         return (t.to(dt) if dt is not None else t).pin_memory()
 
-    to = lambda a, dt=None: (torch.from_numpy(np.ascontiguousarray(a)).to(dt)  # noqa: E731
-                             if dt else torch.from_numpy(np.ascontiguousarray(a))).to(dev)
-    W1, W2, pos, tb = to(li.W1, bf), to(li.W2, bf), to(li.pos_bias), to(li.time_bias)
     host = dict(x=pinned(li.x, bf), off=pinned(li.seq_offsets), ts=pinned(li.timestamps))
     devb = [{k: torch.empty_like(v, device=dev) for k, v in host.items()} for _ in range(2)]
     out_dev = [torch.empty((li.T, li.D), dtype=bf, device=dev) for _ in range(2)]
@@ -682,9 +697,7 @@ def e2e_layer(args, li, dev, stream, flops, world, hstu, ws):
             if used[b]:
                 stream.wait_event(ev["out"][b])
             d = devb[b]
-            hstu.hstu_layer_fwd(d["x"], W1, W2, d["off"], d["ts"], pos, tb, li.H, li.d,
-                                li.max_seqlen, ln_eps=li.ln_eps, out=out_dev[b], workspace=ws,
-                                stream=stream)
+            layer_call(d["x"], out_dev[b], d["off"], d["ts"], stream)
             ev["run"][b].record(stream)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev["run"][b])
@@ -936,6 +949,9 @@ def parse_args(argv=None):
     ap.add_argument("--fp8", action="store_true",
                     help="with --config 5: the layer with both projections in FP8 "
                          "(hstu_layer_fp8_fwd, weights quantized once)")
+    ap.add_argument("--input-norm", action="store_true",
+                    help="with --config 5: LayerNorm on the layer's input before f1 (fused with "
+                         "the E4M3 quantization under --fp8)")
     ap.add_argument("--backward", action="store_true",
                     help="time the fp32 attention backward (hstu_attn_bwd_f32) on the "
                          "--config workload's shapes instead of the forward")
@@ -986,6 +1002,15 @@ def main(argv=None):
             sub = fn(args, rank, world, local, peaks, kind, cfg_id=c,
                      cpu_budget_s=min(args.cpu_budget_s, 8.0))
             subs[sub["config"]["workload"]] = sub
+        # the layer's variants: E4M3 projections, and the input LayerNorm (for
+        # the FP8 layer fused with x's quantization); the oracle's rate is the
+        # bf16 line's
+        for fp8, norm in ((True, False), (False, True), (True, True)):
+            sub = bench_layer(args, rank, world, local, peaks, kind, cfg_id=5, cpu_budget_s=0,
+                              fp8=fp8, input_norm=norm)
+            name = sub["config"]["workload"] + ("_fp8" if fp8 else "") + ("_input_ln" if norm
+                                                                          else "")
+            subs[name] = sub
         line["configs"] = subs
         line["gpu_launches_all_lines"] = line["gpu_launches"] + sum(
             v["gpu_launches"] for v in subs.values())

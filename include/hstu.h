@@ -16,8 +16,9 @@
  *   out[o+i,h,:] = (1/max_seqlen) * sum_{j<=i} silu(s_ij) * v[o+j,h,:]
  *
  * with silu(x) = x * sigmoid(x). No softmax, no 1/sqrt(d) score scale.
- * Besides the bf16 forward path: row-wise E4M3 (FP8) projections and the
- * attention backward (fp32), in their own sections below.
+ * Sections below: the attention; the layer around it (projections, the
+ * input and output LayerNorms, the whole layer); row-wise E4M3 (FP8)
+ * projections; the attention backward (fp32).
  *
  * Conventions for every entry point:
  *  - Pointers marked "device" must be device memory of the current CUDA device
@@ -46,7 +47,7 @@
 extern "C" {
 #endif
 
-#define HSTU_ABI_VERSION 1
+#define HSTU_ABI_VERSION 2
 
 typedef enum hstu_status {
     HSTU_OK = 0,
@@ -206,28 +207,72 @@ hstu_status_t hstu_debug_wait_timeout(int32_t wait_us, void* stream);
 
 /* ---------------------------------------------------------------- layer */
 
-/* ---------------------------------------------------------------- backward */
+/* The HSTU layer around the attention, in the order the generative-
+ * recommenders README gives for HSTU Ultra ("HSTU Ultra attention
+ * benchmark": input normalization, the UVQK projection, attention, output
+ * normalization with gating and the output projection, residual). The pages
+ * name the pieces (hstu_compute_uqvk, hstu_compute_output) but print no
+ * formula; the readings taken are: SiLU on all of U|V|Q|K, LayerNorm over a
+ * token's features with biased variance and eps inside the square root,
+ * gating by U after the output LayerNorm, residual x + Y W2^T. */
 
-/* Gradients of the attention (fp32 path, CUDA cores; the pages' reference
- * implementation has forward and backward attention kernels,
- * generative-recommenders README, "HSTU Ultra attention benchmark") for an
- * upstream gradient dout of hstu_attn_fwd's output. With s_ij = q_i.k_j +
- * pos + time, p_ij = silu(s_ij)/N:
- *   dv_j = sum_{i>=j} p_ij dout_i;  ds_ij = (dout_i.v_j) silu'(s_ij) / N
- *   dq_i = sum_{j<=i} ds_ij k_j;    dk_j = sum_{i>=j} ds_ij q_i
- *   dpos[h][min(i-j, P-1)] and dtime[h][bucket] sum the ds_ij of their pairs.
- * q, k, dq, dk: device fp32 [T, H, d_qk] contiguous; v, dout, dv: [T, H,
- * d_v]; dpos [H, num_pos] required when pos_bias is given, dtime [H,
- * num_time_buckets] when timestamps and time_bias are (both overwritten);
- * d_qk, d_v <= 128; num_pos + num_time_buckets <= 12288. Other arguments as
- * hstu_attn_run. Two kernel launches (a query pass and a key pass) plus the
- * table clears. */
-hstu_status_t hstu_attn_bwd_f32(const float* q, const float* k, const float* v, const float* dout,
-                                const int64_t* seq_offsets, int32_t B, int64_t total_tokens,
-                                int32_t H, int32_t d_qk, int32_t d_v, const int64_t* timestamps,
-                                const float* pos_bias, int32_t num_pos, const float* time_bias,
-                                int32_t num_time_buckets, int32_t max_seqlen, float* dq, float* dk,
-                                float* dv, float* dpos, float* dtime, void* stream);
+/* y[M, N] = epilogue(x[M, K] W[N, K]^T + bias[N]) on tcgen05 tensor cores.
+ * x, W, y, residual: device bf16, row strides ldx, ldw (=K typically), ldy, ldr.
+ * bias: device fp32 [N] or NULL. residual: [M, N] bf16, required for
+ * HSTU_EPI_RESIDUAL, else ignored. K % 64 == 0, N % 128 == 0.
+ * The UVQK projection (f1, SiLU epilogue) and the output projection (f2,
+ * residual epilogue) of the layer (README, "HSTU Ultra attention
+ * benchmark": UVQK and output projection). */
+hstu_status_t hstu_linear_fwd(const void* x, int64_t ldx, int64_t M, int32_t K,
+                              const void* W, int64_t ldw, int32_t N, const float* bias,
+                              hstu_epilogue_t epilogue, const void* residual, int64_t ldr,
+                              void* y, int64_t ldy, void* stream);
+
+/* y[m, :] = LayerNorm(a[m, :]) * u[m, :] over F features (biased variance, eps
+ * inside the square root, then gamma, beta; NULL = 1, 0). a, u, y: device bf16
+ * with row strides lda, ldu, ldy; gamma, beta: device fp32 [F] or NULL.
+ * F % 256 == 0 and F <= 2048. The output normalization and gating step of
+ * the layer (README, "HSTU Ultra attention benchmark": fused output
+ * normalization and gating). */
+hstu_status_t hstu_layernorm_gate_fwd(const void* a, int64_t lda, const void* u, int64_t ldu,
+                                      int64_t M, int32_t F, const float* gamma,
+                                      const float* beta, float eps, void* y, int64_t ldy,
+                                      void* stream);
+
+/* y[m, :] = LayerNorm(a[m, :]) over F features (as hstu_layernorm_gate_fwd
+ * without the gate). The layer's input normalization before the UVQK
+ * projection (README, "HSTU Ultra attention benchmark": input norm). */
+hstu_status_t hstu_layernorm_fwd(const void* a, int64_t lda, int64_t M, int32_t F,
+                                 const float* gamma, const float* beta, float eps, void* y,
+                                 int64_t ldy, void* stream);
+
+/* Workspace bytes of hstu_layer_fwd (D: the model width of x). */
+size_t hstu_layer_workspace_bytes(int64_t total_tokens, int32_t B, int32_t D, int32_t H,
+                                  int32_t d, int32_t max_seqlen);
+
+/* One HSTU layer forward (bf16, fp32 accumulation) on `stream`:
+ *   0. xn = LayerNorm(x)             over the D features, when input_norm != 0
+ *                                    (affine in_gamma, in_beta [D] or NULL;
+ *                                    eps ln_eps); else xn = x
+ *   1. UVQK = silu(xn W1^T + b1)     x [T, D], W1 [4*H*d, D]; columns U|V|Q|K
+ *   2. A = attention(Q, K, V)        as hstu_attn_fwd, d_qk = d_v = d
+ *   3. Y = LayerNorm(A) * U          over the H*d features of each token
+ *   4. out = x + Y W2^T + b2         W2 [D, H*d]; the residual adds x itself
+ * x, W1, W2, out: device bf16 row-major; b1 [4Hd], b2 [D], ln_gamma, ln_beta
+ * [Hd]: device fp32 or NULL. Other arguments as hstu_attn_run. D % 128 == 0
+ * (D % 256 == 0 and D <= 2048 with the input norm), d in {64, 128},
+ * H*d % 256 == 0. README, "HSTU Ultra attention benchmark". */
+hstu_status_t hstu_layer_fwd(const void* x, int64_t total_tokens, int32_t D,
+                             const void* W1, const float* b1,
+                             const void* W2, const float* b2,
+                             const float* ln_gamma, const float* ln_beta, float ln_eps,
+                             int32_t input_norm, const float* in_gamma, const float* in_beta,
+                             const int64_t* seq_offsets, int32_t B, int32_t H, int32_t d,
+                             const int64_t* timestamps,
+                             const float* pos_bias, int32_t num_pos,
+                             const float* time_bias, int32_t num_time_buckets,
+                             int32_t max_seqlen, void* out,
+                             void* workspace, size_t workspace_bytes, void* stream);
 
 /* ---------------------------------------------------------------- FP8 projections */
 
@@ -235,13 +280,14 @@ hstu_status_t hstu_attn_bwd_f32(const float* q, const float* k, const float* v, 
  * reference and benchmark": row-wise E4M3 quantization of the projection
  * operands). For each row r of x (device bf16 [M, K], row stride ldx):
  *   amax = max |x[r, :]|, inv = 448 / amax, scales[r] = amax / 448 (fp32,
- *   rounded to nearest; an all-zero row gets inv = 0, scales[r] = 1),
- *   codes[r, c] = E4M3(fp32(x[r, c] * inv)), rounding to nearest (ties to an
- *   even mantissa) and saturating finite overflow at +-448,
- * so that x[r, c] ~ value(codes[r, c]) * scales[r]. codes: device uint8
- * [M, K], row stride ldq (multiple of 16); scales: device fp32 [M]. K % 16
- * == 0, ldx % 8 == 0, x and codes 16-byte aligned. One launch, one warp per
- * row. */
+ *   rounded to nearest), codes[r, c] = E4M3(fp32(x[r, c] * inv)), rounding
+ *   to nearest (ties to an even mantissa) and saturating finite overflow at
+ *   +-448, so that x[r, c] ~ value(codes[r, c]) * scales[r]. A row whose inv
+ *   is not a finite fp32 number (all zeros, or amax below 448 / FLT_MAX) gets
+ *   inv = 0 and scales[r] = 1: zero codes.
+ * codes: device uint8 [M, K], row stride ldq (multiple of 16); scales: device
+ * fp32 [M]. K % 16 == 0, ldx % 8 == 0, x and codes 16-byte aligned. One
+ * launch, one warp per row. */
 hstu_status_t hstu_quant_rows_e4m3(const void* x, int64_t ldx, int64_t M, int32_t K, void* codes,
                                    int64_t ldq, float* scales, void* stream);
 
@@ -266,71 +312,62 @@ hstu_status_t hstu_layernorm_gate_fp8_fwd(const void* a, int64_t lda, const void
                                           const float* beta, float eps, void* codes,
                                           int64_t ldq, float* scales, void* stream);
 
-/* y[M, N] = epilogue(x[M, K] W[N, K]^T + bias[N]) on tcgen05 tensor cores.
- * x, W, y, residual: device bf16, row strides ldx, ldw (=K typically), ldy, ldr.
- * bias: device fp32 [N] or NULL. residual: [M, N] bf16, required for
- * HSTU_EPI_RESIDUAL, else ignored. K % 64 == 0, N % 128 == 0.
- * This is the UVQK projection (f1, SiLU epilogue) and the output projection
- * (f2, residual epilogue) of the HSTU layer. */
-hstu_status_t hstu_linear_fwd(const void* x, int64_t ldx, int64_t M, int32_t K,
-                              const void* W, int64_t ldw, int32_t N, const float* bias,
-                              hstu_epilogue_t epilogue, const void* residual, int64_t ldr,
-                              void* y, int64_t ldy, void* stream);
-
-/* y[m, :] = LayerNorm(a[m, :]) * u[m, :] over F features (biased variance, eps
- * inside the square root, then gamma, beta; NULL = 1, 0). a, u, y: device bf16
- * with row strides lda, ldu, ldy; gamma, beta: device fp32 [F] or NULL.
- * F % 256 == 0 and F <= 2048. The output normalization and gating step of
- * the HSTU layer. */
-hstu_status_t hstu_layernorm_gate_fwd(const void* a, int64_t lda, const void* u, int64_t ldu,
-                                      int64_t M, int32_t F, const float* gamma,
-                                      const float* beta, float eps, void* y, int64_t ldy,
-                                      void* stream);
-
-/* Workspace bytes of hstu_layer_fwd. */
-size_t hstu_layer_workspace_bytes(int64_t total_tokens, int32_t B, int32_t H, int32_t d,
-                                  int32_t max_seqlen);
-
-/* One HSTU layer forward (bf16, fp32 accumulation), four steps on `stream`:
- *   1. UVQK = silu(x W1^T + b1)     x [T, D], W1 [4*H*d, D]; columns U|V|Q|K
- *   2. A = attention(Q, K, V)        as hstu_attn_fwd, d_qk = d_v = d
- *   3. Y = LayerNorm(A) * U          over the H*d features of each token
- *   4. out = x + Y W2^T + b2         W2 [D, H*d]
- * x, W1, W2, out: device bf16 row-major; b1 [4Hd], b2 [D], ln_gamma, ln_beta
- * [Hd]: device fp32 or NULL. Other arguments as hstu_attn_run. D % 128 == 0,
- * D % 64 == 0, d in {64, 128}, H*d % 256 == 0. */
-hstu_status_t hstu_layer_fwd(const void* x, int64_t total_tokens, int32_t D,
-                             const void* W1, const float* b1,
-                             const void* W2, const float* b2,
-                             const float* ln_gamma, const float* ln_beta, float ln_eps,
-                             const int64_t* seq_offsets, int32_t B, int32_t H, int32_t d,
-                             const int64_t* timestamps,
-                             const float* pos_bias, int32_t num_pos,
-                             const float* time_bias, int32_t num_time_buckets,
-                             int32_t max_seqlen, void* out,
-                             void* workspace, size_t workspace_bytes, void* stream);
+/* hstu_layernorm_fwd with the bf16 result row quantized row-wise to E4M3 in
+ * the same kernel (codes and scales as hstu_layernorm_gate_fp8_fwd): the
+ * fused input-LayerNorm-to-FP8 step before the UVQK projection (README,
+ * "HSTU Ultra attention benchmark": fused LayerNorm-to-FP8 quantization for
+ * the UVQK projection). */
+hstu_status_t hstu_layernorm_fp8_fwd(const void* a, int64_t lda, int64_t M, int32_t F,
+                                     const float* gamma, const float* beta, float eps,
+                                     void* codes, int64_t ldq, float* scales, void* stream);
 
 /* Workspace bytes of hstu_layer_fp8_fwd (D: the model width of x). */
 size_t hstu_layer_fp8_workspace_bytes(int64_t total_tokens, int32_t B, int32_t D, int32_t H,
                                       int32_t d, int32_t max_seqlen);
 
-/* hstu_layer_fwd with both projections in FP8: x is quantized row-wise to
- * E4M3, f1 runs on E4M3 codes (SiLU epilogue), the attention in bf16, the
- * LayerNorm gate writes E4M3 codes of its bf16 result, and f2 runs on E4M3
- * codes with the bf16 residual x. W1q [4*H*d, D] / w1_scales [4*H*d] and W2q
- * [D, H*d] / w2_scales [D] are the weights quantized once by
- * hstu_quant_rows_e4m3 (device uint8 / fp32). D % 128 == 0, H*d % 256 == 0
- * (so both K are multiples of 128), d in {64, 128}; other arguments as
- * hstu_layer_fwd. Seven launches: quantize, f1, plan, bias tables, attention,
- * LayerNorm gate, f2. */
+/* hstu_layer_fwd with both projections in FP8: x (or, with input_norm,
+ * LayerNorm(x) in the same pass) is quantized row-wise to E4M3, f1 runs on
+ * E4M3 codes (SiLU epilogue), the attention in bf16, the LayerNorm gate writes
+ * E4M3 codes of its bf16 result, and f2 runs on E4M3 codes with the bf16
+ * residual x. W1q [4*H*d, D] / w1_scales [4*H*d] and W2q [D, H*d] / w2_scales
+ * [D] are the weights quantized once by hstu_quant_rows_e4m3 (device uint8 /
+ * fp32). D % 128 == 0 (D % 256 == 0 and D <= 2048 with the input norm),
+ * H*d % 256 == 0 (so both K are multiples of 128), d in {64, 128}; other
+ * arguments as hstu_layer_fwd. Seven launches: quantize (or LayerNorm and
+ * quantize), f1, plan, bias tables, attention, LayerNorm gate, f2. */
 hstu_status_t hstu_layer_fp8_fwd(const void* x, int64_t total_tokens, int32_t D, const void* W1q,
                                  const float* w1_scales, const float* b1, const void* W2q,
                                  const float* w2_scales, const float* b2, const float* ln_gamma,
-                                 const float* ln_beta, float ln_eps, const int64_t* seq_offsets,
+                                 const float* ln_beta, float ln_eps, int32_t input_norm,
+                                 const float* in_gamma, const float* in_beta,
+                                 const int64_t* seq_offsets,
                                  int32_t B, int32_t H, int32_t d, const int64_t* timestamps,
                                  const float* pos_bias, int32_t num_pos, const float* time_bias,
                                  int32_t num_time_buckets, int32_t max_seqlen, void* out,
                                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------- backward */
+
+/* Gradients of the attention (fp32 path, CUDA cores; the pages' reference
+ * implementation has forward and backward attention kernels,
+ * generative-recommenders README, "HSTU Ultra attention benchmark") for an
+ * upstream gradient dout of hstu_attn_fwd's output. With s_ij = q_i.k_j +
+ * pos + time, p_ij = silu(s_ij)/N:
+ *   dv_j = sum_{i>=j} p_ij dout_i;  ds_ij = (dout_i.v_j) silu'(s_ij) / N
+ *   dq_i = sum_{j<=i} ds_ij k_j;    dk_j = sum_{i>=j} ds_ij q_i
+ *   dpos[h][min(i-j, P-1)] and dtime[h][bucket] sum the ds_ij of their pairs.
+ * q, k, dq, dk: device fp32 [T, H, d_qk] contiguous; v, dout, dv: [T, H,
+ * d_v]; dpos [H, num_pos] required when pos_bias is given, dtime [H,
+ * num_time_buckets] when timestamps and time_bias are (both overwritten);
+ * d_qk, d_v <= 128; num_pos + num_time_buckets <= 12288. Other arguments as
+ * hstu_attn_run. Two kernel launches (a query pass and a key pass) plus the
+ * table clears. */
+hstu_status_t hstu_attn_bwd_f32(const float* q, const float* k, const float* v, const float* dout,
+                                const int64_t* seq_offsets, int32_t B, int64_t total_tokens,
+                                int32_t H, int32_t d_qk, int32_t d_v, const int64_t* timestamps,
+                                const float* pos_bias, int32_t num_pos, const float* time_bias,
+                                int32_t num_time_buckets, int32_t max_seqlen, float* dq, float* dk,
+                                float* dv, float* dpos, float* dtime, void* stream);
 
 #ifdef __cplusplus
 }

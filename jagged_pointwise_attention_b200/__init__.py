@@ -26,7 +26,7 @@ __all__ = [
     "hstu_layer_fwd", "hstu_layer_workspace_bytes", "hstu_linear_fwd",
     "hstu_layernorm_gate_fwd", "hstu_debug_bias_indices", "hstu_debug_wait_timeout",
     "hstu_attn_bwd_f32", "hstu_quant_rows_e4m3", "hstu_linear_fp8_fwd",
-    "hstu_layernorm_gate_fp8_fwd",
+    "hstu_layernorm_gate_fp8_fwd", "hstu_layernorm_fwd", "hstu_layernorm_fp8_fwd",
     "hstu_layer_fp8_workspace_bytes", "hstu_layer_fp8_fwd",
     "hstu_device_status", "HstuError", "library_path",
 ]
@@ -252,8 +252,37 @@ def hstu_layernorm_gate_fwd(a: torch.Tensor, u: torch.Tensor, gamma=None, beta=N
     return out
 
 
-def hstu_layer_workspace_bytes(total_tokens: int, B: int, H: int, d: int, max_seqlen: int) -> int:
-    return int(_lib().hstu_layer_workspace_bytes(total_tokens, B, H, d, max_seqlen))
+def hstu_layernorm_fwd(a: torch.Tensor, gamma=None, beta=None, eps: float = 1e-5,
+                       out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """LayerNorm(a) over the last axis (bf16 rows, any row stride): the layer's
+    input normalization."""
+    _on_cuda(a, gamma, beta, out)
+    M, F = a.shape
+    if out is None:
+        out = torch.empty((M, F), dtype=torch.bfloat16, device=a.device)
+    _native.check("hstu_layernorm_fwd", _lib().hstu_layernorm_fwd(
+        _ptr(a), a.stride(0), M, F, _ptr(gamma), _ptr(beta), float(eps), _ptr(out),
+        out.stride(0), _stream(stream)))
+    return out
+
+
+def hstu_layernorm_fp8_fwd(a: torch.Tensor, gamma=None, beta=None, eps: float = 1e-5,
+                           stream=None):
+    """LayerNorm(a) with the bf16 result rows quantized to E4M3 in the same
+    kernel: (codes uint8 [M, F], scales fp32 [M])."""
+    _on_cuda(a, gamma, beta)
+    M, F = a.shape
+    codes = torch.empty((M, F), dtype=torch.uint8, device=a.device)
+    scales = torch.empty(M, dtype=torch.float32, device=a.device)
+    _native.check("hstu_layernorm_fp8_fwd", _lib().hstu_layernorm_fp8_fwd(
+        _ptr(a), a.stride(0), M, F, _ptr(gamma), _ptr(beta), float(eps), _ptr(codes),
+        codes.stride(0), _ptr(scales), _stream(stream)))
+    return codes, scales
+
+
+def hstu_layer_workspace_bytes(total_tokens: int, B: int, D: int, H: int, d: int,
+                               max_seqlen: int) -> int:
+    return int(_lib().hstu_layer_workspace_bytes(total_tokens, B, D, H, d, max_seqlen))
 
 
 def hstu_layer_fwd(x: torch.Tensor, W1: torch.Tensor, W2: torch.Tensor, seq_offsets: torch.Tensor,
@@ -261,10 +290,13 @@ def hstu_layer_fwd(x: torch.Tensor, W1: torch.Tensor, W2: torch.Tensor, seq_offs
                    time_bias: Optional[torch.Tensor], H: int, d: int, max_seqlen: int,
                    b1=None, b2=None, ln_gamma=None, ln_beta=None, ln_eps: float = 1e-5,
                    out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-                   stream=None) -> torch.Tensor:
+                   stream=None, input_norm: bool = False, in_gamma=None,
+                   in_beta=None) -> torch.Tensor:
     """One HSTU layer forward: x + (LayerNorm(attn(Q, K, V)) * U) W2^T + b2 with
-    U|V|Q|K = silu(x W1^T + b1). x [T, D] bf16, W1 [4Hd, D], W2 [D, Hd]."""
-    _on_cuda(x, W1, W2, seq_offsets, timestamps, pos_bias, time_bias, b1, b2, ln_gamma, ln_beta)
+    U|V|Q|K = silu(x' W1^T + b1), x' = x or, with input_norm, LayerNorm(x)
+    (affine in_gamma, in_beta). x [T, D] bf16, W1 [4Hd, D], W2 [D, Hd]."""
+    _on_cuda(x, W1, W2, seq_offsets, timestamps, pos_bias, time_bias, b1, b2, ln_gamma, ln_beta,
+             in_gamma, in_beta)
     T, D = x.shape
     B = seq_offsets.numel() - 1
     for t in (x, W1, W2):
@@ -273,10 +305,11 @@ def hstu_layer_fwd(x: torch.Tensor, W1: torch.Tensor, W2: torch.Tensor, seq_offs
     if out is None:
         out = torch.empty_like(x)
     if workspace is None:
-        workspace = _workspace(hstu_layer_workspace_bytes(T, B, H, d, max_seqlen), x.device)
+        workspace = _workspace(hstu_layer_workspace_bytes(T, B, D, H, d, max_seqlen), x.device)
     _native.check("hstu_layer_fwd", _lib().hstu_layer_fwd(
         _ptr(x), T, D, _ptr(W1), _ptr(b1), _ptr(W2), _ptr(b2), _ptr(ln_gamma), _ptr(ln_beta),
-        float(ln_eps), _ptr(seq_offsets), B, H, d, _ptr(timestamps), _ptr(pos_bias),
+        float(ln_eps), 1 if input_norm else 0, _ptr(in_gamma), _ptr(in_beta),
+        _ptr(seq_offsets), B, H, d, _ptr(timestamps), _ptr(pos_bias),
         0 if pos_bias is None else pos_bias.shape[1], _ptr(time_bias),
         0 if time_bias is None else time_bias.shape[1], int(max_seqlen), _ptr(out),
         _ptr(workspace), workspace.numel(), _stream(stream)))
@@ -308,11 +341,13 @@ def hstu_layer_fp8_fwd(x: torch.Tensor, W1q: torch.Tensor, w1_scales: torch.Tens
                        time_bias: Optional[torch.Tensor], H: int, d: int, max_seqlen: int,
                        b1=None, b2=None, ln_gamma=None, ln_beta=None, ln_eps: float = 1e-5,
                        out: Optional[torch.Tensor] = None,
-                       workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+                       workspace: Optional[torch.Tensor] = None, stream=None,
+                       input_norm: bool = False, in_gamma=None, in_beta=None) -> torch.Tensor:
     """hstu_layer_fwd with both projections in FP8 (E4M3 weights from
-    hstu_quant_rows_e4m3, quantized once; activations quantized in the call)."""
+    hstu_quant_rows_e4m3, quantized once; activations quantized in the call,
+    with input_norm the input LayerNorm in the same pass)."""
     _on_cuda(x, W1q, w1_scales, W2q, w2_scales, seq_offsets, timestamps, pos_bias, time_bias, b1,
-             b2, ln_gamma, ln_beta)
+             b2, ln_gamma, ln_beta, in_gamma, in_beta)
     T, D = x.shape
     B = seq_offsets.numel() - 1
     if x.dtype != torch.bfloat16 or not x.is_contiguous():
@@ -326,7 +361,8 @@ def hstu_layer_fp8_fwd(x: torch.Tensor, W1q: torch.Tensor, w1_scales: torch.Tens
         workspace = _workspace(hstu_layer_fp8_workspace_bytes(T, B, D, H, d, max_seqlen), x.device)
     _native.check("hstu_layer_fp8_fwd", _lib().hstu_layer_fp8_fwd(
         _ptr(x), T, D, _ptr(W1q), _ptr(w1_scales), _ptr(b1), _ptr(W2q), _ptr(w2_scales), _ptr(b2),
-        _ptr(ln_gamma), _ptr(ln_beta), float(ln_eps), _ptr(seq_offsets), B, H, d,
+        _ptr(ln_gamma), _ptr(ln_beta), float(ln_eps), 1 if input_norm else 0, _ptr(in_gamma),
+        _ptr(in_beta), _ptr(seq_offsets), B, H, d,
         _ptr(timestamps), _ptr(pos_bias), 0 if pos_bias is None else pos_bias.shape[1],
         _ptr(time_bias), 0 if time_bias is None else time_bias.shape[1], int(max_seqlen),
         _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream)))

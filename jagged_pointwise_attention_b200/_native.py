@@ -41,16 +41,20 @@ SIGNATURES = {
                                            c_p, ctypes.c_int, c_p, c_i64, c_p, c_i64, c_p]),
     "hstu_layernorm_gate_fwd": (ctypes.c_int, [c_p, c_i64, c_p, c_i64, c_i64, c_i32, c_p, c_p,
                                                c_f32, c_p, c_i64, c_p]),
-    "hstu_layer_workspace_bytes": (c_sz, [c_i64, c_i32, c_i32, c_i32, c_i32]),
+    "hstu_layernorm_fwd": (ctypes.c_int, [c_p, c_i64, c_i64, c_i32, c_p, c_p, c_f32, c_p, c_i64,
+                                          c_p]),
+    "hstu_layernorm_fp8_fwd": (ctypes.c_int, [c_p, c_i64, c_i64, c_i32, c_p, c_p, c_f32, c_p,
+                                              c_i64, c_p, c_p]),
+    "hstu_layer_workspace_bytes": (c_sz, [c_i64, c_i32, c_i32, c_i32, c_i32, c_i32]),
     "hstu_layer_fwd": (ctypes.c_int, [c_p, c_i64, c_i32, c_p, c_p, c_p, c_p, c_p, c_p, c_f32,
-                                      c_p, c_i32, c_i32, c_i32, c_p, c_p, c_i32, c_p, c_i32,
-                                      c_i32, c_p, c_p, c_sz, c_p]),
+                                      c_i32, c_p, c_p, c_p, c_i32, c_i32, c_i32, c_p, c_p, c_i32,
+                                      c_p, c_i32, c_i32, c_p, c_p, c_sz, c_p]),
     "hstu_layernorm_gate_fp8_fwd": (ctypes.c_int, [c_p, c_i64, c_p, c_i64, c_i64, c_i32, c_p, c_p,
                                                    c_f32, c_p, c_i64, c_p, c_p]),
     "hstu_layer_fp8_workspace_bytes": (c_sz, [c_i64, c_i32, c_i32, c_i32, c_i32, c_i32]),
     "hstu_layer_fp8_fwd": (ctypes.c_int, [c_p, c_i64, c_i32, c_p, c_p, c_p, c_p, c_p, c_p, c_p,
-                                          c_p, c_f32, c_p, c_i32, c_i32, c_i32, c_p, c_p, c_i32,
-                                          c_p, c_i32, c_i32, c_p, c_p, c_sz, c_p]),
+                                          c_p, c_f32, c_i32, c_p, c_p, c_p, c_i32, c_i32, c_i32,
+                                          c_p, c_p, c_i32, c_p, c_i32, c_i32, c_p, c_p, c_sz, c_p]),
 }
 
 HSTU_OK, HSTU_ERR_INVALID_ARG, HSTU_ERR_UNSUPPORTED, HSTU_ERR_CUDA, HSTU_ERR_TIMEOUT, \

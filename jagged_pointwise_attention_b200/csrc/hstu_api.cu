@@ -439,39 +439,47 @@ hstu_status_t run_linear(const void* x, int64_t ldx, int64_t M, int32_t K, const
                           ldr, y, ldy, stream);
 }
 
-// Y = LayerNorm(A) * U as bf16 (quant == false) or as row-wise E4M3 codes of
-// that bf16 result with row scales (quant == true)
-hstu_status_t run_ln_gate_any(bool quant, const void* a, int64_t lda, const void* u, int64_t ldu,
-                              int64_t M, int32_t F, const float* gamma, const float* beta,
-                              float eps, void* y, int64_t ldy, void* yq, int64_t ldyq, float* ys,
-                              cudaStream_t stream) {
+// Y = LayerNorm(A) * U (u given) or Y = LayerNorm(A) (u null, gate == false),
+// as bf16 (quant == false) or as row-wise E4M3 codes of that bf16 result with
+// row scales (quant == true)
+hstu_status_t run_ln_gate_any(bool quant, bool gate, const void* a, int64_t lda, const void* u,
+                              int64_t ldu, int64_t M, int32_t F, const float* gamma,
+                              const float* beta, float eps, void* y, int64_t ldy, void* yq,
+                              int64_t ldyq, float* ys, cudaStream_t stream) {
     if (M < 0 || F < 1 || !(eps >= 0.0f)) return HSTU_ERR_INVALID_ARG;
     if (F % 256 || F > 2048) return HSTU_ERR_UNSUPPORTED;
     if (M == 0) return HSTU_OK;
-    if (!a || !u || lda < F || ldu < F || lda % 8 || ldu % 8 || !aligned16(a) || !aligned16(u))
-        return HSTU_ERR_INVALID_ARG;
+    if (!a || lda < F || lda % 8 || !aligned16(a)) return HSTU_ERR_INVALID_ARG;
+    if (gate && (!u || ldu < F || ldu % 8 || !aligned16(u))) return HSTU_ERR_INVALID_ARG;
     if (quant ? (!yq || !ys || ldyq < F || ldyq % 16 || !aligned16(yq))
               : (!y || ldy < F || ldy % 8 || !aligned16(y)))
         return HSTU_ERR_INVALID_ARG;
     LnGateArgs args{static_cast<const __nv_bfloat16*>(a), lda, static_cast<const __nv_bfloat16*>(u),
                     ldu, M, gamma, beta, eps, static_cast<__nv_bfloat16*>(y), ldy,
                     static_cast<uint8_t*>(yq), ldyq, ys};
-    const unsigned grid = static_cast<unsigned>((M + 7) / 8);
-#define HSTU_LN_CASES(Q)                                                       \
-    switch (F / 256) {                                                         \
-        case 1: ln_gate_kernel<1, Q><<<grid, 256, 0, stream>>>(args); break;   \
-        case 2: ln_gate_kernel<2, Q><<<grid, 256, 0, stream>>>(args); break;   \
-        case 3: ln_gate_kernel<3, Q><<<grid, 256, 0, stream>>>(args); break;   \
-        case 4: ln_gate_kernel<4, Q><<<grid, 256, 0, stream>>>(args); break;   \
-        case 5: ln_gate_kernel<5, Q><<<grid, 256, 0, stream>>>(args); break;   \
-        case 6: ln_gate_kernel<6, Q><<<grid, 256, 0, stream>>>(args); break;   \
-        case 7: ln_gate_kernel<7, Q><<<grid, 256, 0, stream>>>(args); break;   \
-        default: ln_gate_kernel<8, Q><<<grid, 256, 0, stream>>>(args); break;  \
+    // eight rows per block and pass; up to eight blocks per SM, each striding
+    // over the rows
+    const int64_t blocks = (M + 7) / 8, cap = static_cast<int64_t>(num_sms()) * 8;
+    const unsigned grid = static_cast<unsigned>(blocks < cap ? blocks : cap);
+#define HSTU_LN_CASES(Q, GT)                                                        \
+    switch (F / 256) {                                                              \
+        case 1: ln_gate_kernel<1, Q, GT><<<grid, 256, 0, stream>>>(args); break;    \
+        case 2: ln_gate_kernel<2, Q, GT><<<grid, 256, 0, stream>>>(args); break;    \
+        case 3: ln_gate_kernel<3, Q, GT><<<grid, 256, 0, stream>>>(args); break;    \
+        case 4: ln_gate_kernel<4, Q, GT><<<grid, 256, 0, stream>>>(args); break;    \
+        case 5: ln_gate_kernel<5, Q, GT><<<grid, 256, 0, stream>>>(args); break;    \
+        case 6: ln_gate_kernel<6, Q, GT><<<grid, 256, 0, stream>>>(args); break;    \
+        case 7: ln_gate_kernel<7, Q, GT><<<grid, 256, 0, stream>>>(args); break;    \
+        default: ln_gate_kernel<8, Q, GT><<<grid, 256, 0, stream>>>(args); break;   \
     }
-    if (quant) {
-        HSTU_LN_CASES(true)
+    if (quant && gate) {
+        HSTU_LN_CASES(true, true)
+    } else if (quant) {
+        HSTU_LN_CASES(true, false)
+    } else if (gate) {
+        HSTU_LN_CASES(false, true)
     } else {
-        HSTU_LN_CASES(false)
+        HSTU_LN_CASES(false, false)
     }
 #undef HSTU_LN_CASES
     return launch_status();
@@ -480,21 +488,23 @@ hstu_status_t run_ln_gate_any(bool quant, const void* a, int64_t lda, const void
 hstu_status_t run_ln_gate(const void* a, int64_t lda, const void* u, int64_t ldu, int64_t M,
                           int32_t F, const float* gamma, const float* beta, float eps, void* y,
                           int64_t ldy, cudaStream_t stream) {
-    return run_ln_gate_any(false, a, lda, u, ldu, M, F, gamma, beta, eps, y, ldy, nullptr, 0,
-                           nullptr, stream);
+    return run_ln_gate_any(false, true, a, lda, u, ldu, M, F, gamma, beta, eps, y, ldy, nullptr,
+                           0, nullptr, stream);
 }
 
+// bf16 layer workspace: [UVQK bf16][A bf16][Y bf16][LayerNorm(x) bf16][attention workspace]
 struct LayerWs {
-    size_t uvqk, attn, y, plan, total;
+    size_t uvqk, attn, y, xn, plan, total;
 };
 
-LayerWs layer_ws(int64_t T, int32_t B, int32_t H, int32_t d, int32_t max_seqlen) {
+LayerWs layer_ws(int64_t T, int32_t B, int32_t D, int32_t H, int32_t d, int32_t max_seqlen) {
     LayerWs w{};
     const size_t F = static_cast<size_t>(H) * d;
     w.uvqk = 0;
     w.attn = round_up(w.uvqk + static_cast<size_t>(T) * 4 * F * 2, 256);
     w.y = round_up(w.attn + static_cast<size_t>(T) * F * 2, 256);
-    w.plan = round_up(w.y + static_cast<size_t>(T) * F * 2, 256);
+    w.xn = round_up(w.y + static_cast<size_t>(T) * F * 2, 256);
+    w.plan = round_up(w.xn + static_cast<size_t>(T) * D * 2, 256);
     // window tables for any num_pos: at most one per 128-token diagonal offset
     w.total = w.plan + hstu_attn_workspace_bytes(B, T, max_seqlen, H, 128 * max_tiles_of(max_seqlen));
     return w;
@@ -711,15 +721,31 @@ hstu_status_t hstu_layernorm_gate_fwd(const void* a, int64_t lda, const void* u,
     return run_ln_gate(a, lda, u, ldu, M, F, gamma, beta, eps, y, ldy, as_stream(stream));
 }
 
-size_t hstu_layer_workspace_bytes(int64_t total_tokens, int32_t B, int32_t H, int32_t d,
+hstu_status_t hstu_layernorm_fwd(const void* a, int64_t lda, int64_t M, int32_t F,
+                                 const float* gamma, const float* beta, float eps, void* y,
+                                 int64_t ldy, void* stream) {
+    return run_ln_gate_any(false, false, a, lda, nullptr, 0, M, F, gamma, beta, eps, y, ldy,
+                           nullptr, 0, nullptr, as_stream(stream));
+}
+
+hstu_status_t hstu_layernorm_fp8_fwd(const void* a, int64_t lda, int64_t M, int32_t F,
+                                     const float* gamma, const float* beta, float eps,
+                                     void* codes, int64_t ldq, float* scales, void* stream) {
+    return run_ln_gate_any(true, false, a, lda, nullptr, 0, M, F, gamma, beta, eps, nullptr, 0,
+                           codes, ldq, scales, as_stream(stream));
+}
+
+size_t hstu_layer_workspace_bytes(int64_t total_tokens, int32_t B, int32_t D, int32_t H, int32_t d,
                                   int32_t max_seqlen) {
-    if (total_tokens < 0 || H < 1 || d < 1 || !plan_sizes_ok(B, total_tokens, max_seqlen)) return 0;
-    return layer_ws(total_tokens, B, H, d, max_seqlen).total;
+    if (total_tokens < 0 || D < 1 || H < 1 || d < 1 || !plan_sizes_ok(B, total_tokens, max_seqlen))
+        return 0;
+    return layer_ws(total_tokens, B, D, H, d, max_seqlen).total;
 }
 
 hstu_status_t hstu_layer_fwd(const void* x, int64_t total_tokens, int32_t D, const void* W1,
                              const float* b1, const void* W2, const float* b2,
                              const float* ln_gamma, const float* ln_beta, float ln_eps,
+                             int32_t input_norm, const float* in_gamma, const float* in_beta,
                              const int64_t* seq_offsets, int32_t B, int32_t H, int32_t d,
                              const int64_t* timestamps, const float* pos_bias, int32_t num_pos,
                              const float* time_bias, int32_t num_time_buckets,
@@ -731,9 +757,10 @@ hstu_status_t hstu_layer_fwd(const void* x, int64_t total_tokens, int32_t D, con
     const int32_t F = H * d;
     if (D % 128 || (d != 64 && d != 128) || F % 256 || F > 2048 || (4 * F) % 128)
         return HSTU_ERR_UNSUPPORTED;
+    if (input_norm && (D % 256 || D > 2048)) return HSTU_ERR_UNSUPPORTED;
     if (T == 0 || B == 0) return HSTU_OK;
     if (!x || !W1 || !W2 || !out || !seq_offsets || !workspace) return HSTU_ERR_INVALID_ARG;
-    const LayerWs w = layer_ws(T, B, H, d, max_seqlen);
+    const LayerWs w = layer_ws(T, B, D, H, d, max_seqlen);
     if (workspace_bytes < w.total || !aligned16(workspace)) return HSTU_ERR_INVALID_ARG;
     cudaStream_t s = as_stream(stream);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -742,8 +769,17 @@ hstu_status_t hstu_layer_fwd(const void* x, int64_t total_tokens, int32_t D, con
     __nv_bfloat16* ygate = reinterpret_cast<__nv_bfloat16*>(ws + w.y);
     void* plan_ws = ws + w.plan;
     const size_t plan_bytes = workspace_bytes - w.plan;
-    hstu_status_t st = run_linear(x, D, T, D, W1, D, 4 * F, b1, HSTU_EPI_SILU, nullptr, 0, uvqk,
-                                  4 * F, s);
+    // 1. [LayerNorm(x) ->] f1 with the SiLU epilogue
+    const void* xin = x;
+    hstu_status_t st = HSTU_OK;
+    if (input_norm) {
+        __nv_bfloat16* xn = reinterpret_cast<__nv_bfloat16*>(ws + w.xn);
+        st = run_ln_gate_any(false, false, x, D, nullptr, 0, T, D, in_gamma, in_beta, ln_eps, xn,
+                             D, nullptr, 0, nullptr, s);
+        if (st != HSTU_OK) return st;
+        xin = xn;
+    }
+    st = run_linear(xin, D, T, D, W1, D, 4 * F, b1, HSTU_EPI_SILU, nullptr, 0, uvqk, 4 * F, s);
     if (st != HSTU_OK) return st;
     st = plan_attn(seq_offsets, B, T, max_seqlen, plan_ws, plan_bytes, s);
     if (st != HSTU_OK) return st;
@@ -761,8 +797,8 @@ hstu_status_t hstu_layernorm_gate_fp8_fwd(const void* a, int64_t lda, const void
                                           int64_t M, int32_t F, const float* gamma,
                                           const float* beta, float eps, void* codes,
                                           int64_t ldq, float* scales, void* stream) {
-    return run_ln_gate_any(true, a, lda, u, ldu, M, F, gamma, beta, eps, nullptr, 0, codes, ldq,
-                           scales, as_stream(stream));
+    return run_ln_gate_any(true, true, a, lda, u, ldu, M, F, gamma, beta, eps, nullptr, 0, codes,
+                           ldq, scales, as_stream(stream));
 }
 
 size_t hstu_layer_fp8_workspace_bytes(int64_t total_tokens, int32_t B, int32_t D, int32_t H,
@@ -775,7 +811,9 @@ size_t hstu_layer_fp8_workspace_bytes(int64_t total_tokens, int32_t B, int32_t D
 hstu_status_t hstu_layer_fp8_fwd(const void* x, int64_t total_tokens, int32_t D, const void* W1q,
                                  const float* w1_scales, const float* b1, const void* W2q,
                                  const float* w2_scales, const float* b2, const float* ln_gamma,
-                                 const float* ln_beta, float ln_eps, const int64_t* seq_offsets,
+                                 const float* ln_beta, float ln_eps, int32_t input_norm,
+                                 const float* in_gamma, const float* in_beta,
+                                 const int64_t* seq_offsets,
                                  int32_t B, int32_t H, int32_t d, const int64_t* timestamps,
                                  const float* pos_bias, int32_t num_pos, const float* time_bias,
                                  int32_t num_time_buckets, int32_t max_seqlen, void* out,
@@ -785,6 +823,7 @@ hstu_status_t hstu_layer_fp8_fwd(const void* x, int64_t total_tokens, int32_t D,
         return HSTU_ERR_INVALID_ARG;
     const int32_t F = H * d;
     if (D % 128 || (d != 64 && d != 128) || F % 256 || F > 2048) return HSTU_ERR_UNSUPPORTED;
+    if (input_norm && (D % 256 || D > 2048)) return HSTU_ERR_UNSUPPORTED;
     if (T == 0 || B == 0) return HSTU_OK;
     if (!x || !W1q || !w1_scales || !W2q || !w2_scales || !out || !seq_offsets || !workspace)
         return HSTU_ERR_INVALID_ARG;
@@ -800,8 +839,11 @@ hstu_status_t hstu_layer_fp8_fwd(const void* x, int64_t total_tokens, int32_t D,
     float* sy = reinterpret_cast<float*>(ws + w.sy);
     void* plan_ws = ws + w.plan;
     const size_t plan_bytes = workspace_bytes - w.plan;
-    // 1. x -> E4M3 rows, f1 in FP8 with the SiLU epilogue
-    hstu_status_t st = hstu_quant_rows_e4m3(x, D, T, D, xq, D, sx, stream);
+    // 1. x, or LayerNorm(x) in the same pass, -> E4M3 rows; f1 in FP8 with the
+    // SiLU epilogue
+    hstu_status_t st = input_norm ? run_ln_gate_any(true, false, x, D, nullptr, 0, T, D, in_gamma,
+                                                    in_beta, ln_eps, nullptr, 0, xq, D, sx, s)
+                                  : hstu_quant_rows_e4m3(x, D, T, D, xq, D, sx, stream);
     if (st != HSTU_OK) return st;
     st = run_linear_any(true, xq, D, sx, T, D, W1q, D, w1_scales, 4 * F, b1, HSTU_EPI_SILU,
                         nullptr, 0, uvqk, 4 * F, s);
@@ -815,8 +857,8 @@ hstu_status_t hstu_layer_fp8_fwd(const void* x, int64_t total_tokens, int32_t D,
     st = run_attn(c);
     if (st != HSTU_OK) return st;
     // 3. LayerNorm gate quantized to E4M3 rows in the same kernel
-    st = run_ln_gate_any(true, attn, F, uvqk, 4 * F, T, F, ln_gamma, ln_beta, ln_eps, nullptr, 0,
-                         yq, F, sy, s);
+    st = run_ln_gate_any(true, true, attn, F, uvqk, 4 * F, T, F, ln_gamma, ln_beta, ln_eps,
+                         nullptr, 0, yq, F, sy, s);
     if (st != HSTU_OK) return st;
     // 4. f2 in FP8 with the residual
     return run_linear_any(true, yq, F, sy, T, F, W2q, F, w2_scales, D, b2, HSTU_EPI_RESIDUAL, x,

@@ -45,7 +45,7 @@ def test_every_header_symbol_is_exported(lib):
 
 
 def test_library_loads_without_gpu(lib):
-    assert lib.hstu_abi_version() == 1
+    assert lib.hstu_abi_version() == 2
     assert lib.hstu_status_string(0) == b"ok"
     assert lib.hstu_status_string(4).startswith(b"device pipeline wait")
 
@@ -68,8 +68,8 @@ def test_workspace_queries(lib):
     assert lib.hstu_attn_workspace_bytes(1, 10, 0, 1, 1) == 0
     assert lib.hstu_attn_workspace_bytes(1, 10, 131073, 1, 1) == 0
     assert lib.hstu_attn_workspace_bytes(1, 10, 10, 0, 1) == 0
-    lw = lib.hstu_layer_workspace_bytes(1000, 4, 4, 128, 512)
-    assert lw >= 1000 * 512 * 2 * 6
+    lw = lib.hstu_layer_workspace_bytes(1000, 4, 512, 4, 128, 512)
+    assert lw >= 1000 * 512 * 2 * 7          # U|V|Q|K, A, Y, LayerNorm(x)
 
 
 def _attn(lib, **kw):
@@ -144,8 +144,16 @@ def test_fp8_validation(lib):
     # fused LayerNorm gate quantization: code stride % 16
     assert lib.hstu_layernorm_gate_fp8_fwd(16, 512, 16, 512, 4, 512, None, None,
                                            ctypes.c_float(1e-5), 16, 520, 16, None) == INV
-    assert lib.hstu_layer_fp8_workspace_bytes(1000, 4, 512, 4, 128, 512) > \
-        lib.hstu_layer_workspace_bytes(1000, 4, 4, 128, 512) - 1
+    assert lib.hstu_layer_fp8_workspace_bytes(1000, 4, 512, 4, 128, 512) > 1000 * 512 * 2 * 5
+    # LayerNorm (input norm) and its fused quantization: F % 256, strides
+    assert lib.hstu_layernorm_fwd(16, 512, 4, 384, None, None, ctypes.c_float(1e-5), 16, 512,
+                                  None) == UNS
+    assert lib.hstu_layernorm_fwd(16, 500, 4, 512, None, None, ctypes.c_float(1e-5), 16, 512,
+                                  None) == INV
+    assert lib.hstu_layernorm_fp8_fwd(16, 512, 4, 512, None, None, ctypes.c_float(1e-5), 16, 520,
+                                      16, None) == INV
+    assert lib.hstu_layernorm_fwd(16, 512, 0, 512, None, None, ctypes.c_float(1e-5), 16, 512,
+                                  None) == 0
 
 
 def test_backward_validation(lib):

@@ -8,7 +8,7 @@ import torch
 import jagged_pointwise_attention_b200 as hstu
 import oracle
 from gen import make_layer_inputs, round_to_bf16
-from gpu_util import assert_bf16_close, dev
+from gpu_util import assert_bf16_close, dev, errors
 
 pytestmark = pytest.mark.gpu
 
@@ -114,3 +114,80 @@ def test_layer_workload_sampled_rows():
         rows += [o, o + 1, o + 127, o + 128, o + n // 2, o + n - 1]
     rows = np.array(sorted(set(r for r in rows if r < li.T)), dtype=np.int64)
     assert_bf16_close(got[rows], _layer_oracle(li, rows), "layer workload", strict_abs=True)
+
+
+# --------------------------------------------------------------------------- input LayerNorm
+
+import dataclasses  # noqa: E402
+
+
+def test_layernorm():
+    """The layer's input normalization, affine and identity, on rows where
+    eps dominates the variance, on a row-strided view, and M = 0."""
+    rng = np.random.default_rng(3)
+    M, F = 333, 768
+    a = round_to_bf16((rng.standard_normal((M, F)) * 2.0 + 0.5).astype(np.float32))
+    a[:4] *= 1e-4
+    g = (1 + 0.1 * rng.standard_normal(F)).astype(np.float32)
+    bt = (0.1 * rng.standard_normal(F)).astype(np.float32)
+    got = hstu.hstu_layernorm_fwd(bf(a), dev(g), dev(bt), 1e-5)
+    assert hstu.hstu_device_status() == 0
+    assert_bf16_close(got.float().cpu().numpy(), oracle.layernorm(a, g, bt, 1e-5), "layernorm")
+    got = hstu.hstu_layernorm_fwd(bf(a))
+    assert_bf16_close(got.float().cpu().numpy(), oracle.layernorm(a), "layernorm identity")
+    wide = torch.zeros((M, F + 256), dtype=torch.bfloat16, device="cuda")
+    wide[:, 128:128 + F] = bf(a)
+    got = hstu.hstu_layernorm_fwd(wide[:, 128:128 + F], dev(g), None, 1e-3)
+    assert_bf16_close(got.float().cpu().numpy(), oracle.layernorm(a, g, None, 1e-3), "strided")
+    assert hstu.hstu_layernorm_fwd(bf(a[:0])).shape == (0, F)
+
+
+def _shifted(li):
+    """Layer inputs whose rows have a mean and a spread far from 0 and 1, so the
+    input normalization changes x (the workload's x is N(0, 1) per element)."""
+    rng = np.random.default_rng(li.seed + 1)
+    T, D = li.x.shape
+    x = li.x * rng.uniform(0.3, 2.5, (T, 1)) + rng.uniform(-1.5, 1.5, (T, 1))
+    return dataclasses.replace(li, x=round_to_bf16(x.astype(np.float32)))
+
+
+def _in_affine(D, seed=9):
+    rng = np.random.default_rng(seed)
+    return ((1 + 0.2 * rng.standard_normal(D)).astype(np.float32),
+            (0.2 * rng.standard_normal(D)).astype(np.float32))
+
+
+def test_layer_input_norm_small_full():
+    li = _shifted(make_layer_inputs(5, lengths_override=[130, 0, 1, 257, 40]))
+    ig, ib = _in_affine(li.x.shape[1])
+    got = _layer_gpu(li, input_norm=True, in_gamma=dev(ig), in_beta=dev(ib))
+    want = oracle.layer(li.seq_offsets, li.x, li.W1, li.W2, li.H, li.d, li.timestamps,
+                        li.pos_bias, li.time_bias, li.max_seqlen, ln_eps=li.ln_eps,
+                        input_norm=True, in_gamma=ig, in_beta=ib)
+    assert_bf16_close(got - li.x, want - li.x, "layer input norm (out - x)")
+    # without the affine terms, and the normalization is really applied
+    got = _layer_gpu(li, input_norm=True)
+    want = oracle.layer(li.seq_offsets, li.x, li.W1, li.W2, li.H, li.d, li.timestamps,
+                        li.pos_bias, li.time_bias, li.max_seqlen, ln_eps=li.ln_eps,
+                        input_norm=True)
+    assert_bf16_close(got - li.x, want - li.x, "layer input norm identity (out - x)")
+    plain = _layer_gpu(li)
+    rel, _ = errors(plain - li.x, want - li.x)
+    assert rel > 0.1, rel
+
+
+def test_layer_input_norm_workload_sampled_rows():
+    li = _shifted(make_layer_inputs(5))
+    ig, ib = _in_affine(li.x.shape[1])
+    got = _layer_gpu(li, input_norm=True, in_gamma=dev(ig), in_beta=dev(ib))
+    assert np.all(np.isfinite(got))
+    off, lens = li.seq_offsets, np.diff(li.seq_offsets)
+    rows = []
+    for s in (int(np.argmin(lens)), 5, 29):
+        o, n = int(off[s]), int(lens[s])
+        rows += [o, o + 64, o + n // 3, o + n - 1]
+    rows = np.array(sorted(set(r for r in rows if r < li.T)), dtype=np.int64)
+    want = oracle.layer(li.seq_offsets, li.x, li.W1, li.W2, li.H, li.d, li.timestamps,
+                        li.pos_bias, li.time_bias, li.max_seqlen, ln_eps=li.ln_eps, rows=rows,
+                        input_norm=True, in_gamma=ig, in_beta=ib)
+    assert_bf16_close(got[rows] - li.x[rows], want - li.x[rows], "layer input norm workload")
