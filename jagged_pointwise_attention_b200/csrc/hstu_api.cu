@@ -155,6 +155,27 @@ int num_sms() {
     return cached[dev];
 }
 
+// Grid for a kernel whose blocks stride over `blocks` units of work: at most
+// as many blocks as fit on the device at once, so none waits for a second
+// wave. `cache` holds the per-device count of resident blocks per SM.
+template <typename K>
+unsigned resident_grid(K kernel, int threads, int64_t blocks, int* cache) {
+    int dev = 0;
+    int per_sm = 1;
+    if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices) {
+        if (cache[dev] == 0) {
+            int n = 0;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, 0) !=
+                    cudaSuccess || n < 1)
+                n = 1;
+            cache[dev] = n;
+        }
+        per_sm = cache[dev];
+    }
+    const int64_t cap = static_cast<int64_t>(num_sms()) * per_sm;
+    return static_cast<unsigned>(blocks < cap ? blocks : cap);
+}
+
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 bool plan_sizes_ok(int32_t B, int64_t T, int32_t max_seqlen) {
@@ -362,11 +383,12 @@ template <int EPI, int BN, bool FP8 = false>
 hstu_status_t launch_gemm(unsigned grid, cudaStream_t stream, const CUtensorMap& ta,
                           const CUtensorMap& tb, const CUtensorMap& ty, const CUtensorMap& tr,
                           const GemmArgs& g) {
+    constexpr int EW = GemmEpiWarps<EPI, FP8>::value;
     static int done[kMaxDevices] = {0};
-    if (!ensure_smem(gemm_bf16_kernel<EPI, BN, FP8>, GemmSmem<BN>::kAlloc, done))
+    if (!ensure_smem(gemm_bf16_kernel<EPI, BN, FP8>, GemmSmem<BN, EW>::kAlloc, done))
         return HSTU_ERR_CUDA;
     gemm_bf16_kernel<EPI, BN, FP8>
-        <<<grid, kGemmThreads, GemmSmem<BN>::kAlloc, stream>>>(ta, tb, ty, tr, g);
+        <<<grid, (EW + 2) * 32, GemmSmem<BN, EW>::kAlloc, stream>>>(ta, tb, ty, tr, g);
     return launch_status();
 }
 
@@ -457,20 +479,26 @@ hstu_status_t run_ln_gate_any(bool quant, bool gate, const void* a, int64_t lda,
     LnGateArgs args{static_cast<const __nv_bfloat16*>(a), lda, static_cast<const __nv_bfloat16*>(u),
                     ldu, M, gamma, beta, eps, static_cast<__nv_bfloat16*>(y), ldy,
                     static_cast<uint8_t*>(yq), ldyq, ys};
-    // eight rows per block and pass; up to eight blocks per SM, each striding
-    // over the rows
-    const int64_t blocks = (M + 7) / 8, cap = static_cast<int64_t>(num_sms()) * 8;
-    const unsigned grid = static_cast<unsigned>(blocks < cap ? blocks : cap);
-#define HSTU_LN_CASES(Q, GT)                                                        \
-    switch (F / 256) {                                                              \
-        case 1: ln_gate_kernel<1, Q, GT><<<grid, 256, 0, stream>>>(args); break;    \
-        case 2: ln_gate_kernel<2, Q, GT><<<grid, 256, 0, stream>>>(args); break;    \
-        case 3: ln_gate_kernel<3, Q, GT><<<grid, 256, 0, stream>>>(args); break;    \
-        case 4: ln_gate_kernel<4, Q, GT><<<grid, 256, 0, stream>>>(args); break;    \
-        case 5: ln_gate_kernel<5, Q, GT><<<grid, 256, 0, stream>>>(args); break;    \
-        case 6: ln_gate_kernel<6, Q, GT><<<grid, 256, 0, stream>>>(args); break;    \
-        case 7: ln_gate_kernel<7, Q, GT><<<grid, 256, 0, stream>>>(args); break;    \
-        default: ln_gate_kernel<8, Q, GT><<<grid, 256, 0, stream>>>(args); break;   \
+    // eight rows per block and pass; as many blocks as are resident at once,
+    // each striding over the rows
+    const int64_t blocks = (M + 7) / 8;
+#define HSTU_LN_LAUNCH(NV, Q, GT)                                                       \
+    {                                                                                   \
+        static int occ[kMaxDevices] = {0};                                              \
+        const unsigned grid = resident_grid(ln_gate_kernel<NV, Q, GT>, 256, blocks, occ); \
+        ln_gate_kernel<NV, Q, GT><<<grid, 256, 0, stream>>>(args);                      \
+        break;                                                                          \
+    }
+#define HSTU_LN_CASES(Q, GT)                     \
+    switch (F / 256) {                           \
+        case 1: HSTU_LN_LAUNCH(1, Q, GT)         \
+        case 2: HSTU_LN_LAUNCH(2, Q, GT)         \
+        case 3: HSTU_LN_LAUNCH(3, Q, GT)         \
+        case 4: HSTU_LN_LAUNCH(4, Q, GT)         \
+        case 5: HSTU_LN_LAUNCH(5, Q, GT)         \
+        case 6: HSTU_LN_LAUNCH(6, Q, GT)         \
+        case 7: HSTU_LN_LAUNCH(7, Q, GT)         \
+        default: HSTU_LN_LAUNCH(8, Q, GT)        \
     }
     if (quant && gate) {
         HSTU_LN_CASES(true, true)
@@ -482,6 +510,7 @@ hstu_status_t run_ln_gate_any(bool quant, bool gate, const void* a, int64_t lda,
         HSTU_LN_CASES(false, false)
     }
 #undef HSTU_LN_CASES
+#undef HSTU_LN_LAUNCH
     return launch_status();
 }
 
