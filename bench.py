@@ -729,30 +729,45 @@ def e2e_layer(args, li, dev, stream, flops, world, layer_call):
                         "i-2's device-to-host copy (three streams, two buffer sets)"}
 
 
-def bench_backward(args, rank, world, local, peaks, peak_kind):
-    """The fp32 attention backward on the --config workload (its lengths,
-    heads, head dimension and bias tables, inputs in fp32). Algorithmic FLOPs:
-    the four contractions dV = P^T dO, dP = dO V^T, dQ = dS K, dK = dS^T Q over
-    the causal pairs, twice the forward's. The kernels run on CUDA cores, so
-    the roofline is fp32 FMA: SMs x 128 lanes x 2 FLOP x the max SM clock."""
+def bench_backward(args, rank, world, local, peaks, peak_kind, cfg_id=None):
+    """The attention backward on tensor cores (hstu_attn_bwd: bf16 inputs,
+    fp32 gradients) on an attention workload (its lengths, heads, head
+    dimension and bias tables). One step: the clears of dq and the table
+    gradients, the plan, the backward kernel. Algorithmic FLOPs: the four
+    contractions dV = P^T dO, dP = dO V^T, dQ = dS K, dK = dS^T Q over the
+    causal pairs, twice the forward's (the kernel also recomputes S = Q K^T,
+    which is not counted). Roofline: those FLOPs against the dense bf16 peak."""
     import torch
     import jagged_pointwise_attention_b200 as hstu
     from gen import CONFIGS, make_attn_inputs
-    cfg = CONFIGS[args.config]
+    cfg_id = args.config if cfg_id is None else cfg_id
+    cfg = CONFIGS[cfg_id]
     if cfg["kind"] == "layer":
         raise SystemExit("--backward takes an attention workload (--config 2, 3 or 4)")
-    inp = make_attn_inputs(args.config, seed=1000 + args.config + 7919 * rank)
+    seed = 1000 + cfg_id + 7919 * rank
+    inp = make_attn_inputs(cfg_id, seed=seed)
     dev = torch.device("cuda", local)
+    bf = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(dev).to(torch.bfloat16)  # noqa: E731
     f32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(dev)  # noqa: E731
     i64 = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)  # noqa: E731
-    q, k, v = f32(inp.q), f32(inp.k), f32(inp.v)
-    dout = torch.randn(v.shape, generator=torch.Generator().manual_seed(7), dtype=torch.float32).to(dev)
+    q, k, v = bf(inp.q), bf(inp.k), bf(inp.v)
+    dout = torch.randn(v.shape, generator=torch.Generator().manual_seed(7),
+                       dtype=torch.float32).to(dev).to(torch.bfloat16)
     off, ts, pos, tb = i64(inp.seq_offsets), i64(inp.timestamps), f32(inp.pos_bias), f32(inp.time_bias)
     lengths = np.diff(inp.seq_offsets)
-    flops = 2 * causal_flops(lengths, inp.H, inp.q.shape[2], inp.v.shape[2])
+    d = int(inp.q.shape[2])
+    flops = 2 * causal_flops(lengths, inp.H, d, int(inp.v.shape[2]))
+    T, H = inp.T, inp.H
+    outs = (torch.empty((T, H, d), dtype=torch.float32, device=dev),
+            torch.empty((T, H, d), dtype=torch.float32, device=dev),
+            torch.empty((T, H, d), dtype=torch.float32, device=dev),
+            torch.empty_like(pos), torch.empty_like(tb))
+    ws = torch.empty(hstu.hstu_attn_bwd_workspace_bytes(inp.B, T, inp.max_seqlen),
+                     dtype=torch.uint8, device=dev)
 
     def step():
-        hstu.hstu_attn_bwd_f32(q, k, v, dout, off, ts, pos, tb, inp.max_seqlen)
+        hstu.hstu_attn_bwd(q, k, v, dout, off, ts, pos, tb, inp.max_seqlen, workspace=ws,
+                           out=outs)
 
     for _ in range(args.warmup):
         step()
@@ -769,25 +784,29 @@ def bench_backward(args, rank, world, local, peaks, peak_kind):
     torch.cuda.synchronize(dev)
     sampler.stop()
     _barrier(world)
+    assert hstu.hstu_device_status() == 0
     max_ms, tot = reduce_timing(e0.elapsed_time(e1), float(flops) * args.steps, world, dev)
     value = tot / (max_ms * 1e-3) / 1e12
-    clocks = sampler.summary()
-    sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    peak = sms * 128 * 2 * (clocks.get("sm_max_mhz") or 1965) * 1e6 / 1e12
-    return {"metric": "HSTU jagged attn bwd TFLOP/s (causal, fp32 CUDA cores)",
+    step_tf = flops / (max_ms / args.steps * 1e-3) / 1e12
+    in_mb = 4 * T * H * d * 2 / 2 ** 20
+    return {"metric": "HSTU jagged attn bwd TFLOP/s (causal, bf16 tensor cores)",
             "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(max_ms / args.steps, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16 inputs, fp32 gradients",
             "data": "synthetic (seeded generator; no dataset)",
-            "config": {"workload": cfg["name"] + "_backward_f32", "B": inp.B, "H": inp.H,
-                       "d": int(inp.q.shape[2]), "total_tokens": inp.T,
-                       "parallelism": "dp%d" % world},
-            "roofline": {"bound": "alu", "achieved": round(value, 3), "peak": round(peak, 1),
-                         "unit": "TFLOP/s", "frac": round(value / peak, 4),
-                         "peak_kind": "fp32 FMA: %d SMs x 128 lanes x 2 x max SM clock" % sms,
-                         "traffic": None,
-                         "kernel": "attn_bwd_q_kernel + attn_bwd_kv_kernel"},
-            "gpu_launches": 2 * args.steps, "clocks": clocks}
+            "config": {"workload": cfg["name"] + "_backward", "B": inp.B, "H": H, "d": d,
+                       "total_tokens": T, "seed": seed, "parallelism": "dp%d" % world,
+                       "l2": "q, k, v, dout %.0f MB, dq/dk/dv %.0f MB: %s" % (
+                           in_mb, 3 * T * H * d * 4 / 2 ** 20,
+                           "inputs larger than L2" if in_mb > 126 else
+                           "short workload: inputs fit in L2 (timed back to back)")},
+            "roofline": {"bound": "tensor", "achieved": round(step_tf, 2),
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": round(step_tf / peaks["bf16_tflops"], 4),
+                         "peak_kind": "burst bf16 dense, %s" % peak_kind, "traffic": None,
+                         "kernel": "whole backward step (clears, plan, attn_bwd_bf16_kernel)"},
+            "gpu_launches": 2 * args.steps, "clocks": sampler.summary()}
 
 
 def bench_fp8_linear(args, rank, world, local, peaks, peak_kind):
@@ -953,8 +972,8 @@ def parse_args(argv=None):
                     help="with --config 5: LayerNorm on the layer's input before f1 (fused with "
                          "the E4M3 quantization under --fp8)")
     ap.add_argument("--backward", action="store_true",
-                    help="time the fp32 attention backward (hstu_attn_bwd_f32) on the "
-                         "--config workload's shapes instead of the forward")
+                    help="time the tensor-core attention backward (hstu_attn_bwd) on the "
+                         "--config workload instead of the forward")
     ap.add_argument("--fp8-linear", action="store_true",
                     help="time the row-wise E4M3 projections (quantize + FP8 GEMM) against the "
                          "bf16 ones on the projection shapes instead of the attention")
@@ -986,7 +1005,7 @@ def main(argv=None):
     from gen import CONFIGS
     if args.backward or args.fp8_linear:
         if args.config is None:
-            args.config = 2 if args.backward else 4
+            args.config = 4
         fn = bench_backward if args.backward else bench_fp8_linear
         line = fn(args, rank, world, local, peaks, kind)
     elif args.config is not None:
@@ -1011,6 +1030,10 @@ def main(argv=None):
             name = sub["config"]["workload"] + ("_fp8" if fp8 else "") + ("_input_ln" if norm
                                                                           else "")
             subs[name] = sub
+        # the attention backward on the long and the short-history workloads
+        for c in (4, 2):
+            sub = bench_backward(args, rank, world, local, peaks, kind, cfg_id=c)
+            subs[sub["config"]["workload"]] = sub
         line["configs"] = subs
         line["gpu_launches_all_lines"] = line["gpu_launches"] + sum(
             v["gpu_launches"] for v in subs.values())

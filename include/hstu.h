@@ -18,7 +18,7 @@
  * with silu(x) = x * sigmoid(x). No softmax, no 1/sqrt(d) score scale.
  * Sections below: the attention; the layer around it (projections, the
  * input and output LayerNorms, the whole layer); row-wise E4M3 (FP8)
- * projections; the attention backward (fp32).
+ * projections; the attention backward (bf16 on tensor cores, and fp32).
  *
  * Conventions for every entry point:
  *  - Pointers marked "device" must be device memory of the current CUDA device
@@ -368,6 +368,32 @@ hstu_status_t hstu_attn_bwd_f32(const float* q, const float* k, const float* v, 
                                 const float* pos_bias, int32_t num_pos, const float* time_bias,
                                 int32_t num_time_buckets, int32_t max_seqlen, float* dq, float* dk,
                                 float* dv, float* dpos, float* dtime, void* stream);
+
+/* Gradients of the attention on tensor cores (tcgen05), bf16 inputs, same
+ * formulas as hstu_attn_bwd_f32. q, k, v, dout: device bf16 [T, H, d] with
+ * per-token strides q_stride .. dout_stride in elements (multiples of 8, at
+ * least H*d; heads contiguous in a token), d = d_qk = d_v in {64, 128}
+ * (HSTU_ERR_UNSUPPORTED otherwise, and for dtype HSTU_DTYPE_F32: use
+ * hstu_attn_bwd_f32). Outputs are fp32, contiguous [T, H, d] and 16-byte
+ * aligned: dq is zeroed and accumulated; dk and dv rows are written for
+ * every token of a sequence (rows of tokens outside every sequence are left
+ * as they are); dpos [H, num_pos] (required when pos_bias is given) and dtime
+ * [H, num_time_buckets] (required when timestamps and time_bias are) are
+ * zeroed and accumulated. Products are rounded as in the forward: p and ds
+ * in bf16, sums in fp32; table gradients and dq are accumulated with
+ * atomics, so their last bits may differ between runs. `workspace` (device,
+ * 16-byte aligned, hstu_attn_bwd_workspace_bytes(B, T, max_seqlen) bytes)
+ * holds the work list; one plan launch, one backward launch, and the
+ * clears. Other arguments as hstu_attn_fwd. Asynchronous on `stream`. */
+size_t hstu_attn_bwd_workspace_bytes(int32_t B, int64_t total_tokens, int32_t max_seqlen);
+hstu_status_t hstu_attn_bwd(hstu_dtype_t dtype, const void* q, int64_t q_stride, const void* k,
+                            int64_t k_stride, const void* v, int64_t v_stride, const void* dout,
+                            int64_t dout_stride, const int64_t* seq_offsets, int32_t B,
+                            int64_t total_tokens, int32_t H, int32_t d, const int64_t* timestamps,
+                            const float* pos_bias, int32_t num_pos, const float* time_bias,
+                            int32_t num_time_buckets, int32_t max_seqlen, float* dq, float* dk,
+                            float* dv, float* dpos, float* dtime, void* workspace,
+                            size_t workspace_bytes, void* stream);
 
 #ifdef __cplusplus
 }

@@ -25,7 +25,7 @@ __all__ = [
     "hstu_attn_fwd", "hstu_attn_plan", "hstu_attn_run", "hstu_attn_workspace_bytes",
     "hstu_layer_fwd", "hstu_layer_workspace_bytes", "hstu_linear_fwd",
     "hstu_layernorm_gate_fwd", "hstu_debug_bias_indices", "hstu_debug_wait_timeout",
-    "hstu_attn_bwd_f32", "hstu_quant_rows_e4m3", "hstu_linear_fp8_fwd",
+    "hstu_attn_bwd", "hstu_attn_bwd_workspace_bytes", "hstu_attn_bwd_f32", "hstu_quant_rows_e4m3", "hstu_linear_fp8_fwd",
     "hstu_layernorm_gate_fp8_fwd", "hstu_layernorm_fwd", "hstu_layernorm_fp8_fwd",
     "hstu_layer_fp8_workspace_bytes", "hstu_layer_fp8_fwd",
     "hstu_device_status", "HstuError", "library_path",
@@ -367,6 +367,45 @@ def hstu_layer_fp8_fwd(x: torch.Tensor, W1q: torch.Tensor, w1_scales: torch.Tens
         _ptr(time_bias), 0 if time_bias is None else time_bias.shape[1], int(max_seqlen),
         _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream)))
     return out
+
+
+def hstu_attn_bwd_workspace_bytes(B: int, total_tokens: int, max_seqlen: int) -> int:
+    return int(_lib().hstu_attn_bwd_workspace_bytes(B, total_tokens, max_seqlen))
+
+
+def hstu_attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dout: torch.Tensor,
+                  seq_offsets: torch.Tensor, timestamps: Optional[torch.Tensor],
+                  pos_bias: Optional[torch.Tensor], time_bias: Optional[torch.Tensor],
+                  max_seqlen: int, workspace: Optional[torch.Tensor] = None, out=None,
+                  stream=None):
+    """Gradients of the attention on tensor cores for the upstream gradient
+    dout: q, k, v, dout bf16 [T, H, d] (d = 64 or 128, heads contiguous per
+    token, any token stride); returns fp32 (dq, dk, dv, dpos, dtime), dpos /
+    dtime None when the term is absent. `out` may pass preallocated (dq, dk,
+    dv, dpos, dtime)."""
+    _on_cuda(q, k, v, dout, seq_offsets, timestamps, pos_bias, time_bias)
+    for t in (q, k, v, dout):
+        if t.dtype != torch.bfloat16 or t.stride(2) != 1 or t.stride(1) != t.shape[2]:
+            raise ValueError("q, k, v, dout must be bf16 with heads contiguous in a token")
+    T, H, d = q.shape
+    B = seq_offsets.numel() - 1
+    use_time = timestamps is not None and time_bias is not None
+    if out is None:
+        f32 = dict(dtype=torch.float32, device=q.device)
+        out = (torch.empty((T, H, d), **f32), torch.empty((T, H, d), **f32),
+               torch.empty((T, H, d), **f32),
+               None if pos_bias is None else torch.empty_like(pos_bias),
+               torch.empty_like(time_bias) if use_time else None)
+    dq, dk, dv, dpos, dtime = out
+    if workspace is None:
+        workspace = _workspace(hstu_attn_bwd_workspace_bytes(B, T, max_seqlen), q.device)
+    _native.check("hstu_attn_bwd", _lib().hstu_attn_bwd(
+        _native.HSTU_DTYPE_BF16, _ptr(q), q.stride(0), _ptr(k), k.stride(0), _ptr(v), v.stride(0),
+        _ptr(dout), dout.stride(0), _ptr(seq_offsets), B, T, H, d, _ptr(timestamps),
+        _ptr(pos_bias), 0 if pos_bias is None else pos_bias.shape[1], _ptr(time_bias),
+        0 if time_bias is None else time_bias.shape[1], int(max_seqlen), _ptr(dq), _ptr(dk),
+        _ptr(dv), _ptr(dpos), _ptr(dtime), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return dq, dk, dv, dpos, dtime
 
 
 def hstu_attn_bwd_f32(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dout: torch.Tensor,

@@ -36,6 +36,10 @@ SIGNATURES = {
     "hstu_attn_bwd_f32": (ctypes.c_int, [c_p, c_p, c_p, c_p, c_p, c_i32, c_i64, c_i32, c_i32,
                                          c_i32, c_p, c_p, c_i32, c_p, c_i32, c_i32, c_p, c_p, c_p,
                                          c_p, c_p, c_p]),
+    "hstu_attn_bwd_workspace_bytes": (c_sz, [c_i32, c_i64, c_i32]),
+    "hstu_attn_bwd": (ctypes.c_int, [ctypes.c_int, c_p, c_i64, c_p, c_i64, c_p, c_i64, c_p, c_i64,
+                                     c_p, c_i32, c_i64, c_i32, c_i32, c_p, c_p, c_i32, c_p, c_i32,
+                                     c_i32, c_p, c_p, c_p, c_p, c_p, c_p, c_sz, c_p]),
     "hstu_quant_rows_e4m3": (ctypes.c_int, [c_p, c_i64, c_i64, c_i32, c_p, c_i64, c_p, c_p]),
     "hstu_linear_fp8_fwd": (ctypes.c_int, [c_p, c_i64, c_p, c_i64, c_i32, c_p, c_i64, c_p, c_i32,
                                            c_p, ctypes.c_int, c_p, c_i64, c_p, c_i64, c_p]),

@@ -12,6 +12,7 @@
 
 #include "hstu.h"
 #include "attn_bwd_simt.cuh"
+#include "attn_bwd_tc.cuh"
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
 #include "bias_prep.cuh"
@@ -63,6 +64,22 @@ bool make_tmap_bf16_box(CUtensorMap* tm, const void* base, uint64_t inner, uint6
     const CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// fp32 [rows, inner] with boxes of 32 x 32 (128-byte rows, 128-byte swizzle).
+bool make_tmap_f32_32(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t rows,
+                      uint64_t row_stride_bytes) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {row_stride_bytes};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -716,6 +733,80 @@ hstu_status_t hstu_attn_bwd_f32(const float* q, const float* k, const float* v, 
     } else {
         attn_bwd_q_kernel<128><<<grid, 128, tab_bytes, s>>>(a);
         attn_bwd_kv_kernel<128><<<grid, 128, 0, s>>>(a);
+    }
+    return launch_status();
+}
+
+size_t hstu_attn_bwd_workspace_bytes(int32_t B, int64_t total_tokens, int32_t max_seqlen) {
+    if (!plan_sizes_ok(B, total_tokens, max_seqlen)) return 0;
+    return attn_plan_bytes(B, total_tokens, max_seqlen);
+}
+
+hstu_status_t hstu_attn_bwd(hstu_dtype_t dtype, const void* q, int64_t q_stride, const void* k,
+                            int64_t k_stride, const void* v, int64_t v_stride, const void* dout,
+                            int64_t dout_stride, const int64_t* seq_offsets, int32_t B,
+                            int64_t total_tokens, int32_t H, int32_t d, const int64_t* timestamps,
+                            const float* pos_bias, int32_t num_pos, const float* time_bias,
+                            int32_t num_time_buckets, int32_t max_seqlen, float* dq, float* dk,
+                            float* dv, float* dpos, float* dtime, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+    const int64_t T = total_tokens;
+    if (dtype != HSTU_DTYPE_BF16 && dtype != HSTU_DTYPE_F32) return HSTU_ERR_INVALID_ARG;
+    if (!plan_sizes_ok(B, T, max_seqlen) || H < 1 || d < 1) return HSTU_ERR_INVALID_ARG;
+    if (dtype != HSTU_DTYPE_BF16 || (d != 64 && d != 128)) return HSTU_ERR_UNSUPPORTED;
+    if (pos_bias && num_pos < 1) return HSTU_ERR_INVALID_ARG;
+    const bool use_time = timestamps && time_bias;
+    if (use_time && (num_time_buckets < 1 || num_time_buckets > kMaxTimeBuckets))
+        return HSTU_ERR_INVALID_ARG;
+    if ((pos_bias && !dpos) || (use_time && !dtime)) return HSTU_ERR_INVALID_ARG;
+    cudaStream_t s = as_stream(stream);
+    const int P = pos_bias ? num_pos : 0, NB = use_time ? num_time_buckets : 0;
+    if (pos_bias && cudaMemsetAsync(dpos, 0, static_cast<size_t>(H) * P * sizeof(float), s) != cudaSuccess)
+        return HSTU_ERR_CUDA;
+    if (use_time &&
+        cudaMemsetAsync(dtime, 0, static_cast<size_t>(H) * NB * sizeof(float), s) != cudaSuccess)
+        return HSTU_ERR_CUDA;
+    if (B == 0 || T == 0) return HSTU_OK;
+    if (!q || !k || !v || !dout || !seq_offsets || !dq || !dk || !dv || !workspace)
+        return HSTU_ERR_INVALID_ARG;
+    const int64_t row = int64_t{H} * d;
+    if (q_stride < row || k_stride < row || v_stride < row || dout_stride < row || q_stride % 8 ||
+        k_stride % 8 || v_stride % 8 || dout_stride % 8)
+        return HSTU_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq) ||
+        !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
+        return HSTU_ERR_INVALID_ARG;
+    if (workspace_bytes < attn_plan_bytes(B, T, max_seqlen)) return HSTU_ERR_INVALID_ARG;
+    if (cudaMemsetAsync(dq, 0, static_cast<size_t>(T) * row * sizeof(float), s) != cudaSuccess)
+        return HSTU_ERR_CUDA;
+    hstu_status_t st = launch_plan(seq_offsets, B, T, max_seqlen, workspace, s);
+    if (st != HSTU_OK) return st;
+    CUtensorMap tq, tk, tv, tdo, tdq;
+    if (!make_tmap_bf16(&tq, q, row, T, q_stride * 2, 128) ||
+        !make_tmap_bf16(&tk, k, row, T, k_stride * 2, 128) ||
+        !make_tmap_bf16(&tv, v, row, T, v_stride * 2, 128) ||
+        !make_tmap_bf16(&tdo, dout, row, T, dout_stride * 2, 128) ||
+        !make_tmap_f32_32(&tdq, dq, row, T, row * 4))
+        return HSTU_ERR_CUDA;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    BwdArgs a{reinterpret_cast<const int4*>(ws + kAttnWsHeader), reinterpret_cast<const int*>(ws),
+              static_cast<int>(max_units_of(B, T, max_seqlen)),
+              reinterpret_cast<const uint4*>(ws + kAttnWsHeader + attn_units_bytes(B, T, max_seqlen)),
+              H, T, use_time ? timestamps : nullptr, pos_bias, P > 0 ? P : 1,
+              use_time ? time_bias : nullptr, NB > 0 ? NB : 1,
+              1.0f / static_cast<float>(max_seqlen), dq, dk, dv, pos_bias ? dpos : nullptr,
+              use_time ? dtime : nullptr};
+    const unsigned grid = static_cast<unsigned>(num_sms());
+    if (d == 64) {
+        static int done[kMaxDevices] = {0};
+        if (!ensure_smem(attn_bwd_bf16_kernel<64>, BwdSmem<64>::kAlloc, done)) return HSTU_ERR_CUDA;
+        attn_bwd_bf16_kernel<64><<<grid, BwdCfg<64>::kThreads, BwdSmem<64>::kAlloc, s>>>(
+            tq, tk, tv, tdo, tdq, a);
+    } else {
+        static int done[kMaxDevices] = {0};
+        if (!ensure_smem(attn_bwd_bf16_kernel<128>, BwdSmem<128>::kAlloc, done)) return HSTU_ERR_CUDA;
+        attn_bwd_bf16_kernel<128><<<grid, BwdCfg<128>::kThreads, BwdSmem<128>::kAlloc, s>>>(
+            tq, tk, tv, tdo, tdq, a);
     }
     return launch_status();
 }

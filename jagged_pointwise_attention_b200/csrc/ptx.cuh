@@ -128,6 +128,17 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* tm, const void* 
         : "memory");
 }
 
+// Element-wise add of a shared-memory box into global memory through a
+// tensor map (fp32 maps: float add); rows past the tensor are clipped.
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* tm, const void* src, int32_t x,
+                                                  int32_t y) {
+    asm volatile(
+        "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(tm)),
+        "r"(smem_u32(src)), "r"(x), "r"(y)
+        : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit_group() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }

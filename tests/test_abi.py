@@ -177,6 +177,38 @@ def test_backward_validation(lib):
     assert bwd(B=0, T=0) == 0
 
 
+def test_tc_backward_validation(lib):
+    INV, UNS = _native.HSTU_ERR_INVALID_ARG, _native.HSTU_ERR_UNSUPPORTED
+    BF16, F32 = _native.HSTU_DTYPE_BF16, _native.HSTU_DTYPE_F32
+
+    def bwd(**kw):
+        a = dict(dt=BF16, q=16, qs=256, k=16, ks=256, v=16, vs=256, dout=16, dos=256, off=16, B=2,
+                 T=10, H=2, d=128, ts=None, pos=None, P=0, tb=None, NB=0, N=8, dq=16, dk=16,
+                 dvv=16, dpos=None, dtime=None, ws=16, wsb=1 << 20)
+        a.update(kw)
+        return lib.hstu_attn_bwd(a["dt"], a["q"], a["qs"], a["k"], a["ks"], a["v"], a["vs"],
+                                 a["dout"], a["dos"], a["off"], a["B"], a["T"], a["H"], a["d"],
+                                 a["ts"], a["pos"], a["P"], a["tb"], a["NB"], a["N"], a["dq"],
+                                 a["dk"], a["dvv"], a["dpos"], a["dtime"], a["ws"], a["wsb"], None)
+    assert bwd(d=32) == UNS
+    assert bwd(d=96) == UNS
+    assert bwd(dt=F32) == UNS                           # the fp32 path is hstu_attn_bwd_f32
+    assert bwd(dt=7) == INV
+    assert bwd(H=0) == INV
+    assert bwd(pos=16, P=8) == INV                      # dpos missing
+    assert bwd(ts=16, tb=16, NB=8) == INV               # dtime missing
+    assert bwd(ts=16, tb=16, NB=2000, dtime=16) == INV  # bucket count
+    assert bwd(q=None) == INV
+    assert bwd(ws=None) == INV
+    assert bwd(qs=255) == INV                           # stride below H * d
+    assert bwd(ks=264 + 4) == INV                       # stride not a multiple of 8
+    assert bwd(dq=20) == INV                            # fp32 outputs 16-byte aligned
+    assert bwd(wsb=8) == INV                            # workspace below the plan's size
+    assert bwd(B=0, T=0) == 0
+    assert lib.hstu_attn_bwd_workspace_bytes(4, 1000, 512) >= 256
+    assert lib.hstu_attn_bwd_workspace_bytes(-1, 1000, 512) == 0
+
+
 def test_binding_fails_loudly_without_library(tmp_path):
     with pytest.raises(ImportError):
         _native.load(str(tmp_path / "missing.so"))
