@@ -28,11 +28,14 @@
 // reductions (staged through the dS^T buffer, free once dQ_i is computed);
 // after the item's last step they store dK_j and dV_j (fp32).
 //
-// Warp roles: 0-7 pointwise (two warps per TMEM lane quarter, 64 query
-// columns each), 8 TMA producer, 9 MMA issuer and TMEM owner.
+// Warp roles: 0-15 pointwise (four warps per TMEM lane quarter, one 32-column
+// chunk of queries each: with four warps per scheduler one warp's TMEM, SFU
+// and shared-memory latencies hide behind the others' arithmetic), 16 TMA
+// producer, 17 MMA issuer and TMEM owner.
 //
 // Pointwise arithmetic per pair in fp32: s = S + pos + time; one tanh gives
-// sg = 1/2 + tanh(s/2)/2, then p and ds. Before each step the pointwise warps
+// sg = 1/2 + tanh(s/2)/2, then p and ds without the factor 1/N, which is
+// applied once to every gradient as it leaves the kernel. Before each step the pointwise warps
 // stage the step's bias data in shared memory: the 255 position-table values
 // the tile's diagonals read, the 128 query timestamps with each 32-column
 // chunk's smallest and largest, and the head's time-table row. The time
@@ -85,9 +88,10 @@ struct BwdCfg {
     static_assert(D == 64 || D == 128, "head dimension");
     static constexpr int kKB = D / 64;                      // 64-column blocks of a tile
     static constexpr int kTileBytes = kTile * D * 2;
-    static constexpr int kPointwiseThreads = 256;
-    static constexpr int kWarpTMA = 8, kWarpMMA = 9;
-    static constexpr int kThreads = 320;
+    static constexpr int kPointwiseWarps = 16;
+    static constexpr int kPointwiseThreads = 32 * kPointwiseWarps;
+    static constexpr int kWarpTMA = kPointwiseWarps, kWarpMMA = kPointwiseWarps + 1;
+    static constexpr int kThreads = 32 * (kPointwiseWarps + 2);
     static constexpr uint32_t kColS = 0, kColP = 128, kColV = 256, kColK = 256 + D;
 };
 
@@ -104,9 +108,9 @@ struct BwdSmem {
     static constexpr int kOffQts = kOffPosW + 1024;                // 128 query timestamps
     static constexpr int kOffCmm = kOffQts + 1024;                 // per chunk: min, max timestamp
     static constexpr int kOffTb = kOffCmm + 64;                    // 64 floats: the head's time table
-    static constexpr int kOffDiag = kOffTb + 256;                  // [8 warps][2 chunks][64] diagonal sums
-    static constexpr int kOffTslot = kOffDiag + 8 * 128 * 4;       // [8 warps][64] bucket sums
-    static constexpr int kOffBar = kOffTslot + 8 * 64 * 4;
+    static constexpr int kOffDiag = kOffTb + 256;                  // [16 warps][64] diagonal sums
+    static constexpr int kOffTslot = kOffDiag + 16 * 64 * 4;       // [16 warps][64] bucket sums
+    static constexpr int kOffBar = kOffTslot + 16 * 64 * 4;
     static constexpr int kNumBars = 18;
     static constexpr int kOffTmem = kOffBar + kNumBars * 8;
     static constexpr int kOffAbort = kOffTmem + 8;
@@ -218,70 +222,107 @@ __device__ __forceinline__ void warp_bucket_add(float* slots, bool has, int b, f
     __syncwarp();
 }
 
-// The pointwise work of one 32-column chunk for one key row (lane): s, p, ds;
-// P^T and dS^T packed as bf16 pairs; the chunk's diagonal sums of ds into
-// the warp's chunk area (entry 31 + e - lane for pair (lane, e)); the time
-// gradient by bucket. TM: 0 = one bucket per row over the chunk (b0), 1 = at
-// most four buckets per row (b0 .. b0 + 3, summed in registers), 2 = any.
-// Straight-line code over the 32 pairs for TM 0 and 1.
+// Shared-memory store by lane 31 only, as a predicated instruction (no branch
+// in the straight-line pair loop).
+__device__ __forceinline__ void st_shared_if_lane31(float* p, float v, int lane) {
+    asm volatile(
+        "{\n\t.reg .pred q;\n\tsetp.eq.u32 q, %2, 31;\n\t@q st.shared.f32 [%0], %1;\n\t}" ::"r"(
+            smem_u32(p)),
+        "f"(v), "r"(lane));
+}
+
+// The pointwise work of one 32-column chunk for one key row (lane), in two
+// halves of 16 columns: s, p = silu(s) and ds = dp silu'(s), both without
+// the 1/N (applied to the sums at the end); P^T packed as bf16 pairs back
+// into TMEM in place of the chunk's S^T columns (c0 .. c0 + 15) and dS^T
+// into the 128-byte swizzled row `ds_row` of the chunk's 64-query block
+// (16-byte units u0 .. u0 + 3); the chunk's diagonal sums of ds into the
+// warp's area `diag` (entry 31 + e - lane for pair (lane, e); entry 63 is
+// scratch); the time gradient by bucket into the warp's slots. Rows see
+// buckets b0 .. b0 + nbk - 1 over the chunk, at most `most` for any row of
+// the warp. TM 0: one bucket per row (most == 1); TM 1: up to four (summed in
+// registers in the pair loop); TM 2: any (summed afterwards in passes over
+// windows of four buckets). Straight-line code over the pairs.
 template <int TM>
-__device__ __forceinline__ void bwd_chunk(const uint32_t (&sv)[32], const uint32_t (&pv)[32],
+__device__ __forceinline__ void bwd_chunk(uint32_t tS_c, uint32_t tP_c, uint8_t* ds_row, int u0,
                                           int c0, int r, int lo, int span, const float* s_posw,
                                           const long long* s_qts, const float* s_tb, long long tk,
-                                          int NB, float inv_n, bool has_time, int b0, int nbk,
-                                          float* diag, float* tslot, uint32_t (&pk_p)[16],
-                                          uint32_t (&pk_ds)[16]) {
+                                          int NB, bool has_time, int b0, int nbk, int most,
+                                          float* diag, float* tslot) {
     const int lane = threadIdx.x & 31;
     const float tb0 = has_time ? s_tb[b0] : 0.f;
     float dsum = 0.f;                       // running diagonal sum, passed one lane down
-    float t0 = 0.f, t1 = 0.f, t2 = 0.f, t3 = 0.f;   // TM 0 / 1: per bucket b0 + i
-    float run = 0.f;                        // TM 2: current bucket run
-    int run_b = -1;
-    float pe = 0.f, de = 0.f;
+    float t0 = 0.f, t1 = 0.f, t2 = 0.f, t3 = 0.f;   // TM 0 / 1: buckets b0 .. b0 + 3
 #pragma unroll
-    for (int e = 0; e < 32; ++e) {
-        const int c = c0 + e;
-        const bool keep = static_cast<unsigned>(c - lo) < static_cast<unsigned>(span);
-        float sc = __uint_as_float(sv[e]) + s_posw[c - r + 127];
-        int bk = b0;
-        if (TM == 0) {
-            sc += tb0;
-        } else {
-            bk = time_bucket_of(s_qts[c] - tk, NB);
-            sc += s_tb[bk];
+    for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t sv[16], pv[16], pk_p[8], pk_ds[8];
+        float dsv[TM == 2 ? 16 : 1];
+        tmem_ld16x2(tS_c + 16 * h2, tP_c + 16 * h2, sv, pv);
+        float pe = 0.f, de = 0.f;
+#pragma unroll
+        for (int e2 = 0; e2 < 16; ++e2) {
+            const int e = 16 * h2 + e2;
+            const int c = c0 + e;
+            const bool keep = static_cast<unsigned>(c - lo) < static_cast<unsigned>(span);
+            float sc = __uint_as_float(sv[e2]) + s_posw[c - r + 127];
+            int j = 0;
+            if (TM == 0) {
+                sc += tb0;
+            } else {
+                const int bk = time_bucket_of(s_qts[c] - tk, NB);
+                sc += s_tb[bk];
+                j = bk - b0;
+            }
+            const float sg = fmaf(0.5f, tanh_approx(0.5f * sc), 0.5f);
+            const float p = keep ? sc * sg : 0.f;
+            const float g = fmaf(sg * sc, 1.f - sg, sg);
+            const float ds = keep ? __uint_as_float(pv[e2]) * g : 0.f;
+            if (TM == 2) dsv[TM == 2 ? e2 : 0] = ds;
+            // the diagonal through (lane, e) continues from (lane - 1, e - 1);
+            // it leaves the chunk at lane 31 (entry e) or at column 31 (below)
+            const float up = __shfl_up_sync(0xffffffffu, dsum, 1);
+            dsum = (lane == 0 ? 0.f : up) + ds;
+            st_shared_if_lane31(diag + e, dsum, lane);
+            if (TM == 0) {
+                t0 += ds;
+            } else if (TM == 1) {
+                if (j == 0) t0 += ds;
+                if (j == 1) t1 += ds;
+                if (j == 2) t2 += ds;
+                if (j == 3) t3 += ds;
+            }
+            if (e2 & 1) {
+                pk_p[e2 >> 1] = pack_bf16x2(pe, p);
+                pk_ds[e2 >> 1] = pack_bf16x2(de, ds);
+            } else {
+                pe = p;
+                de = ds;
+            }
         }
-        const float sg = fmaf(0.5f, tanh_approx(0.5f * sc), 0.5f);
-        const float p = keep ? sc * sg * inv_n : 0.f;
-        const float g = fmaf(sg * sc, 1.f - sg, sg);
-        const float ds = keep ? __uint_as_float(pv[e]) * g * inv_n : 0.f;
-        // the diagonal through (lane, e) continues from (lane - 1, e - 1); it
-        // ends in this chunk at lane 31 (entry e) or at column 31 (below)
-        const float up = __shfl_up_sync(0xffffffffu, dsum, 1);
-        dsum = (lane == 0 ? 0.f : up) + ds;
-        if (lane == 31) diag[e] = dsum;
-        if (TM == 0) {
-            t0 += ds;
-        } else if (TM == 1) {
-            const int j = bk - b0;
-            t0 += j == 0 ? ds : 0.f;
-            t1 += j == 1 ? ds : 0.f;
-            t2 += j == 2 ? ds : 0.f;
-            t3 += j == 3 ? ds : 0.f;
-        } else {
-            const bool flush = bk != run_b && run_b >= 0;
-            if (__any_sync(0xffffffffu, flush)) warp_bucket_add(tslot, flush, run_b, run);
-            run = bk != run_b ? ds : run + ds;
-            run_b = bk;
-        }
-        if (e & 1) {
-            pk_p[e >> 1] = pack_bf16x2(pe, p);
-            pk_ds[e >> 1] = pack_bf16x2(de, ds);
-        } else {
-            pe = p;
-            de = ds;
+        // the half's P^T words over S^T columns this warp has already read
+        tmem_st8_async(tS_c + 8 * h2, pk_p);
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+            *reinterpret_cast<uint4*>(ds_row + (((u0 + 2 * h2 + j) ^ (r & 7)) << 4)) =
+                make_uint4(pk_ds[4 * j], pk_ds[4 * j + 1], pk_ds[4 * j + 2], pk_ds[4 * j + 3]);
+        if (TM == 2) {
+            // time gradient of the half: windows of four buckets from b0
+#pragma unroll 1
+            for (int wb = 0; wb < most; wb += 4) {
+                float t[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int e2 = 0; e2 < 16; ++e2) {
+                    const int j = time_bucket_of(s_qts[c0 + 16 * h2 + e2] - tk, NB) - b0 - wb;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) t[k] += j == k ? dsv[TM == 2 ? e2 : 0] : 0.f;
+                }
+#pragma unroll
+                for (int k = 0; k < 4; ++k) warp_bucket_add(tslot, wb + k < nbk, b0 + wb + k, t[k]);
+            }
         }
     }
-    if (lane < 31) diag[62 - lane] = dsum;
+    diag[lane < 31 ? 62 - lane : 63] = dsum;
+    __syncwarp();
     if (has_time) {
         if (TM == 0) {
             warp_bucket_add(tslot, true, b0, t0);
@@ -290,8 +331,6 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&sv)[32], const uint32
             warp_bucket_add(tslot, nbk > 1, b0 + 1, t1);
             warp_bucket_add(tslot, nbk > 2, b0 + 2, t2);
             warp_bucket_add(tslot, nbk > 3, b0 + 3, t3);
-        } else {
-            warp_bucket_add(tslot, run_b >= 0, run_b, run);
         }
     }
 }
@@ -348,8 +387,8 @@ attn_bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         mbar_init(&bars[kBwDrain], 1);
         mbar_fence_init();
     }
-    for (int i = tid; i < 8 * 128; i += blockDim.x) s_diag[i] = 0.f;
-    for (int i = tid; i < 8 * 64; i += blockDim.x) s_tslot[i] = 0.f;
+    for (int i = tid; i < 16 * 64; i += blockDim.x) s_diag[i] = 0.f;
+    for (int i = tid; i < 16 * 64; i += blockDim.x) s_tslot[i] = 0.f;
     if (warp == C::kWarpMMA) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
@@ -520,33 +559,42 @@ attn_bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         __syncwarp();
     } else {
         // ------------------------------------------------------------ pointwise stage
-        const int qd = warp & 3, hf = warp >> 2;            // TMEM lane quarter, column half
+        const int qd = warp & 3, cq = warp >> 2;            // TMEM lane quarter, column chunk
         const int r = qd * 32 + lane;                       // key row (S^T) / query row (dQ)
-        const int ptid = tid;                               // 0..255
+        const int ptid = tid;                               // 0..511
         const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
         const uint32_t tS = tmem + lane_base + C::kColS, tP = tmem + lane_base + C::kColP;
         const uint32_t tV = tmem + lane_base + C::kColV, tK = tmem + lane_base + C::kColK;
         uint8_t* ds_row = smem + L::kOffDS + r * 128;
-        // chunk cc's diagonal sums: entry i is tile diagonal (c - r + 127)
-        // hf*64 - 32 qd + 96 + 32 cc + i, i = 0 .. 62
-        float* my_diag = s_diag + warp * 128;
+        // the chunk's diagonal sums: entry i is tile diagonal (c - r + 127)
+        // 32 cq - 32 qd + 96 + i, i = 0 .. 62
+        float* my_diag = s_diag + warp * 64;
         float* my_tslot = s_tslot + warp * 64;
 
-        // bias data of a step into shared memory (every pointwise thread takes part)
-        auto stage = [&](const BwdStep& st) {
+        // bias data of a step: this thread's share is loaded into registers
+        // early (pre_*) and written into shared memory later (every pointwise
+        // thread takes part in both)
+        float pre_pos = 0.f, pre_tb = 0.f;
+        long long pre_ts = 0;
+        auto stage_load = [&](const BwdStep& st) {
             if (!st.valid) return;
-            if (ptid < 255) {
+            if (has_pos && ptid < 255) {
                 const int rel = st.q0 - st.kt0 - 127 + ptid;
-                s_posw[ptid] = has_pos ? __ldg(a.pos + static_cast<int64_t>(st.h) * a.P +
-                                               min(max(rel, 0), a.P - 1))
-                                       : 0.f;
+                pre_pos = __ldg(a.pos + static_cast<int64_t>(st.h) * a.P + min(max(rel, 0), a.P - 1));
             }
             if (has_time) {
-                if (ptid < 64) s_tb[ptid] = __ldg(a.tb + static_cast<int64_t>(st.h) * a.NB + min(ptid, a.NB - 1));
+                if (ptid < 64) pre_tb = __ldg(a.tb + static_cast<int64_t>(st.h) * a.NB + min(ptid, a.NB - 1));
+                if (ptid < 128) pre_ts = __ldg(a.ts + min(static_cast<int64_t>(st.q0) + ptid, a.T - 1));
+            }
+        };
+        auto stage_store = [&](const BwdStep& st) {
+            if (!st.valid) return;
+            if (ptid < 255) s_posw[ptid] = pre_pos;
+            if (has_time) {
+                if (ptid < 64) s_tb[ptid] = pre_tb;
                 if (ptid < 128) {
-                    const long long t = __ldg(a.ts + min(static_cast<int64_t>(st.q0) + ptid, a.T - 1));
-                    s_qts[ptid] = t;
-                    long long mn = t, mx = t;
+                    s_qts[ptid] = pre_ts;
+                    long long mn = pre_ts, mx = pre_ts;
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) {
                         mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
@@ -559,7 +607,7 @@ attn_bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 }
             }
         };
-        auto step_of = [&](int w, int s) -> BwdStep {
+        auto step_of = [&](int w, int s) -> BwdStep {   // first step of an item only
             BwdStep st{0, 0, 0, false};
             if (w >= n_items) return st;
             const BwdItem I = bwd_item(a, w);
@@ -570,13 +618,18 @@ attn_bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             st.valid = true;
             return st;
         };
-        stage(step_of(blockIdx.x, 0));
+        {
+            const BwdStep first = step_of(blockIdx.x, 0);
+            stage_load(first);
+            stage_store(first);
+        }
         mbar_arrive(&bars[kBwStaged]);
 
         int n = 0;
         bool ok = true;
         for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
             const BwdItem I = bwd_item(a, w);
+            const BwdStep next_item = step_of(w + gridDim.x, 0);
             const int ktok = I.kt0 + r;
             const bool kvalid = ktok < I.key_end;
             // end (exclusive) of the sequence of key row r
@@ -587,47 +640,36 @@ attn_bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 const int q0 = I.qt0 + s * kTile;
                 const int lo = ktok - q0;                    // first kept query column
                 const int span = kvalid ? max(kend - q0 - lo, 0) : 0;   // kept: lo <= c < lo + span
+                // the next step's bias data, loaded while this one is computed
+                const BwdStep next =
+                    s + 1 < I.nq ? BwdStep{q0 + kTile, I.kt0, I.h, true} : next_item;
+                stage_load(next);
                 if (!warp_wait(&bars[kBwStaged], n & 1, abort_flag) ||
                     !warp_wait(&bars[kBwSFull], n & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-#pragma unroll 1
-                for (int cc = 0; cc < 2; ++cc) {
-                    const int c0 = hf * 64 + cc * 32;
-                    uint32_t sv[32], pv[32];
-                    tmem_ld32(tS + c0, sv);
-                    tmem_ld32(tP + c0, pv);
+                {
+                    const int c0 = cq * 32;
                     // buckets each row sees over the chunk: b0 .. b0 + nbk - 1
                     int b0 = 0, nbk = 1;
                     if (has_time) {
-                        b0 = time_bucket_of(s_cmm[2 * (c0 >> 5)] - tk, a.NB);
-                        nbk = time_bucket_of(s_cmm[2 * (c0 >> 5) + 1] - tk, a.NB) - b0 + 1;
+                        b0 = time_bucket_of(s_cmm[2 * cq] - tk, a.NB);
+                        nbk = time_bucket_of(s_cmm[2 * cq + 1] - tk, a.NB) - b0 + 1;
                     }
                     const int most = __reduce_max_sync(0xffffffffu, static_cast<unsigned>(nbk));
-                    uint32_t pk_p[16], pk_ds[16];
-                    float* diag = my_diag + cc * 64;
-                    if (most == 1)
-                        bwd_chunk<0>(sv, pv, c0, r, lo, span, s_posw, s_qts, s_tb, tk, a.NB, a.inv_n,
-                                     has_time, b0, nbk, diag, my_tslot, pk_p, pk_ds);
-                    else if (most <= 4)
-                        bwd_chunk<1>(sv, pv, c0, r, lo, span, s_posw, s_qts, s_tb, tk, a.NB, a.inv_n,
-                                     has_time, b0, nbk, diag, my_tslot, pk_p, pk_ds);
-                    else
-                        bwd_chunk<2>(sv, pv, c0, r, lo, span, s_posw, s_qts, s_tb, tk, a.NB, a.inv_n,
-                                     has_time, b0, nbk, diag, my_tslot, pk_p, pk_ds);
-                    // P^T in place of the chunk's S^T columns (c0 .. c0 + 15)
-                    tmem_st16_async(tS + c0, pk_p);
-                    // dS^T row r, queries c0 .. c0 + 31: four 16-byte units of the
-                    // 128-byte swizzled row of block c0 / 64
-                    uint8_t* blk = ds_row + (c0 >> 6) * 16384;
+                    uint8_t* dsr = ds_row + (c0 >> 6) * 16384;
                     const int u0 = (c0 & 63) >> 3;
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        *reinterpret_cast<uint4*>(blk + (((u0 + j) ^ (r & 7)) << 4)) =
-                            make_uint4(pk_ds[4 * j], pk_ds[4 * j + 1], pk_ds[4 * j + 2],
-                                       pk_ds[4 * j + 3]);
+                    if (most == 1)
+                        bwd_chunk<0>(tS + c0, tP + c0, dsr, u0, c0, r, lo, span, s_posw, s_qts, s_tb,
+                                     tk, a.NB, has_time, b0, nbk, most, my_diag, my_tslot);
+                    else if (most <= 4)
+                        bwd_chunk<1>(tS + c0, tP + c0, dsr, u0, c0, r, lo, span, s_posw, s_qts, s_tb,
+                                     tk, a.NB, has_time, b0, nbk, most, my_diag, my_tslot);
+                    else
+                        bwd_chunk<2>(tS + c0, tP + c0, dsr, u0, c0, r, lo, span, s_posw, s_qts, s_tb,
+                                     tk, a.NB, has_time, b0, nbk, most, my_diag, my_tslot);
                 }
                 tmem_wait_st();
                 tc_fence_before();
@@ -643,28 +685,27 @@ attn_bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 if (has_pos && ptid < 255) {
                     float v = 0.f;
 #pragma unroll
-                    for (int ww = 0; ww < 8; ++ww) {
-#pragma unroll
-                        for (int cc = 0; cc < 2; ++cc) {
-                            const int i = ptid - ((ww >> 2) * 64 - (ww & 3) * 32 + 96 + 32 * cc);
-                            if (i >= 0 && i <= 62) v += s_diag[ww * 128 + cc * 64 + i];
-                        }
+                    for (int ww = 0; ww < 16; ++ww) {
+                        const int i = ptid - ((ww >> 2) * 32 - (ww & 3) * 32 + 96);
+                        if (i >= 0 && i <= 62) v += s_diag[ww * 64 + i];
                     }
                     if (v != 0.f) {
                         const int rel = q0 - I.kt0 + ptid - 127;
-                        atomicAdd(a.dpos + static_cast<int64_t>(I.h) * a.P + min(max(rel, 0), a.P - 1), v);
+                        atomicAdd(a.dpos + static_cast<int64_t>(I.h) * a.P + min(max(rel, 0), a.P - 1),
+                                  v * a.inv_n);
                     }
                 }
                 if (has_time && ptid < 64) {
                     float v = 0.f;
 #pragma unroll
-                    for (int ww = 0; ww < 8; ++ww) {
+                    for (int ww = 0; ww < 16; ++ww) {
                         v += s_tslot[ww * 64 + ptid];
                         s_tslot[ww * 64 + ptid] = 0.f;
                     }
-                    if (v != 0.f && ptid < a.NB) atomicAdd(a.dtime + static_cast<int64_t>(I.h) * a.NB + ptid, v);
+                    if (v != 0.f && ptid < a.NB)
+                        atomicAdd(a.dtime + static_cast<int64_t>(I.h) * a.NB + ptid, v * a.inv_n);
                 }
-                stage(s + 1 < I.nq ? step_of(w, s + 1) : step_of(w + gridDim.x, 0));
+                stage_store(next);
                 mbar_arrive(&bars[kBwStaged]);
                 // dQ_i of the step into dq
                 if (!warp_wait(&bars[kBwDQFull], n & 1, abort_flag)) {
@@ -674,26 +715,30 @@ attn_bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 tc_fence_after();
                 {
                     // dQ_i rows through the dS^T buffer (its MMAs have completed):
-                    // each warp stages 32 x 32 fp32 blocks (128-byte swizzle) and
-                    // adds them into dq with a bulk tensor reduction; rows of
-                    // queries outside the sequence are zero (every ds of theirs is)
-                    uint8_t* buf = smem + L::kOffDS + warp * 4096;
+                    // each warp stages 32 x 16 fp32 blocks (64-byte swizzle) of its
+                    // D/4 columns and adds them into dq with a bulk tensor
+                    // reduction; rows of queries outside the sequence are zero
+                    // (every ds of theirs is)
+                    uint8_t* buf = smem + L::kOffDS + warp * 2048;
 #pragma unroll 1
                     for (int cb = 0; cb < D / 64; ++cb) {
-                        uint32_t v[32];
-                        tmem_ld32(tP + hf * (D / 2) + cb * 32, v);
+                        uint32_t v[16];
+                        tmem_ld16(tP + cq * (D / 4) + cb * 16, v);
                         if (cb > 0) {
                             if (lane == 0) bulk_wait_group_read<0>();
                             __syncwarp();
                         }
 #pragma unroll
-                        for (int u = 0; u < 8; ++u)
-                            *reinterpret_cast<uint4*>(buf + lane * 128 + ((u ^ (lane & 7)) << 4)) =
-                                make_uint4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+                        for (int u = 0; u < 4; ++u)
+                            *reinterpret_cast<float4*>(buf + lane * 64 + ((u ^ ((lane >> 1) & 3)) << 4)) =
+                                make_float4(__uint_as_float(v[4 * u]) * a.inv_n,
+                                            __uint_as_float(v[4 * u + 1]) * a.inv_n,
+                                            __uint_as_float(v[4 * u + 2]) * a.inv_n,
+                                            __uint_as_float(v[4 * u + 3]) * a.inv_n);
                         fence_proxy_async_smem();
                         __syncwarp();
                         if (lane == 0) {
-                            tma_reduce_add_2d(&tmDQ, buf, I.h * D + hf * (D / 2) + cb * 32, q0 + qd * 32);
+                            tma_reduce_add_2d(&tmDQ, buf, I.h * D + cq * (D / 4) + cb * 16, q0 + qd * 32);
                             bulk_commit_group();
                         }
                     }
@@ -704,25 +749,29 @@ attn_bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 mbar_arrive(&bars[kBwDQFree]);
                 if (s == I.nq - 1) {
                     // the item's dV_j and dK_j (their MMAs completed before dQ's)
-                    const int64_t row = (static_cast<int64_t>(ktok) * a.H + I.h) * D + hf * (D / 2);
+                    const int64_t row = (static_cast<int64_t>(ktok) * a.H + I.h) * D + cq * (D / 4);
 #pragma unroll 1
                     for (int cb = 0; cb < D / 64; ++cb) {
-                        uint32_t v[32];
-                        tmem_ld32(tV + hf * (D / 2) + cb * 32, v);
+                        uint32_t v[16];
+                        tmem_ld16(tV + cq * (D / 4) + cb * 16, v);
                         if (kvalid) {
 #pragma unroll
-                            for (int j = 0; j < 8; ++j)
-                                *reinterpret_cast<float4*>(a.dv + row + cb * 32 + 4 * j) =
-                                    make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                                                __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+                            for (int j = 0; j < 4; ++j)
+                                *reinterpret_cast<float4*>(a.dv + row + cb * 16 + 4 * j) =
+                                    make_float4(__uint_as_float(v[4 * j]) * a.inv_n,
+                                                __uint_as_float(v[4 * j + 1]) * a.inv_n,
+                                                __uint_as_float(v[4 * j + 2]) * a.inv_n,
+                                                __uint_as_float(v[4 * j + 3]) * a.inv_n);
                         }
-                        tmem_ld32(tK + hf * (D / 2) + cb * 32, v);
+                        tmem_ld16(tK + cq * (D / 4) + cb * 16, v);
                         if (kvalid) {
 #pragma unroll
-                            for (int j = 0; j < 8; ++j)
-                                *reinterpret_cast<float4*>(a.dk + row + cb * 32 + 4 * j) =
-                                    make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                                                __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+                            for (int j = 0; j < 4; ++j)
+                                *reinterpret_cast<float4*>(a.dk + row + cb * 16 + 4 * j) =
+                                    make_float4(__uint_as_float(v[4 * j]) * a.inv_n,
+                                                __uint_as_float(v[4 * j + 1]) * a.inv_n,
+                                                __uint_as_float(v[4 * j + 2]) * a.inv_n,
+                                                __uint_as_float(v[4 * j + 3]) * a.inv_n);
                         }
                     }
                     tc_fence_before();

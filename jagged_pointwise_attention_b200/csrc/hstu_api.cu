@@ -67,18 +67,18 @@ bool make_tmap_bf16_box(CUtensorMap* tm, const void* base, uint64_t inner, uint6
     return r == CUDA_SUCCESS;
 }
 
-// fp32 [rows, inner] with boxes of 32 x 32 (128-byte rows, 128-byte swizzle).
-bool make_tmap_f32_32(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t rows,
-                      uint64_t row_stride_bytes) {
+// fp32 [rows, inner] with boxes of 16 x 32 (64-byte rows, 64-byte swizzle).
+bool make_tmap_f32_16x32(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t rows,
+                         uint64_t row_stride_bytes) {
     auto fn = encode_fn();
     if (fn == nullptr) return false;
     cuuint64_t dims[2] = {inner, rows};
     cuuint64_t strides[1] = {row_stride_bytes};
-    cuuint32_t box[2] = {32, 32};
+    cuuint32_t box[2] = {16, 32};
     cuuint32_t estr[2] = {1, 1};
     const CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims,
                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -786,7 +786,7 @@ hstu_status_t hstu_attn_bwd(hstu_dtype_t dtype, const void* q, int64_t q_stride,
         !make_tmap_bf16(&tk, k, row, T, k_stride * 2, 128) ||
         !make_tmap_bf16(&tv, v, row, T, v_stride * 2, 128) ||
         !make_tmap_bf16(&tdo, dout, row, T, dout_stride * 2, 128) ||
-        !make_tmap_f32_32(&tdq, dq, row, T, row * 4))
+        !make_tmap_f32_16x32(&tdq, dq, row, T, row * 4))
         return HSTU_ERR_CUDA;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     BwdArgs a{reinterpret_cast<const int4*>(ws + kAttnWsHeader), reinterpret_cast<const int*>(ws),
