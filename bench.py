@@ -289,6 +289,11 @@ def bench_attention(args, rank, world, local, peaks, peak_kind, cfg_id=None, cpu
     cfg = CONFIGS[cfg_id]
     seed = 1000 + cfg_id + 7919 * rank
     inp = make_attn_inputs(cfg_id, seed=seed)
+    if args.sample_seqs:
+        # a smaller case of the same kernel (the workload's first sequences):
+        # for profiler captures, not for bench lines
+        from gen import take_sequences
+        inp = take_sequences(inp, list(range(min(args.sample_seqs, inp.B))))
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
     bf = torch.bfloat16 if inp.dtype == "bf16" else torch.float32
@@ -434,7 +439,8 @@ def bench_attention(args, rank, world, local, peaks, peak_kind, cfg_id=None, cpu
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": inp.dtype,
         "data": "synthetic (seeded generator; no dataset)",
         "config": workload_config(cfg_id, inp.B, inp.T, inp.max_seqlen, seed, world,
-                                  {"H": H, "d": d, "l2": l2_note(in_bytes, ncopies)}),
+                                  {"H": H, "d": d, "l2": l2_note(in_bytes, ncopies),
+                                   **({"first_sequences_only": inp.B} if args.sample_seqs else {})}),
         "launch": "eager" if args.no_graph else "one CUDA graph of the K steps (plan + run each)",
         "pct_of_bf16_peak": {"measured_burst": round(100 * value / peaks["bf16_tflops"], 2),
                              "nominal_2250": round(100 * value / NOMINAL_BF16_TFLOPS, 2)},
@@ -746,6 +752,11 @@ def bench_backward(args, rank, world, local, peaks, peak_kind, cfg_id=None):
         raise SystemExit("--backward takes an attention workload (--config 2, 3 or 4)")
     seed = 1000 + cfg_id + 7919 * rank
     inp = make_attn_inputs(cfg_id, seed=seed)
+    if args.sample_seqs:
+        # a smaller case of the same kernel (the workload's first sequences):
+        # for profiler captures, not for bench lines
+        from gen import take_sequences
+        inp = take_sequences(inp, list(range(min(args.sample_seqs, inp.B))))
     dev = torch.device("cuda", local)
     bf = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(dev).to(torch.bfloat16)  # noqa: E731
     f32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(dev)  # noqa: E731
@@ -795,7 +806,8 @@ def bench_backward(args, rank, world, local, peaks, peak_kind, cfg_id=None):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16 inputs, fp32 gradients",
             "data": "synthetic (seeded generator; no dataset)",
-            "config": {"workload": cfg["name"] + "_backward", "B": inp.B, "H": H, "d": d,
+            "config": {"workload": cfg["name"] + "_backward" + (
+                           "_first%d" % inp.B if args.sample_seqs else ""), "B": inp.B, "H": H, "d": d,
                        "total_tokens": T, "seed": seed, "parallelism": "dp%d" % world,
                        "l2": "q, k, v, dout %.0f MB, dq/dk/dv %.0f MB: %s" % (
                            in_mb, 3 * T * H * d * 4 / 2 ** 20,
@@ -974,6 +986,9 @@ def parse_args(argv=None):
     ap.add_argument("--backward", action="store_true",
                     help="time the tensor-core attention backward (hstu_attn_bwd) on the "
                          "--config workload instead of the forward")
+    ap.add_argument("--sample-seqs", type=int, default=0,
+                    help="only the workload's first N sequences (a smaller case of the same "
+                         "kernels, for profiler captures)")
     ap.add_argument("--fp8-linear", action="store_true",
                     help="time the row-wise E4M3 projections (quantize + FP8 GEMM) against the "
                          "bf16 ones on the projection shapes instead of the attention")

@@ -15,4 +15,5 @@ from .hstu_inputs import (  # noqa: F401
     make_inputs,
     round_to_bf16,
     custom_attn_inputs,
+    take_sequences,
 )
