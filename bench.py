@@ -835,6 +835,10 @@ def bench_fp8_linear(args, rank, world, local, peaks, peak_kind):
     fp8_peak = 2 * peaks["bf16_tflops"]
     shapes = [("f1_layer_T79913_K512_N2048_silu", 79913, 512, 2048, "silu"),
               ("addmm_bench_m4096_k512_n512", 4096, 512, 512, "none")]
+    if args.sample_rows:
+        # a smaller case of the same kernels (for profiler captures)
+        shapes = [("f1_rows%d_K512_N2048_silu" % args.sample_rows, args.sample_rows, 512, 2048,
+                   "silu")]
     out = []
 
     def timed(fn):
@@ -989,6 +993,9 @@ def parse_args(argv=None):
     ap.add_argument("--sample-seqs", type=int, default=0,
                     help="only the workload's first N sequences (a smaller case of the same "
                          "kernels, for profiler captures)")
+    ap.add_argument("--sample-rows", type=int, default=0,
+                    help="with --fp8-linear: only the f1 shape, with this many rows (a smaller "
+                         "case of the same kernels, for profiler captures)")
     ap.add_argument("--fp8-linear", action="store_true",
                     help="time the row-wise E4M3 projections (quantize + FP8 GEMM) against the "
                          "bf16 ones on the projection shapes instead of the attention")
