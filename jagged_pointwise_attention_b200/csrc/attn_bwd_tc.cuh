@@ -222,6 +222,12 @@ __device__ __forceinline__ void warp_bucket_add(float* slots, bool has, int b, f
     __syncwarp();
 }
 
+// warp_bucket_add as a call, for the rare per-pair flushes of TM 2 (keeps the
+// unrolled pair loop small).
+__device__ __noinline__ void warp_bucket_add_call(float* slots, bool has, int b, float v) {
+    warp_bucket_add(slots, has, b, v);
+}
+
 // Shared-memory store by lane 31 only, as a predicated instruction (no branch
 // in the straight-line pair loop).
 __device__ __forceinline__ void st_shared_if_lane31(float* p, float v, int lane) {
@@ -241,8 +247,10 @@ __device__ __forceinline__ void st_shared_if_lane31(float* p, float v, int lane)
 // scratch); the time gradient by bucket into the warp's slots. Rows see
 // buckets b0 .. b0 + nbk - 1 over the chunk, at most `most` for any row of
 // the warp. TM 0: one bucket per row (most == 1); TM 1: up to four (summed in
-// registers in the pair loop); TM 2: any (summed afterwards in passes over
-// windows of four buckets). Straight-line code over the pairs.
+// registers in the pair loop); TM 2: any, as runs of one bucket per row over
+// the kept pairs (the bucket is monotone in the query timestamp, so a row
+// sees few runs), each run added into the warp's slots when any lane's run
+// ends. Straight-line code over the pairs for TM 0 and 1.
 template <int TM>
 __device__ __forceinline__ void bwd_chunk(uint32_t tS_c, uint32_t tP_c, uint8_t* ds_row, int u0,
                                           int c0, int r, int lo, int span, const float* s_posw,
@@ -253,10 +261,11 @@ __device__ __forceinline__ void bwd_chunk(uint32_t tS_c, uint32_t tP_c, uint8_t*
     const float tb0 = has_time ? s_tb[b0] : 0.f;
     float dsum = 0.f;                       // running diagonal sum, passed one lane down
     float t0 = 0.f, t1 = 0.f, t2 = 0.f, t3 = 0.f;   // TM 0 / 1: buckets b0 .. b0 + 3
+    float run = 0.f;                        // TM 2: the row's current bucket run
+    int run_b = -1;
 #pragma unroll
     for (int h2 = 0; h2 < 2; ++h2) {
         uint32_t sv[16], pv[16], pk_p[8], pk_ds[8];
-        float dsv[TM == 2 ? 16 : 1];
         tmem_ld16x2(tS_c + 16 * h2, tP_c + 16 * h2, sv, pv);
         float pe = 0.f, de = 0.f;
 #pragma unroll
@@ -277,7 +286,6 @@ __device__ __forceinline__ void bwd_chunk(uint32_t tS_c, uint32_t tP_c, uint8_t*
             const float p = keep ? sc * sg : 0.f;
             const float g = fmaf(sg * sc, 1.f - sg, sg);
             const float ds = keep ? __uint_as_float(pv[e2]) * g : 0.f;
-            if (TM == 2) dsv[TM == 2 ? e2 : 0] = ds;
             // the diagonal through (lane, e) continues from (lane - 1, e - 1);
             // it leaves the chunk at lane 31 (entry e) or at column 31 (below)
             const float up = __shfl_up_sync(0xffffffffu, dsum, 1);
@@ -290,6 +298,13 @@ __device__ __forceinline__ void bwd_chunk(uint32_t tS_c, uint32_t tP_c, uint8_t*
                 if (j == 1) t1 += ds;
                 if (j == 2) t2 += ds;
                 if (j == 3) t3 += ds;
+            } else {
+                const int bk = j + b0;
+                const bool ends = keep && bk != run_b && run_b >= 0;
+                if (__any_sync(0xffffffffu, ends)) warp_bucket_add_call(tslot, ends, run_b, run);
+                const bool starts = keep && bk != run_b;
+                run = starts ? ds : run + ds;
+                run_b = starts ? bk : run_b;
             }
             if (e2 & 1) {
                 pk_p[e2 >> 1] = pack_bf16x2(pe, p);
@@ -305,21 +320,6 @@ __device__ __forceinline__ void bwd_chunk(uint32_t tS_c, uint32_t tP_c, uint8_t*
         for (int j = 0; j < 2; ++j)
             *reinterpret_cast<uint4*>(ds_row + (((u0 + 2 * h2 + j) ^ (r & 7)) << 4)) =
                 make_uint4(pk_ds[4 * j], pk_ds[4 * j + 1], pk_ds[4 * j + 2], pk_ds[4 * j + 3]);
-        if (TM == 2) {
-            // time gradient of the half: windows of four buckets from b0
-#pragma unroll 1
-            for (int wb = 0; wb < most; wb += 4) {
-                float t[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int e2 = 0; e2 < 16; ++e2) {
-                    const int j = time_bucket_of(s_qts[c0 + 16 * h2 + e2] - tk, NB) - b0 - wb;
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) t[k] += j == k ? dsv[TM == 2 ? e2 : 0] : 0.f;
-                }
-#pragma unroll
-                for (int k = 0; k < 4; ++k) warp_bucket_add(tslot, wb + k < nbk, b0 + wb + k, t[k]);
-            }
-        }
     }
     diag[lane < 31 ? 62 - lane : 63] = dsum;
     __syncwarp();
@@ -331,6 +331,8 @@ __device__ __forceinline__ void bwd_chunk(uint32_t tS_c, uint32_t tP_c, uint8_t*
             warp_bucket_add(tslot, nbk > 1, b0 + 1, t1);
             warp_bucket_add(tslot, nbk > 2, b0 + 2, t2);
             warp_bucket_add(tslot, nbk > 3, b0 + 3, t3);
+        } else {
+            warp_bucket_add(tslot, run_b >= 0, run_b, run);
         }
     }
 }
