@@ -429,7 +429,7 @@ def bench_attention(args, rank, world, local, peaks, peak_kind, cfg_id=None, cpu
         v, nrows, secs, thr = oracle_sample_rate(
             inp, args.cpu_budget_s if cpu_budget_s is None else cpu_budget_s)
         cpu = {"value": round(v, 6), "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
-               "sample": "%d random query rows (all heads) of the same batch, fp64, %.1f s"
+               "sample": "%d random query rows (all heads) of the same batch, fp64, %.3f s"
                          % (nrows, secs)}
 
     clocks = sampler.summary()
@@ -644,7 +644,7 @@ def bench_layer(args, rank, world, local, peaks, peak_kind, cfg_id=None, cpu_bud
             li, args.cpu_budget_s if cpu_budget_s is None else cpu_budget_s)
         cpu = {"value": round(v, 6), "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
                "sample": "%d random whole sequences (%d tokens) of the same batch, the whole "
-                         "layer in fp64, %.1f s" % (nseq, ntok, secs)}
+                         "layer in fp64, %.3f s" % (nseq, ntok, secs)}
     return {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(max_ms / args.steps, 4),

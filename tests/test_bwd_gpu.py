@@ -126,6 +126,14 @@ def test_tc_bwd_long_sequences_many_steps():
     _check_tc(inp, dout, "long")
 
 
+def test_tc_bwd_sequence_over_2k_tokens():
+    """A ragged batch with a 2100-token sequence (17 key tiles walking up to
+    17 query tiles each) against the oracle, d = 128, bias tables that clip
+    and clamp."""
+    inp, dout = _bf16_inputs([2100, 300, 1], H=1, d=128, num_pos=1500, num_buckets=40, seed=14)
+    _check_tc(inp, dout, "2100 tokens")
+
+
 def test_tc_bwd_packed_short_sequences():
     """Batches of short sequences share tiles: pairs across a sequence
     boundary inside a tile must contribute nothing."""
