@@ -24,19 +24,22 @@
 //     dV_j += P^T dO_i      TS   (A from TMEM, dO_i MN-major) -> TMEM [256, 256 + D)
 //     dK_j += dS^T Q_i      SS   (dS^T K-major, Q_i MN-major)  -> TMEM [256 + D, 256 + 2D)
 //     dQ_i  = dS K_j        SS   (dS^T read MN-major, K_j MN-major) -> TMEM [128, 128 + D)
-// and the pointwise warps add dQ_i into the fp32 dq with bulk tensor
-// reductions (staged through the dS^T buffer, free once dQ_i is computed);
-// after the item's last step they store dK_j and dV_j (fp32).
+// and the pointwise warps read dQ_i out of TMEM (which frees its columns for
+// the next dP^T) and add it into the fp32 dq with bulk tensor reductions,
+// staged through the dS^T buffer (free once dQ_i is computed; the next step's
+// dS^T stores wait until those stages have been read); after the item's last
+// step they store dK_j and dV_j (fp32).
 //
 // Warp roles: 0-15 pointwise (four warps per TMEM lane quarter, one 32-column
 // chunk of queries each: with four warps per scheduler one warp's TMEM, SFU
 // and shared-memory latencies hide behind the others' arithmetic), 16 TMA
-// producer, 17 MMA issuer and TMEM owner.
+// producer, 17 MMA issuer and TMEM owner, 18 table warp (bias staging and
+// table-gradient flushes, off the pointwise warps' path).
 //
 // Pointwise arithmetic per pair in fp32: s = S + pos + time; one tanh gives
 // sg = 1/2 + tanh(s/2)/2, then p and ds without the factor 1/N, which is
-// applied once to every gradient as it leaves the kernel. Before each step the pointwise warps
-// stage the step's bias data in shared memory: the 255 position-table values
+// applied once to every gradient as it leaves the kernel. Two steps ahead the table warp
+// stages a step's bias data in shared memory: the 255 position-table values
 // the tile's diagonals read, the 128 query timestamps with each 32-column
 // chunk's smallest and largest, and the head's time-table row. The time
 // bucket is floor(log2(max(1, dt))) clamped to NB - 1 from a count of leading
@@ -49,9 +52,11 @@
 // (l - 1, e - 1)), so each diagonal's sum leaves through lane 31 or stays in
 // the last column's lanes, into the warp's own diagonal buffer; the time
 // gradient sums ds per row over runs of one bucket and adds the runs into the
-// warp's own bucket slots, merging lanes with equal buckets first. After each
-// step the buffers of the eight warps are summed per tile diagonal and per
-// bucket and added to the global tables with atomics.
+// warp's own bucket slots, merging lanes with equal buckets first. Once every
+// pointwise warp is done with a step, the table warp sums the sixteen warps'
+// buffers per tile diagonal and per bucket and adds them to the global tables
+// with atomics. Bias data and sums have two buffers, by step parity, so the
+// table warp works on step m (and stages step m + 2) while step m + 1 runs.
 //
 // Every wait is bounded; a wait that runs out raises kErrTimeout, the other
 // roles notice through a shared abort flag, and the CTA drains its own copies
@@ -91,7 +96,9 @@ struct BwdCfg {
     static constexpr int kPointwiseWarps = 16;
     static constexpr int kPointwiseThreads = 32 * kPointwiseWarps;
     static constexpr int kWarpTMA = kPointwiseWarps, kWarpMMA = kPointwiseWarps + 1;
-    static constexpr int kThreads = 32 * (kPointwiseWarps + 2);
+    static constexpr int kWarpTable = kPointwiseWarps + 2;
+    // 19 warps: at most five per scheduler, the same 96-register cap as 18
+    static constexpr int kThreads = 32 * (kPointwiseWarps + 3);
     static constexpr uint32_t kColS = 0, kColP = 128, kColV = 256, kColK = 256 + D;
 };
 
@@ -104,14 +111,15 @@ struct BwdSmem {
     static constexpr int kOffQ = kOffV + C::kTileBytes;            // [2 stages]
     static constexpr int kOffDO = kOffQ + 2 * C::kTileBytes;       // [kDOStages]
     static constexpr int kOffDS = kOffDO + kDOStages * C::kTileBytes;  // dS^T: 2 blocks of 64 queries
-    static constexpr int kOffPosW = kOffDS + 2 * 16384;            // 256 floats: pos of the tile diagonals
-    static constexpr int kOffQts = kOffPosW + 1024;                // 128 query timestamps
-    static constexpr int kOffCmm = kOffQts + 1024;                 // per chunk: min, max timestamp
-    static constexpr int kOffTb = kOffCmm + 64;                    // 64 floats: the head's time table
-    static constexpr int kOffDiag = kOffTb + 256;                  // [16 warps][64] diagonal sums
-    static constexpr int kOffTslot = kOffDiag + 16 * 64 * 4;       // [16 warps][64] bucket sums
-    static constexpr int kOffBar = kOffTslot + 16 * 64 * 4;
-    static constexpr int kNumBars = 18;
+    // a step's bias data and table sums, two buffers by step parity
+    static constexpr int kOffPosW = kOffDS + 2 * 16384;            // [2][256] floats: pos of the tile diagonals
+    static constexpr int kOffQts = kOffPosW + 2 * 1024;            // [2][128] query timestamps
+    static constexpr int kOffCmm = kOffQts + 2 * 1024;             // [2][4 chunks]: min, max timestamp
+    static constexpr int kOffTb = kOffCmm + 2 * 64;                // [2][64] floats: the head's time table
+    static constexpr int kOffDiag = kOffTb + 2 * 256;              // [2][16 warps][64] diagonal sums
+    static constexpr int kOffTslot = kOffDiag + 2 * 16 * 64 * 4;   // [2][16 warps][64] bucket sums
+    static constexpr int kOffBar = kOffTslot + 2 * 16 * 64 * 4;
+    static constexpr int kNumBars = 21;
     static constexpr int kOffTmem = kOffBar + kNumBars * 8;
     static constexpr int kOffAbort = kOffTmem + 8;
     static constexpr int kBytes = kOffAbort + 8;
@@ -127,13 +135,14 @@ enum {
     kBwDOFull = 6,      // +stage: dO_i landed
     kBwDOFree = 8,      // +stage: MMA commit after dV_i (the last MMA that reads dO_i)
     kBwSFull = 10,      // MMA commit: S^T and dP^T of the step are in TMEM
-    kBwPFull = 11,      // the 256 pointwise threads: P^T in TMEM, dS^T in shared memory
+    kBwPFull = 11,      // the pointwise threads: P^T in TMEM, dS^T in shared memory
     kBwDQFull = 12,     // MMA commit after dQ (dV and dK before it have completed too)
-    kBwDQFree = 13,     // the 256 pointwise threads have read dQ out of TMEM
-    kBwAccFree = 14,    // the 256 pointwise threads have read dK_j and dV_j out of TMEM
-    kBwPwDone = 15,     // the 256 pointwise threads are done with the step's staged data
-    kBwStaged = 16,     // phase n: step n's bias data staged, step n-1's table sums flushed
-    kBwDrain = 17,      // the MMA issuer's last commit
+    kBwDQFree = 13,     // the pointwise threads have read dQ out of TMEM
+    kBwAccFree = 14,    // the pointwise threads have read dK_j and dV_j out of TMEM
+    kBwDSFree = 15,     // the pointwise threads' dQ staging in the dS^T buffer has been read
+    kBwPwDone = 16,     // +parity of the step: the pointwise threads' table sums are complete
+    kBwReady = 18,      // +parity of the step: the table warp staged its bias data, cleared its sums
+    kBwDrain = 20,      // the MMA issuer's last commit
 };
 
 // A work item of the backward: key tile [kt0, key_end) of head h; its query
@@ -250,14 +259,19 @@ __device__ __forceinline__ void st_shared_if_lane31(float* p, float v, int lane)
 // registers in the pair loop); TM 2: any, as runs of one bucket per row over
 // the kept pairs (the bucket is monotone in the query timestamp, so a row
 // sees few runs), each run added into the warp's slots when any lane's run
-// ends. Straight-line code over the pairs for TM 0 and 1.
+// ends. Straight-line code over the pairs for TM 0 and 1. Before its first
+// dS^T store the warp waits for phase `ds_parity` of `ds_free` (the previous
+// step's dQ staging in the same buffer has been read), unless ds_parity < 0;
+// returns false if that wait gave up.
 template <int TM>
-__device__ __forceinline__ void bwd_chunk(uint32_t tS_c, uint32_t tP_c, uint8_t* ds_row, int u0,
+__device__ __forceinline__ bool bwd_chunk(uint32_t tS_c, uint32_t tP_c, uint8_t* ds_row, int u0,
                                           int c0, int r, int lo, int span, const float* s_posw,
                                           const long long* s_qts, const float* s_tb, long long tk,
                                           int NB, bool has_time, int b0, int nbk, int most,
-                                          float* diag, float* tslot) {
+                                          float* diag, float* tslot, uint64_t* ds_free,
+                                          int ds_parity, volatile int* abort_flag) {
     const int lane = threadIdx.x & 31;
+    bool ok = true;
     const float tb0 = has_time ? s_tb[b0] : 0.f;
     float dsum = 0.f;                       // running diagonal sum, passed one lane down
     float t0 = 0.f, t1 = 0.f, t2 = 0.f, t3 = 0.f;   // TM 0 / 1: buckets b0 .. b0 + 3
@@ -316,6 +330,8 @@ __device__ __forceinline__ void bwd_chunk(uint32_t tS_c, uint32_t tP_c, uint8_t*
         }
         // the half's P^T words over S^T columns this warp has already read
         tmem_st8_async(tS_c + 8 * h2, pk_p);
+        if (h2 == 0 && ds_parity >= 0)
+            ok = warp_wait(ds_free, static_cast<uint32_t>(ds_parity), abort_flag);
 #pragma unroll
         for (int j = 0; j < 2; ++j)
             *reinterpret_cast<uint4*>(ds_row + (((u0 + 2 * h2 + j) ^ (r & 7)) << 4)) =
@@ -335,14 +351,129 @@ __device__ __forceinline__ void bwd_chunk(uint32_t tS_c, uint32_t tP_c, uint8_t*
             warp_bucket_add(tslot, run_b >= 0, run_b, run);
         }
     }
+    return ok;
 }
 
-// The step a pointwise thread stages bias data for: query tile q0 of key
-// tile kt0, head h.
+// A step of the backward: query tile q0 of key tile kt0, head h.
 struct BwdStep {
     int q0, kt0, h;
     bool valid;
 };
+
+// Walks a CTA's steps in order: its items w = blockIdx.x, + gridDim.x, ...,
+// each over its query tiles.
+struct BwdCursor {
+    int w, s;
+    BwdItem I;
+    bool valid;
+    __device__ __forceinline__ void start(const BwdArgs& a, int w0, int n_items) {
+        w = w0;
+        s = 0;
+        valid = w < n_items;
+        if (valid) I = bwd_item(a, w);
+    }
+    __device__ __forceinline__ void next(const BwdArgs& a, int n_items) {
+        if (!valid) return;
+        if (++s < I.nq) return;
+        start(a, w + gridDim.x, n_items);
+    }
+    __device__ __forceinline__ BwdStep step() const {
+        return BwdStep{valid ? I.qt0 + s * kTile : 0, valid ? I.kt0 : 0, valid ? I.h : 0, valid};
+    }
+};
+
+// Bias data of step st into one buffer, by one warp: the position table at
+// the tile's 255 diagonals (zero without the position term), the 128 query
+// timestamps with each 32-query chunk's smallest and largest, and the head's
+// time-table row.
+__device__ __forceinline__ void bwd_stage_tables(const BwdArgs& a, const BwdStep& st, float* posw,
+                                                 long long* qts, long long* cmm, float* tbrow,
+                                                 bool has_pos, bool has_time) {
+    if (!st.valid) return;
+    const int lane = threadIdx.x & 31;
+    float pv[8], tv[2];
+    long long tsv[4];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const int i = lane + 32 * k;
+        const int rel = st.q0 - st.kt0 - 127 + i;
+        pv[k] = (has_pos && i < 255)
+                    ? __ldg(a.pos + static_cast<int64_t>(st.h) * a.P + min(max(rel, 0), a.P - 1))
+                    : 0.f;
+    }
+    if (has_time) {
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+            tv[k] = __ldg(a.tb + static_cast<int64_t>(st.h) * a.NB + min(lane + 32 * k, a.NB - 1));
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            tsv[k] = __ldg(a.ts + min(static_cast<int64_t>(st.q0) + lane + 32 * k, a.T - 1));
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+        if (lane + 32 * k < 255) posw[lane + 32 * k] = pv[k];
+    if (has_time) {
+#pragma unroll
+        for (int k = 0; k < 2; ++k) tbrow[lane + 32 * k] = tv[k];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            qts[lane + 32 * k] = tsv[k];
+            long long mn = tsv[k], mx = tsv[k];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+                mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            }
+            if (lane == 0) {
+                cmm[2 * k] = mn;
+                cmm[2 * k + 1] = mx;
+            }
+        }
+    }
+}
+
+// Step st's table sums from one buffer into the global tables, by one warp:
+// each tile diagonal (c - r + 127) collects the diagonal sums of the warps
+// whose 32 x 32 chunk it crosses (warp 4 cq + qd holds diagonal
+// 32 cq - 32 qd + 96 + i at entry i, i = 0 .. 62); each bucket sums the
+// warps' slots, which are cleared for the buffer's next step.
+__device__ __forceinline__ void bwd_flush_tables(const BwdArgs& a, const BwdStep& st, const float* diag,
+                                                 float* tslot, bool has_pos, bool has_time) {
+    if (!st.valid) return;
+    const int lane = threadIdx.x & 31;
+    if (has_pos) {
+#pragma unroll 2
+        for (int k = 0; k < 8; ++k) {
+            const int t = lane + 32 * k;
+            if (t >= 255) continue;
+            float v = 0.f;
+#pragma unroll
+            for (int ww = 0; ww < 16; ++ww) {
+                const int i = t - ((ww >> 2) * 32 - (ww & 3) * 32 + 96);
+                if (i >= 0 && i <= 62) v += diag[ww * 64 + i];
+            }
+            if (v != 0.f) {
+                const int rel = st.q0 - st.kt0 + t - 127;
+                atomicAdd(a.dpos + static_cast<int64_t>(st.h) * a.P + min(max(rel, 0), a.P - 1),
+                          v * a.inv_n);
+            }
+        }
+    }
+    if (has_time) {
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int bk = lane + 32 * k;
+            float v = 0.f;
+#pragma unroll
+            for (int ww = 0; ww < 16; ++ww) {
+                v += tslot[ww * 64 + bk];
+                tslot[ww * 64 + bk] = 0.f;
+            }
+            if (v != 0.f && bk < a.NB)
+                atomicAdd(a.dtime + static_cast<int64_t>(st.h) * a.NB + bk, v * a.inv_n);
+        }
+    }
+}
 
 template <int D>
 __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
@@ -384,13 +515,16 @@ attn_bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         mbar_init(&bars[kBwDQFull], 1);
         mbar_init(&bars[kBwDQFree], C::kPointwiseThreads);
         mbar_init(&bars[kBwAccFree], C::kPointwiseThreads);
-        mbar_init(&bars[kBwPwDone], C::kPointwiseThreads);
-        mbar_init(&bars[kBwStaged], C::kPointwiseThreads);
+        mbar_init(&bars[kBwDSFree], C::kPointwiseThreads);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bars[kBwPwDone + b], C::kPointwiseThreads);
+            mbar_init(&bars[kBwReady + b], 32);
+        }
         mbar_init(&bars[kBwDrain], 1);
         mbar_fence_init();
     }
-    for (int i = tid; i < 16 * 64; i += blockDim.x) s_diag[i] = 0.f;
-    for (int i = tid; i < 16 * 64; i += blockDim.x) s_tslot[i] = 0.f;
+    for (int i = tid; i < 2 * 16 * 64; i += blockDim.x) s_diag[i] = 0.f;
+    for (int i = tid; i < 2 * 16 * 64; i += blockDim.x) s_tslot[i] = 0.f;
     if (warp == C::kWarpMMA) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
@@ -559,79 +693,44 @@ attn_bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             if (!mbar_wait(&bars[kBwDrain], 0, nullptr)) raise_error(kErrTimeout);
         }
         __syncwarp();
+    } else if (warp == C::kWarpTable) {
+        // ------------------------------------------------------------ table warp
+        // Step m uses buffer m & 1. The first two steps are staged up front;
+        // once the pointwise threads are done with step m, its sums go into
+        // the global tables and step m + 2 is staged into the same buffer.
+        BwdCursor st, fl;
+        st.start(a, blockIdx.x, n_items);
+        fl = st;
+        for (int b = 0; b < 2; ++b) {
+            bwd_stage_tables(a, st.step(), s_posw + b * 256, s_qts + b * 128, s_cmm + b * 8,
+                             s_tb + b * 64, has_pos, has_time);
+            mbar_arrive(&bars[kBwReady + b]);
+            st.next(a, n_items);
+        }
+        for (int m = 0; fl.valid; ++m) {
+            const int b = m & 1;
+            if (!warp_wait(&bars[kBwPwDone + b], (m >> 1) & 1, abort_flag)) break;
+            bwd_flush_tables(a, fl.step(), s_diag + b * 1024, s_tslot + b * 1024, has_pos, has_time);
+            bwd_stage_tables(a, st.step(), s_posw + b * 256, s_qts + b * 128, s_cmm + b * 8,
+                             s_tb + b * 64, has_pos, has_time);
+            mbar_arrive(&bars[kBwReady + b]);
+            st.next(a, n_items);
+            fl.next(a, n_items);
+        }
+        __syncwarp();
     } else {
         // ------------------------------------------------------------ pointwise stage
         const int qd = warp & 3, cq = warp >> 2;            // TMEM lane quarter, column chunk
         const int r = qd * 32 + lane;                       // key row (S^T) / query row (dQ)
-        const int ptid = tid;                               // 0..511
         const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
         const uint32_t tS = tmem + lane_base + C::kColS, tP = tmem + lane_base + C::kColP;
         const uint32_t tV = tmem + lane_base + C::kColV, tK = tmem + lane_base + C::kColK;
         uint8_t* ds_row = smem + L::kOffDS + r * 128;
-        // the chunk's diagonal sums: entry i is tile diagonal (c - r + 127)
-        // 32 cq - 32 qd + 96 + i, i = 0 .. 62
-        float* my_diag = s_diag + warp * 64;
-        float* my_tslot = s_tslot + warp * 64;
-
-        // bias data of a step: this thread's share is loaded into registers
-        // early (pre_*) and written into shared memory later (every pointwise
-        // thread takes part in both)
-        float pre_pos = 0.f, pre_tb = 0.f;
-        long long pre_ts = 0;
-        auto stage_load = [&](const BwdStep& st) {
-            if (!st.valid) return;
-            if (has_pos && ptid < 255) {
-                const int rel = st.q0 - st.kt0 - 127 + ptid;
-                pre_pos = __ldg(a.pos + static_cast<int64_t>(st.h) * a.P + min(max(rel, 0), a.P - 1));
-            }
-            if (has_time) {
-                if (ptid < 64) pre_tb = __ldg(a.tb + static_cast<int64_t>(st.h) * a.NB + min(ptid, a.NB - 1));
-                if (ptid < 128) pre_ts = __ldg(a.ts + min(static_cast<int64_t>(st.q0) + ptid, a.T - 1));
-            }
-        };
-        auto stage_store = [&](const BwdStep& st) {
-            if (!st.valid) return;
-            if (ptid < 255) s_posw[ptid] = pre_pos;
-            if (has_time) {
-                if (ptid < 64) s_tb[ptid] = pre_tb;
-                if (ptid < 128) {
-                    s_qts[ptid] = pre_ts;
-                    long long mn = pre_ts, mx = pre_ts;
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) {
-                        mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-                        mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                    }
-                    if (lane == 0) {
-                        s_cmm[2 * warp] = mn;
-                        s_cmm[2 * warp + 1] = mx;
-                    }
-                }
-            }
-        };
-        auto step_of = [&](int w, int s) -> BwdStep {   // first step of an item only
-            BwdStep st{0, 0, 0, false};
-            if (w >= n_items) return st;
-            const BwdItem I = bwd_item(a, w);
-            if (s >= I.nq) return st;
-            st.q0 = I.qt0 + s * kTile;
-            st.kt0 = I.kt0;
-            st.h = I.h;
-            st.valid = true;
-            return st;
-        };
-        {
-            const BwdStep first = step_of(blockIdx.x, 0);
-            stage_load(first);
-            stage_store(first);
-        }
-        mbar_arrive(&bars[kBwStaged]);
 
         int n = 0;
         bool ok = true;
         for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
             const BwdItem I = bwd_item(a, w);
-            const BwdStep next_item = step_of(w + gridDim.x, 0);
             const int ktok = I.kt0 + r;
             const bool kvalid = ktok < I.key_end;
             // end (exclusive) of the sequence of key row r
@@ -642,73 +741,56 @@ attn_bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 const int q0 = I.qt0 + s * kTile;
                 const int lo = ktok - q0;                    // first kept query column
                 const int span = kvalid ? max(kend - q0 - lo, 0) : 0;   // kept: lo <= c < lo + span
-                // the next step's bias data, loaded while this one is computed
-                const BwdStep next =
-                    s + 1 < I.nq ? BwdStep{q0 + kTile, I.kt0, I.h, true} : next_item;
-                stage_load(next);
-                if (!warp_wait(&bars[kBwStaged], n & 1, abort_flag) ||
+                const int b = n & 1;                         // the step's table buffers
+                if (!warp_wait(&bars[kBwReady + b], (n >> 1) & 1, abort_flag) ||
                     !warp_wait(&bars[kBwSFull], n & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 {
+                    const float* posw = s_posw + b * 256;
+                    const long long* qts = s_qts + b * 128;
+                    const long long* cmm = s_cmm + b * 8;
+                    const float* tbrow = s_tb + b * 64;
+                    // the chunk's diagonal sums: entry i is tile diagonal (c - r + 127)
+                    // 32 cq - 32 qd + 96 + i, i = 0 .. 62
+                    float* my_diag = s_diag + b * 1024 + warp * 64;
+                    float* my_tslot = s_tslot + b * 1024 + warp * 64;
+                    const int ds_par = n > 0 ? (n - 1) & 1 : -1;
                     const int c0 = cq * 32;
                     // buckets each row sees over the chunk: b0 .. b0 + nbk - 1
                     int b0 = 0, nbk = 1;
                     if (has_time) {
-                        b0 = time_bucket_of(s_cmm[2 * cq] - tk, a.NB);
-                        nbk = time_bucket_of(s_cmm[2 * cq + 1] - tk, a.NB) - b0 + 1;
+                        b0 = time_bucket_of(cmm[2 * cq] - tk, a.NB);
+                        nbk = time_bucket_of(cmm[2 * cq + 1] - tk, a.NB) - b0 + 1;
                     }
                     const int most = __reduce_max_sync(0xffffffffu, static_cast<unsigned>(nbk));
                     uint8_t* dsr = ds_row + (c0 >> 6) * 16384;
                     const int u0 = (c0 & 63) >> 3;
+                    bool chunk_ok;
                     if (most == 1)
-                        bwd_chunk<0>(tS + c0, tP + c0, dsr, u0, c0, r, lo, span, s_posw, s_qts, s_tb,
-                                     tk, a.NB, has_time, b0, nbk, most, my_diag, my_tslot);
+                        chunk_ok = bwd_chunk<0>(tS + c0, tP + c0, dsr, u0, c0, r, lo, span, posw, qts,
+                                                tbrow, tk, a.NB, has_time, b0, nbk, most, my_diag,
+                                                my_tslot, &bars[kBwDSFree], ds_par, abort_flag);
                     else if (most <= 4)
-                        bwd_chunk<1>(tS + c0, tP + c0, dsr, u0, c0, r, lo, span, s_posw, s_qts, s_tb,
-                                     tk, a.NB, has_time, b0, nbk, most, my_diag, my_tslot);
+                        chunk_ok = bwd_chunk<1>(tS + c0, tP + c0, dsr, u0, c0, r, lo, span, posw, qts,
+                                                tbrow, tk, a.NB, has_time, b0, nbk, most, my_diag,
+                                                my_tslot, &bars[kBwDSFree], ds_par, abort_flag);
                     else
-                        bwd_chunk<2>(tS + c0, tP + c0, dsr, u0, c0, r, lo, span, s_posw, s_qts, s_tb,
-                                     tk, a.NB, has_time, b0, nbk, most, my_diag, my_tslot);
+                        chunk_ok = bwd_chunk<2>(tS + c0, tP + c0, dsr, u0, c0, r, lo, span, posw, qts,
+                                                tbrow, tk, a.NB, has_time, b0, nbk, most, my_diag,
+                                                my_tslot, &bars[kBwDSFree], ds_par, abort_flag);
+                    if (!chunk_ok) {
+                        ok = false;
+                        break;
+                    }
                 }
                 tmem_wait_st();
                 tc_fence_before();
                 fence_proxy_async_smem();
                 mbar_arrive(&bars[kBwPFull]);
-                // every thread is done with this step's staged data and sums:
-                // flush the sums, clear them, stage the next step
-                mbar_arrive(&bars[kBwPwDone]);
-                if (!warp_wait(&bars[kBwPwDone], n & 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                if (has_pos && ptid < 255) {
-                    float v = 0.f;
-#pragma unroll
-                    for (int ww = 0; ww < 16; ++ww) {
-                        const int i = ptid - ((ww >> 2) * 32 - (ww & 3) * 32 + 96);
-                        if (i >= 0 && i <= 62) v += s_diag[ww * 64 + i];
-                    }
-                    if (v != 0.f) {
-                        const int rel = q0 - I.kt0 + ptid - 127;
-                        atomicAdd(a.dpos + static_cast<int64_t>(I.h) * a.P + min(max(rel, 0), a.P - 1),
-                                  v * a.inv_n);
-                    }
-                }
-                if (has_time && ptid < 64) {
-                    float v = 0.f;
-#pragma unroll
-                    for (int ww = 0; ww < 16; ++ww) {
-                        v += s_tslot[ww * 64 + ptid];
-                        s_tslot[ww * 64 + ptid] = 0.f;
-                    }
-                    if (v != 0.f && ptid < a.NB)
-                        atomicAdd(a.dtime + static_cast<int64_t>(I.h) * a.NB + ptid, v * a.inv_n);
-                }
-                stage_store(next);
-                mbar_arrive(&bars[kBwStaged]);
+                mbar_arrive(&bars[kBwPwDone + b]);
                 // dQ_i of the step into dq
                 if (!warp_wait(&bars[kBwDQFull], n & 1, abort_flag)) {
                     ok = false;
@@ -716,16 +798,22 @@ attn_bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 }
                 tc_fence_after();
                 {
-                    // dQ_i rows through the dS^T buffer (its MMAs have completed):
-                    // each warp stages 32 x 16 fp32 blocks (64-byte swizzle) of its
-                    // D/4 columns and adds them into dq with a bulk tensor
-                    // reduction; rows of queries outside the sequence are zero
+                    // this warp's D/4 columns of dQ_i leave TMEM first, so the
+                    // next dP^T can be computed there; then they go through the
+                    // dS^T buffer (its MMAs have completed) as 32 x 16 fp32
+                    // blocks (64-byte swizzle), added into dq with bulk tensor
+                    // reductions; rows of queries outside the sequence are zero
                     // (every ds of theirs is)
+                    uint32_t v[D / 64][16];
+                    if constexpr (D == 128)
+                        tmem_ld16x2(tP + cq * 32, tP + cq * 32 + 16, v[0], v[1]);
+                    else
+                        tmem_ld16(tP + cq * 16, v[0]);
+                    tc_fence_before();
+                    mbar_arrive(&bars[kBwDQFree]);
                     uint8_t* buf = smem + L::kOffDS + warp * 2048;
-#pragma unroll 1
+#pragma unroll
                     for (int cb = 0; cb < D / 64; ++cb) {
-                        uint32_t v[16];
-                        tmem_ld16(tP + cq * (D / 4) + cb * 16, v);
                         if (cb > 0) {
                             if (lane == 0) bulk_wait_group_read<0>();
                             __syncwarp();
@@ -733,10 +821,10 @@ attn_bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
 #pragma unroll
                         for (int u = 0; u < 4; ++u)
                             *reinterpret_cast<float4*>(buf + lane * 64 + ((u ^ ((lane >> 1) & 3)) << 4)) =
-                                make_float4(__uint_as_float(v[4 * u]) * a.inv_n,
-                                            __uint_as_float(v[4 * u + 1]) * a.inv_n,
-                                            __uint_as_float(v[4 * u + 2]) * a.inv_n,
-                                            __uint_as_float(v[4 * u + 3]) * a.inv_n);
+                                make_float4(__uint_as_float(v[cb][4 * u]) * a.inv_n,
+                                            __uint_as_float(v[cb][4 * u + 1]) * a.inv_n,
+                                            __uint_as_float(v[cb][4 * u + 2]) * a.inv_n,
+                                            __uint_as_float(v[cb][4 * u + 3]) * a.inv_n);
                         fence_proxy_async_smem();
                         __syncwarp();
                         if (lane == 0) {
@@ -746,9 +834,8 @@ attn_bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     }
                     if (lane == 0) bulk_wait_group_read<0>();
                     __syncwarp();
+                    mbar_arrive(&bars[kBwDSFree]);
                 }
-                tc_fence_before();
-                mbar_arrive(&bars[kBwDQFree]);
                 if (s == I.nq - 1) {
                     // the item's dV_j and dK_j (their MMAs completed before dQ's)
                     const int64_t row = (static_cast<int64_t>(ktok) * a.H + I.h) * D + cq * (D / 4);
