@@ -9,10 +9,13 @@
 //     dq_i = sum_j ds_ij k_j,  dk_j = sum_i ds_ij q_i
 //     dpos[min(i - j, P - 1)] and dtime[bucket(ts_i - ts_j)] sum the ds of their pairs.
 //
-// Persistent kernel over work items (key tile j, head h), static round robin
-// over the forward plan's longest-first list: the plan unit of query tile t
-// (t + 1 key tiles) maps to key tile nt - 1 - t (t + 1 query tiles), so the
-// items with the most query tiles still come first. Key tile K_j and V_j stay
+// Persistent kernel over work items (key tile j, head h): the plan unit of
+// query tile t (t + 1 key tiles) maps to key tile nt - 1 - t, whose item walks
+// t + 1 query tiles. The items are sorted by that count, most first, and dealt
+// to the CTAs in a snake (the order of turns reverses every round), which
+// leaves every CTA within about one item of the mean; a plain round robin
+// over the plan's list, where each sequence's items fall from nt steps to 1,
+// gave some CTAs half again the mean on long batches. Key tile K_j and V_j stay
 // in shared memory while the item walks its query tiles i = j .. nt - 1; Q_i
 // streams through a two-stage TMA ring, dO_i through a two-stage ring (d = 64)
 // or a single buffer (d = 128, for shared memory), reloaded as soon as its
@@ -86,6 +89,8 @@ struct BwdArgs {
     float* dv;                  // [T, H, D] fp32: written
     float* dpos;                // [H, P]: zeroed before, accumulated (with pos)
     float* dtime;               // [H, NB]: zeroed before, accumulated (with the time term)
+    const int* order;           // plan: item-order table, four rows of max_tiles + 2 ints
+    int max_tiles;
 };
 
 template <int D>
@@ -184,6 +189,49 @@ __device__ __forceinline__ BwdItem bwd_item(const BwdArgs& a, int w) {
         it.nq = nk;
     }
     return it;
+}
+
+// The item of a CTA's k-th turn, or -1 past the last. Items are taken in
+// order of cost, most steps first (nq = nk of the unit: c steps for the
+// aligned items of cost c, ranked by sequence, then head; then the packed
+// items, one step each, in list order), and dealt to the CTAs in a snake:
+// turn k takes position k G + b for even k, k G + G - 1 - b for odd k. The
+// plan's table gives, per cost v, the sequences with nt >= v (sge), the
+// aligned items of cost >= v (ige), the first unit (cum) and rank (base) of
+// the sequences with nt == v.
+__device__ __forceinline__ int bwd_item_index(const BwdArgs& a, int k, int n_items) {
+    const int G = gridDim.x, b = blockIdx.x;
+    const int64_t p64 = static_cast<int64_t>(k) * G + ((k & 1) ? G - 1 - b : b);
+    if (p64 >= n_items) return -1;
+    const int p = static_cast<int>(p64);
+    const int stride = a.max_tiles + 2;
+    const int* sge = a.order;
+    const int* ige = a.order + stride;
+    const int* cum = a.order + 2 * stride;
+    const int* base = a.order + 3 * stride;
+    if (p >= __ldg(ige + 1)) return p;               // packed: list order
+    // cost c: ige[c] > p >= ige[c + 1]
+    int lo = 1, hi = a.max_tiles;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (__ldg(ige + mid) > p) lo = mid;
+        else hi = mid - 1;
+    }
+    const int c = lo;
+    const int idx = p - __ldg(ige + c + 1);
+    const int rho = idx / a.H, h = idx - rho * a.H;
+    // tile count v of the sequence of rank rho: sge[v] > rho >= sge[v + 1]
+    lo = c;
+    hi = a.max_tiles;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (__ldg(sge + mid) > rho) lo = mid;
+        else hi = mid - 1;
+    }
+    const int v = lo;
+    const int ubase = __ldg(cum + v) + (rho - __ldg(base + v)) * v;
+    const int w = a.H * ubase + h * v + (v - c);     // the unit with nk = c, head h
+    return w < n_items ? w : -1;
 }
 
 // Smallest row p > r of a packed tile at which a sequence begins (bit p of
@@ -360,22 +408,23 @@ struct BwdStep {
     bool valid;
 };
 
-// Walks a CTA's steps in order: its items w = blockIdx.x, + gridDim.x, ...,
-// each over its query tiles.
+// Walks a CTA's steps in order: the items of its turns k = 0, 1, ..., each
+// over its query tiles.
 struct BwdCursor {
-    int w, s;
+    int k, s;
     BwdItem I;
     bool valid;
-    __device__ __forceinline__ void start(const BwdArgs& a, int w0, int n_items) {
-        w = w0;
+    __device__ __forceinline__ void start(const BwdArgs& a, int k0, int n_items) {
+        k = k0;
         s = 0;
-        valid = w < n_items;
+        const int w = bwd_item_index(a, k, n_items);
+        valid = w >= 0;
         if (valid) I = bwd_item(a, w);
     }
     __device__ __forceinline__ void next(const BwdArgs& a, int n_items) {
         if (!valid) return;
         if (++s < I.nq) return;
-        start(a, w + gridDim.x, n_items);
+        start(a, k + 1, n_items);
     }
     __device__ __forceinline__ BwdStep step() const {
         return BwdStep{valid ? I.qt0 + s * kTile : 0, valid ? I.kt0 : 0, valid ? I.h : 0, valid};
@@ -543,7 +592,7 @@ attn_bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             tma_prefetch_desc(&tmV);
             tma_prefetch_desc(&tmDO);
             bool ok = true;
-            for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
+            for (int k = 0, w; ok && (w = bwd_item_index(a, k, n_items)) >= 0; ++k) {
                 const BwdItem I = bwd_item(a, w);
                 if (kv_loads > 0 && !mbar_wait(&bars[kBwKVFree], (kv_loads - 1) & 1, abort_flag)) {
                     ok = false;
@@ -614,7 +663,7 @@ attn_bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             const uint64_t dS_k = desc_kmajor_sw128(sDS), dS_mn = desc_mnmajor_sw128(sDS, 16384);
             int nitem = 0, n = 0;
             bool ok = true;
-            for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x, ++nitem) {
+            for (int w; ok && (w = bwd_item_index(a, nitem, n_items)) >= 0; ++nitem) {
                 const BwdItem I = bwd_item(a, w);
                 if (!mbar_wait(&bars[kBwKVFull], nitem & 1, abort_flag)) {
                     ok = false;
@@ -699,7 +748,7 @@ attn_bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         // once the pointwise threads are done with step m, its sums go into
         // the global tables and step m + 2 is staged into the same buffer.
         BwdCursor st, fl;
-        st.start(a, blockIdx.x, n_items);
+        st.start(a, 0, n_items);
         fl = st;
         for (int b = 0; b < 2; ++b) {
             bwd_stage_tables(a, st.step(), s_posw + b * 256, s_qts + b * 128, s_cmm + b * 8,
@@ -729,7 +778,7 @@ attn_bwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
 
         int n = 0;
         bool ok = true;
-        for (int w = blockIdx.x; ok && w < n_items; w += gridDim.x) {
+        for (int k = 0, w; ok && (w = bwd_item_index(a, k, n_items)) >= 0; ++k) {
             const BwdItem I = bwd_item(a, w);
             const int ktok = I.kt0 + r;
             const bool kvalid = ktok < I.key_end;

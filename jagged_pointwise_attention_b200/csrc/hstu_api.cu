@@ -271,9 +271,10 @@ hstu_status_t launch_attn_pdl(Kernel kernel, unsigned grid, int threads, size_t 
     return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
 }
 
-// The plan kernel: the longest-first work list into the workspace's plan part.
+// The plan kernel: the longest-first work list into the workspace's plan part
+// (and, for the backward, its item-order table: order_h = H).
 hstu_status_t launch_plan(const int64_t* off, int32_t B, int64_t T, int32_t max_seqlen, void* ws,
-                          cudaStream_t stream) {
+                          cudaStream_t stream, int order_h = 0, int* order_tab = nullptr) {
     const int max_tiles = max_tiles_of(max_seqlen);
     const int64_t max_units = max_units_of(B, T, max_seqlen);
     uint8_t* w = static_cast<uint8_t*>(ws);
@@ -283,7 +284,7 @@ hstu_status_t launch_plan(const int64_t* off, int32_t B, int64_t T, int32_t max_
         off, B, T, max_seqlen, max_tiles, static_cast<int>(max_units),
         reinterpret_cast<int4*>(w + kAttnWsHeader),
         reinterpret_cast<uint4*>(w + kAttnWsHeader + attn_units_bytes(B, T, max_seqlen)),
-        reinterpret_cast<int*>(w), reinterpret_cast<int*>(w + 16));
+        reinterpret_cast<int*>(w), reinterpret_cast<int*>(w + 16), order_h, order_tab);
     return launch_status();
 }
 
@@ -737,9 +738,15 @@ hstu_status_t hstu_attn_bwd_f32(const float* q, const float* k, const float* v, 
     return launch_status();
 }
 
+// backward workspace: the plan's part, then its item-order table (four rows
+// of max_tiles + 2 ints)
+size_t attn_order_bytes(int32_t max_seqlen) {
+    return round_up(static_cast<size_t>(4) * (max_tiles_of(max_seqlen) + 2) * sizeof(int), 256);
+}
+
 size_t hstu_attn_bwd_workspace_bytes(int32_t B, int64_t total_tokens, int32_t max_seqlen) {
     if (!plan_sizes_ok(B, total_tokens, max_seqlen)) return 0;
-    return attn_plan_bytes(B, total_tokens, max_seqlen);
+    return attn_plan_bytes(B, total_tokens, max_seqlen) + attn_order_bytes(max_seqlen);
 }
 
 hstu_status_t hstu_attn_bwd(hstu_dtype_t dtype, const void* q, int64_t q_stride, const void* k,
@@ -776,10 +783,13 @@ hstu_status_t hstu_attn_bwd(hstu_dtype_t dtype, const void* q, int64_t q_stride,
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq) ||
         !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
         return HSTU_ERR_INVALID_ARG;
-    if (workspace_bytes < attn_plan_bytes(B, T, max_seqlen)) return HSTU_ERR_INVALID_ARG;
+    if (workspace_bytes < attn_plan_bytes(B, T, max_seqlen) + attn_order_bytes(max_seqlen))
+        return HSTU_ERR_INVALID_ARG;
     if (cudaMemsetAsync(dq, 0, static_cast<size_t>(T) * row * sizeof(float), s) != cudaSuccess)
         return HSTU_ERR_CUDA;
-    hstu_status_t st = launch_plan(seq_offsets, B, T, max_seqlen, workspace, s);
+    int* order_tab = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) +
+                                            attn_plan_bytes(B, T, max_seqlen));
+    hstu_status_t st = launch_plan(seq_offsets, B, T, max_seqlen, workspace, s, H, order_tab);
     if (st != HSTU_OK) return st;
     CUtensorMap tq, tk, tv, tdo, tdq;
     if (!make_tmap_bf16(&tq, q, row, T, q_stride * 2, 128) ||
@@ -795,7 +805,7 @@ hstu_status_t hstu_attn_bwd(hstu_dtype_t dtype, const void* q, int64_t q_stride,
               H, T, use_time ? timestamps : nullptr, pos_bias, P > 0 ? P : 1,
               use_time ? time_bias : nullptr, NB > 0 ? NB : 1,
               1.0f / static_cast<float>(max_seqlen), dq, dk, dv, pos_bias ? dpos : nullptr,
-              use_time ? dtime : nullptr};
+              use_time ? dtime : nullptr, order_tab, max_tiles_of(max_seqlen)};
     const unsigned grid = static_cast<unsigned>(num_sms());
     if (d == 64) {
         static int done[kMaxDevices] = {0};

@@ -24,6 +24,13 @@
 // sorted by their tile count nt (descending); a sequence of rank rho in the
 // bucket of count v starts at unit cum[v] + (rho - base[v]) * v, cum[v]
 // counting the units of all longer buckets.
+//
+// On request (order_tab non-null) the plan also writes the table from which
+// the attention backward orders its work items by cost: for v = 1 ..
+// max_tiles, in four rows of max_tiles + 2 ints, the number of sequences
+// with nt >= v; the number of items (order_h per unit, one per head) of
+// aligned units with nk >= v; cum[v]; base[v]. Entry max_tiles + 1 of the
+// first two rows is 0.
 #pragma once
 
 #include "common.cuh"
@@ -42,7 +49,8 @@ __device__ __forceinline__ void plan_body(const int64_t* __restrict__ seq_offset
                                           int max_seqlen, int max_tiles, int max_units,
                                           int4* __restrict__ units, uint4* __restrict__ starts,
                                           int* __restrict__ unit_count,
-                                          int* __restrict__ item_counter, int* plan_smem) {
+                                          int* __restrict__ item_counter, int* plan_smem,
+                                          int order_h, int* __restrict__ order_tab) {
     const int NT = max_tiles + 1;        // tile counts 0..max_tiles
     int* cnt = plan_smem;                // sequences with nt == v
     int* base = cnt + NT;                // first rank of nt == v in the descending order
@@ -167,22 +175,42 @@ __device__ __forceinline__ void plan_body(const int64_t* __restrict__ seq_offset
         const int total = n_aligned + n_packed;
         *unit_count = total < max_units ? total : max_units;
     }
+    if (order_tab != nullptr && tid == 0) {
+        // cnt[v] counts the sequences placed in bucket v again
+        const int stride = max_tiles + 2;
+        int items = 0;
+        order_tab[max_tiles + 1] = 0;
+        order_tab[stride + max_tiles + 1] = 0;
+        for (int v = max_tiles; v >= 1; --v) {
+            const int seqs = base[v] + cnt[v];
+            items += order_h * seqs;
+            order_tab[v] = seqs;
+            order_tab[stride + v] = items;
+            order_tab[2 * stride + v] = cum[v];
+            order_tab[3 * stride + v] = base[v];
+        }
+        order_tab[0] = order_tab[1];
+        order_tab[stride] = items;
+        order_tab[2 * stride] = n_aligned;
+        order_tab[3 * stride] = order_tab[1];
+    }
 }
 
 __global__ void __launch_bounds__(1024)
 plan_kernel(const int64_t* __restrict__ seq_offsets, int B, int64_t T, int max_seqlen,
             int max_tiles, int max_units, int4* __restrict__ units, uint4* __restrict__ starts,
-            int* __restrict__ unit_count, int* __restrict__ item_counter) {
+            int* __restrict__ unit_count, int* __restrict__ item_counter, int order_h,
+            int* __restrict__ order_tab) {
     extern __shared__ int plan_smem[];
     // let the attention kernel that follows start its set-up now (it waits
     // for this grid to complete before it reads the work list)
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (B < kPlanSmemOffsets)
         plan_body<true>(seq_offsets, B, T, max_seqlen, max_tiles, max_units, units, starts,
-                        unit_count, item_counter, plan_smem);
+                        unit_count, item_counter, plan_smem, order_h, order_tab);
     else
         plan_body<false>(seq_offsets, B, T, max_seqlen, max_tiles, max_units, units, starts,
-                         unit_count, item_counter, plan_smem);
+                         unit_count, item_counter, plan_smem, order_h, order_tab);
 }
 
 }  // namespace hstu
