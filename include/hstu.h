@@ -383,8 +383,10 @@ hstu_status_t hstu_attn_bwd_f32(const float* q, const float* k, const float* v, 
  * in bf16, sums in fp32; table gradients and dq are accumulated with
  * atomics, so their last bits may differ between runs. `workspace` (device,
  * 16-byte aligned, hstu_attn_bwd_workspace_bytes(B, T, max_seqlen) bytes)
- * holds the work list; one plan launch, one backward launch, and the
- * clears. Other arguments as hstu_attn_fwd. Asynchronous on `stream`. */
+ * holds the work list and the order in which the CTAs take its items (most
+ * query tiles first, dealt in a snake so every CTA gets about the same
+ * number of steps); one plan launch, one backward launch, and the clears.
+ * Other arguments as hstu_attn_fwd. Asynchronous on `stream`. */
 size_t hstu_attn_bwd_workspace_bytes(int32_t B, int64_t total_tokens, int32_t max_seqlen);
 hstu_status_t hstu_attn_bwd(hstu_dtype_t dtype, const void* q, int64_t q_stride, const void* k,
                             int64_t k_stride, const void* v, int64_t v_stride, const void* dout,
